@@ -1,0 +1,388 @@
+"""Benchmark of the multi-precision BCQ GEMV on B200.
+
+Workload: one BCQ weight of the Llama-3.1-8B MLP gate/up shape
+(N = 14336 outputs, K = 4096 inputs, group 128, p_H = 4 stored planes) with
+synthetic seeded data (bit_gemv_bcq_b200/synth.py).  One step is one call for
+every precision p in {2, 3, 4} and batch M in {1, 2, 4, 8, 16}: 15 calls.
+Metric: achieved HBM throughput in GB/s over the algorithmic bytes
+    N*K*p/8 (planes) + N*G*p*2 (scales) + N*G*2 (offsets) + M*K*2 (x) + M*N*2 (y)
+of every call, with microseconds per call reported per (p, M).
+
+Timing: CUDA graphs (one per step, 15 calls) replayed back to back; R
+rotating copies of the weights (> 2x L2 in total) so every call streams from
+HBM; CUDA events on the launching stream; W warm-up steps; clocks sampled
+with nvidia-smi during the timed region.  ``e2e`` measures the same calls
+through the C entry point with host buffers (bcq_gemm_host), copies included.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload on the host cores.  With torchrun (N > 1 GPUs) every rank runs
+an independent replica (no collective on the data path), the timed region is
+bracketed by barriers and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_OUT, K_IN, GROUP, P_H = 14336, 4096, 128, 4
+PRECISIONS = (2, 3, 4)
+BATCHES = (1, 2, 4, 8, 16)
+METRIC = "BCQ GEMV µs & HBM GB/s (% of B200 peak) at p=2/3/4, M=1..16, 14336×4096"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algo_bytes(N, K, M, p):
+    G = K // GROUP
+    return N * K * p // 8 + N * G * p * 2 + N * G * 2 + M * K * 2 + M * N * 2
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, maxs, reasons, powers = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                    powers.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "samples": len(sms), "power_w_max": max(powers) if powers else None,
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from bit_gemv_bcq_b200 import api, synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
+    base = api.BcqWeights.from_canonical(prob.planes, prob.alphas, prob.z, device=dev)
+    per_copy = base.packed.numel() * 4 + sum(a.numel() * 2 for a in base.alphas.values()) \
+        + base.z.numel() * 2
+    R = max(2, math.ceil(2 * L2_BYTES / per_copy) + 1)
+    copies = [base] + [api.BcqWeights(packed=base.packed.clone(),
+                                      alphas={q: a.clone() for q, a in base.alphas.items()},
+                                      z=base.z.clone(), N=base.N, K=base.K, p_H=base.p_H)
+                       for _ in range(R - 1)]
+    x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).to(dev)
+    ys = {M: torch.empty((M, N_OUT), dtype=torch.float16, device=dev) for M in BATCHES}
+    cases = [(p, M) for p in PRECISIONS for M in BATCHES]
+    bytes_step = sum(algo_bytes(N_OUT, K_IN, M, p) for p, M in cases)
+    launches_per_step = sum(math.ceil(M / 4) for _, M in cases)
+
+    stream = torch.cuda.Stream(device=dev)
+    # eager pass: plans and caches every launch shape before capture
+    with torch.cuda.stream(stream):
+        for w in copies[:1]:
+            for p, M in cases:
+                w.gemm(x[:M], p=p, out=ys[M], stream=stream)
+    stream.synchronize()
+    assert api.device_error(stream) == api.BCQ_OK
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
+    step_graphs = []
+    for r in range(R):
+        def step(r=r):
+            for i, (p, M) in enumerate(cases):
+                copies[(r + i) % R].gemm(x[:M], p=p, out=ys[M], stream=stream)
+        step_graphs.append(capture(step))
+
+    # per-call timing of each case: R calls (one per copy) per replay
+    case_graphs = {}
+    for p, M in cases:
+        def one(p=p, M=M):
+            for w in copies:
+                w.gemm(x[:M], p=p, out=ys[M], stream=stream)
+        case_graphs[(p, M)] = capture(one)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            step_graphs[k % R].replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for k in range(args.steps):
+            step_graphs[k % R].replay()
+        t1.record(stream)
+    t1.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    clocks = sampler.stop()
+    err = api.device_error(stream)
+    if err != api.BCQ_OK:
+        raise RuntimeError(f"device error {api.status_string(err)}")
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # per-case microseconds (same stream, events around each replay)
+    per_case = []
+    reps = max(3, min(50, args.steps // 20))
+    for p, M in cases:
+        g = case_graphs[(p, M)]
+        with torch.cuda.stream(stream):
+            g.replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+        b.synchronize()
+        us = a.elapsed_time(b) * 1000.0 / (reps * R)
+        by = algo_bytes(N_OUT, K_IN, M, p)
+        per_case.append({"p": p, "M": M, "us": round(us, 3), "bytes": by,
+                         "GBps": round(by / us / 1e3, 1)})
+
+    result = {"ms_total": ms_total, "bytes_step": bytes_step, "R": R,
+              "per_copy_bytes": per_copy, "launches_per_step": launches_per_step,
+              "per_case": per_case, "clocks": clocks}
+
+    # end to end through bcq_gemm_host: pinned host x and y, copies inside
+    if not args.profile:
+        x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).pin_memory()
+        y_host = {M: torch.empty((M, N_OUT), dtype=torch.float16).pin_memory() for M in BATCHES}
+        x_dev = torch.empty_like(x)
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        h2d = sum(M * K_IN * 2 for _, M in cases)
+        d2h = sum(M * N_OUT * 2 for _, M in cases)
+        for k in range(2):
+            for i, (p, M) in enumerate(cases):
+                api.gemm_host(x_host[:M], copies[(k + i) % R], y_host[M], x_dev[:M], ys[M],
+                              p=p, stream=stream)
+        stream.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for k in range(e2e_steps):
+            for i, (p, M) in enumerate(cases):
+                api.gemm_host(x_host[:M], copies[(k + i) % R], y_host[M], x_dev[:M], ys[M],
+                              p=p, stream=stream)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        result["e2e"] = {"ms": e2e_ms, "steps": e2e_steps, "h2d": h2d, "d2h": d2h}
+    return result
+
+
+# ------------------------------------------------------------- CPU oracle arm
+
+def run_oracle_sample(seed, rows_per_call, prob=None):
+    """The fp64 oracle on a bounded sample: `rows_per_call` output rows of each
+    of the 15 calls.  Returns (seconds, algorithmic bytes of the sample, threads)."""
+    import oracle
+    from bit_gemv_bcq_b200 import synth
+    if prob is None:
+        prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=seed)
+    rng = np.random.default_rng(seed + 1)
+    rows = np.sort(rng.choice(N_OUT, rows_per_call, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    for p in PRECISIONS:
+        for M in BATCHES:
+            oracle.gemm(prob.x[:M], prob.planes, prob.alphas, prob.z, p=p, rows=rows)
+    dt = time.perf_counter() - t0
+    frac = rows_per_call / N_OUT
+    by = sum(algo_bytes(N_OUT, K_IN, M, p) for p in PRECISIONS for M in BATCHES) * frac
+    return dt, by, oracle.num_threads()
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="bcq", choices=["bcq", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-rows", type=int, default=14336,
+                    help="output rows per call in the oracle's timed sample")
+    ap.add_argument("--profile", action="store_true",
+                    help="GPU timing only (no e2e or CPU legs), for profiler runs")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps = max(1, args.steps)
+        # each step: the oracle on a bounded sample of one step of the workload
+        rows = max(16, min(args.cpu_rows, 2048))
+        from bit_gemv_bcq_b200 import synth
+        prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
+        n_steps = min(steps, 5)
+        secs, by, thr = 0.0, 0.0, 1
+        for k in range(n_steps):
+            s, b, thr = run_oracle_sample(args.seed + k, rows, prob)
+            secs += s
+            by += b
+        gbps = by / secs / 1e9
+        line = {"metric": METRIC, "value": round(gbps, 4), "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": n_steps, "warmup": 0, "ms_per_step": round(secs / n_steps * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": "bcq_gemv N=14336 K=4096 g=128 p_H=4; p in {2,3,4} x "
+                                       "M in {1,2,4,8,16}", "parallelism": "single process, host cores"},
+                "cpu_baseline": {"value": round(gbps, 4), "unit": "GB/s", "cores": thr,
+                                 "kind": "oracle",
+                                 "sample": f"{rows} of {N_OUT} output rows of each of the 15 calls per step"},
+                "e2e": {"value": round(gbps, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = run_gpu(args, rank, world, local_rank)
+
+    peak, peak_kind = measured_peaks()
+    ms_step = res["ms_total"] / args.steps
+    value = world * res["bytes_step"] / (ms_step * 1e-3) / 1e9
+    achieved_per_gpu = res["bytes_step"] / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "bcq_gemv N=14336 K=4096 g=128 p_H=4; one step = one call per "
+                               "p in {2,3,4} x M in {1,2,4,8,16} (15 calls), fp16 x/y/scales",
+                   "l2": f"inputs larger than L2: {res['R']} rotating weight copies of "
+                         f"{res['per_copy_bytes'] / 2**20:.1f} MiB",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "timing": "CUDA graph per step, CUDA events on the launching stream"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
+                     "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "gemv_lut_kernel (every launch of the step)"},
+        "per_call": res["per_case"],
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "clocks": res["clocks"],
+    }
+    m1 = [c for c in res["per_case"] if c["M"] == 1]
+    line["headline_m1"] = {f"p{c['p']}": {"us": c["us"], "GBps": c["GBps"],
+                                          "frac": round(c["GBps"] / peak, 4)} for c in m1}
+    if "e2e" in res:
+        e = res["e2e"]
+        line["e2e"] = {"value": round(world * res["bytes_step"] * e["steps"] / (e["ms"] * 1e-3) / 1e9, 2),
+                       "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "ms_per_step": round(e["ms"] / e["steps"], 4),
+                       "path": "bcq_gemm_host (pinned host x/y, copies on the stream)"}
+    if rank == 0 and world == 1 and not args.profile:
+        secs, by, thr = run_oracle_sample(args.seed, args.cpu_rows)
+        line["cpu_baseline"] = {"value": round(by / secs / 1e9, 4), "unit": "GB/s", "cores": thr,
+                                "kind": "oracle",
+                                "sample": f"{args.cpu_rows} of {N_OUT} output rows of each of the "
+                                          f"15 calls ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

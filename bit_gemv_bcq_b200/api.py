@@ -1,0 +1,247 @@
+"""Thin Python binding of libbcq (include/bcq.h).
+
+Argument marshalling only: torch CUDA tensors become raw pointers, the
+current torch stream becomes the CUDA stream, and every step of the matmul
+runs in the library's kernels.  There is no CPU fallback: a missing
+``libbcq.so`` raises ``BcqLibraryError`` on first use.
+
+The same names as the C ABI: ``pack_planes``, ``gemm``, ``gemm_host``,
+``build_lut``, ``device_error``, ``debug_wait_timeout``; ``BcqWeights`` bundles
+the packed planes with their scales and offsets.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbcq.so")
+
+BCQ_OK = 0
+BCQ_ERR_NULL = 1
+BCQ_ERR_SHAPE = 2
+BCQ_ERR_PRECISION = 3
+BCQ_ERR_ALIGN = 4
+BCQ_ERR_CUDA = 5
+BCQ_ERR_TIMEOUT = 6
+BCQ_ERR_UNSUPPORTED = 7
+GROUP = 128
+MAX_M = 64
+
+_lib = None
+
+
+class BcqLibraryError(RuntimeError):
+    pass
+
+
+class BcqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib():
+    """Load libbcq.so (built in-tree by bit_gemv_bcq_b200/build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise BcqLibraryError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python bit_gemv_bcq_b200/build.py` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.bcq_status_string.restype = ctypes.c_char_p
+        L.bcq_status_string.argtypes = [I]
+        L.bcq_version.restype = I
+        L.bcq_version.argtypes = []
+        L.bcq_packed_planes_bytes.restype = S
+        L.bcq_packed_planes_bytes.argtypes = [I, I, I]
+        L.bcq_pack_planes.restype = I
+        L.bcq_pack_planes.argtypes = [P, P, I, I, I, P]
+        L.bcq_gemm.restype = I
+        L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
+        L.bcq_gemm_host.restype = I
+        L.bcq_gemm_host.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, P, P]
+        L.bcq_build_lut.restype = I
+        L.bcq_build_lut.argtypes = [P, I, I, P, P, P]
+        L.bcq_device_error.restype = I
+        L.bcq_device_error.argtypes = [P]
+        L.bcq_debug_wait_timeout.restype = I
+        L.bcq_debug_wait_timeout.argtypes = [I, P]
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
+            "bcq_pack_planes", "bcq_gemm", "bcq_gemm_host", "bcq_build_lut",
+            "bcq_device_error", "bcq_debug_wait_timeout")
+
+
+def status_string(status: int) -> str:
+    return lib().bcq_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != BCQ_OK:
+        raise BcqError(status, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _alpha_array(alphas: dict):
+    arr = (ctypes.c_void_p * 4)()
+    for q in range(1, 5):
+        a = alphas.get(q) if alphas else None
+        if a is not None:
+            _need_cuda(a, f"alpha[{q}]", torch.float16)
+            arr[q - 1] = a.data_ptr()
+        else:
+            arr[q - 1] = None
+    return arr
+
+
+def packed_planes_bytes(p_H: int, N: int, K: int) -> int:
+    return int(lib().bcq_packed_planes_bytes(p_H, N, K))
+
+
+def pack_planes(planes_canon: torch.Tensor, stream=None) -> torch.Tensor:
+    """Canonical planes (int32/uint32 CUDA tensor [p_H][N][K/32], LSB-first
+    bits, 1 = +1) -> packed streaming layout (int32 CUDA tensor)."""
+    _need_cuda(planes_canon, "planes")
+    if planes_canon.element_size() != 4 or planes_canon.dim() != 3:
+        raise ValueError("planes must be a 32-bit [p_H][N][K/32] tensor")
+    p_H, N, KW = planes_canon.shape
+    K = KW * 32
+    nbytes = packed_planes_bytes(p_H, N, K)
+    if nbytes == 0:
+        raise BcqError(BCQ_ERR_SHAPE, "bcq_packed_planes_bytes")
+    out = torch.empty(nbytes // 4, dtype=torch.int32, device=planes_canon.device)
+    _check(lib().bcq_pack_planes(_ptr(planes_canon), _ptr(out), p_H, N, K,
+                                 _stream(stream)), "bcq_pack_planes")
+    return out
+
+
+@dataclass
+class BcqWeights:
+    """One BCQ weight matrix on the device: packed +-1 planes shared by every
+    precision, the scales alpha^(q) of each precision q, and the offset z."""
+    packed: torch.Tensor        # int32, library layout
+    alphas: dict                # {q: fp16 [N][G][q]}
+    z: torch.Tensor | None      # fp16 [N][G] or None
+    N: int
+    K: int
+    p_H: int
+
+    @classmethod
+    def from_canonical(cls, planes, alphas: dict, z=None, device="cuda", stream=None):
+        """planes: uint32 [p_H][N][K/32] (numpy or tensor); alphas {q: fp16
+        [N][G][q]}; z fp16 [N][G] or None."""
+        if isinstance(planes, np.ndarray):
+            planes = torch.from_numpy(np.ascontiguousarray(planes).view(np.int32))
+        planes = planes.to(device).contiguous()
+        p_H, N, KW = planes.shape
+        packed = pack_planes(planes, stream)
+        al = {}
+        for q, a in alphas.items():
+            a = torch.as_tensor(a) if isinstance(a, np.ndarray) else a
+            al[int(q)] = a.to(device=device, dtype=torch.float16).contiguous()
+        zz = None
+        if z is not None:
+            zz = (torch.as_tensor(z) if isinstance(z, np.ndarray) else z)
+            zz = zz.to(device=device, dtype=torch.float16).contiguous()
+        return cls(packed=packed, alphas=al, z=zz, N=N, K=KW * 32, p_H=p_H)
+
+    def gemm(self, x, p=None, p_row=None, out=None, stream=None):
+        return gemm(x, self, p=p, p_row=p_row, out=out, stream=stream)
+
+
+def _prec_args(p, p_row, M):
+    if (p is None) == (p_row is None):
+        raise ValueError("give exactly one of p and p_row")
+    if p is not None:
+        return int(p), None, None
+    pr = np.ascontiguousarray(np.asarray(p_row, dtype=np.int32))
+    if pr.shape != (M,):
+        raise ValueError("p_row must have one entry per row of x")
+    return 0, pr, pr.ctypes.data_as(ctypes.c_void_p)
+
+
+def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
+         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x . W_hat^T (fp16 [M][N]) with uniform precision p or per-row p_row."""
+    _need_cuda(x, "x", torch.float16)
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M][{w.K}]")
+    M = x.shape[0]
+    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.float16, device=x.device)
+    else:
+        _need_cuda(out, "out", torch.float16)
+    alpha = _alpha_array(w.alphas)
+    st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                        _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                        _ptr(out), _stream(stream))
+    _check(st, "bcq_gemm")
+    del pr_keep
+    return out
+
+
+def gemm_host(x_host: torch.Tensor, w: BcqWeights, y_host: torch.Tensor,
+              x_dev: torch.Tensor, y_dev: torch.Tensor, p: int | None = None,
+              p_row=None, stream=None) -> None:
+    """bcq_gemm_host: x and y in (pinned) host memory, copies on the stream.
+    The caller synchronises the stream before reading y_host."""
+    if x_host.is_cuda or y_host.is_cuda:
+        raise ValueError("x_host and y_host must be host tensors")
+    M = x_host.shape[0]
+    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
+    alpha = _alpha_array(w.alphas)
+    st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                             _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                             _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _stream(stream))
+    _check(st, "bcq_gemm_host")
+    del pr_keep
+
+
+def build_lut(x: torch.Tensor, stream=None):
+    """The LUT and group sums as the GEMV kernel builds them:
+    (fp32 [M][K/8][256], fp32 [M][K/128])."""
+    _need_cuda(x, "x", torch.float16)
+    M, K = x.shape
+    lut = torch.empty((M, K // 8, 256), dtype=torch.float32, device=x.device)
+    gs = torch.empty((M, K // GROUP), dtype=torch.float32, device=x.device)
+    _check(lib().bcq_build_lut(_ptr(x), M, K, _ptr(lut), _ptr(gs), _stream(stream)),
+           "bcq_build_lut")
+    return lut, gs
+
+
+def device_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the device error word."""
+    return int(lib().bcq_device_error(_stream(stream)))
+
+
+def debug_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib().bcq_debug_wait_timeout(int(limit_us), _stream(stream)),
+           "bcq_debug_wait_timeout")

@@ -1,0 +1,169 @@
+/*
+ * bcq.h -- C ABI of libbcq, the B200 (sm_100a) multi-precision
+ * binary-coded-quantization (BCQ) matmul.
+ *
+ *   y[m][n] = sum_k x[m][k] * W_hat[n][k]
+ *   W_hat[n][k] = sum_{i=1..p_m} alpha^(p_m)[n][g][i-1] * B_i[n][k] + z[n][g],
+ *   g = k / 128,  B_i[n][k] in {-1, +1}
+ *
+ * Sources (page title, section):
+ *   "AnyBCQ: Hardware Efficient Flexible Binary-Coded Quantization for
+ *   Multi-Precision LLMs" (Paper-Notes page):
+ *     - "研究背景与动机 / 切入角度": weights are a sum of scaled binary
+ *       bit-planes; p-bit inference touches p planes;
+ *     - "关键设计 / 渐进式精度扩展": planes are shared by every precision and
+ *       each precision p has its own scales alpha^(p);
+ *     - "关键设计 / 直接bit-plane运算的CUDA内核": the kernel loads one plane at
+ *       a time, turns the contraction into additions and subtractions of
+ *       cached +-x partial sums (a LUT), scales by alpha_i and accumulates;
+ *       a p-bit call loads only the first p planes;
+ *     - "训练策略": asymmetric, group-wise with group size 128;
+ *     - "吞吐量" and the arXiv abstract: per-request precision selection.
+ *
+ * Conventions shared by every entry point
+ *   - Every buffer is owned by the caller.  Device pointers must point to
+ *     memory of the current CUDA device; "host" pointers to host memory.
+ *   - fp16 data is passed as its IEEE binary16 bit pattern (uint16_t).
+ *   - Canonical bit-planes: uint32 [p_H][N][K/32]; bit j of word w of row n is
+ *     column 32w + j (LSB first); bit value 1 means +1, 0 means -1.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously on it; the call returns after the launch.
+ *   - Every argument is validated before anything is launched.  A call that
+ *     returns an error status has launched nothing and touched no buffer.
+ *   - BCQ_ERR_CUDA reports a failed launch or copy (cudaGetLastError); the
+ *     CUDA error itself can be read with cudaGetLastError() by the caller.
+ *   - Kernels never wait without a limit.  A wait that runs out sets a device
+ *     error word (read with bcq_device_error) and the kernel returns early;
+ *     its outputs are then unspecified.
+ *   - The library allocates no device memory.
+ */
+#ifndef BCQ_H_
+#define BCQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bcq_status {
+  BCQ_OK = 0,
+  BCQ_ERR_NULL = 1,         /* a required pointer is NULL                      */
+  BCQ_ERR_SHAPE = 2,        /* M, N or K out of range, or K not a multiple of 128 */
+  BCQ_ERR_PRECISION = 3,    /* p / p_row / p_H out of range, or a needed alpha is NULL */
+  BCQ_ERR_ALIGN = 4,        /* a device pointer breaks its alignment rule      */
+  BCQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed            */
+  BCQ_ERR_TIMEOUT = 6,      /* a bounded wait inside a kernel ran out          */
+  BCQ_ERR_UNSUPPORTED = 7   /* valid request this build does not handle (e.g. group != 128) */
+} bcq_status;
+
+#define BCQ_GROUP 128       /* columns per scale group                          */
+#define BCQ_MAX_PLANES 4    /* p_H <= 4                                         */
+#define BCQ_MAX_M 64        /* rows of x per call                               */
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* bcq_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int bcq_version(void);
+
+/*
+ * Size in bytes of the packed plane buffer for p_H planes of an N x K weight
+ * (rows padded to a multiple of 32, columns to a multiple of 256).  Returns 0
+ * for invalid shapes (p_H outside 1..4, N < 1, K < 128 or K % 128 != 0).
+ */
+size_t bcq_packed_planes_bytes(int p_H, int N, int K);
+
+/*
+ * Repack canonical bit-planes into the streaming layout bcq_gemm reads.
+ * Offline, once per weight matrix (the format of the stored planes is shared
+ * by every precision: AnyBCQ page, "渐进式精度扩展").
+ *
+ *   planes_canon   device, uint32 [p_H][N][K/32], 4-byte aligned, read only.
+ *   planes_packed  device, bcq_packed_planes_bytes(p_H, N, K) bytes, 16-byte
+ *                  aligned, written entirely (padding included).  Its layout
+ *                  is private to the library; plane i occupies its own
+ *                  sub-blocks so that a p-bit call reads planes 0..p-1 only.
+ * Errors: NULL pointers -> BCQ_ERR_NULL; p_H outside 1..4 -> BCQ_ERR_PRECISION;
+ * N < 1, K < 128, K % 128 != 0 -> BCQ_ERR_SHAPE; misaligned -> BCQ_ERR_ALIGN.
+ */
+bcq_status bcq_pack_planes(const uint32_t* planes_canon, uint32_t* planes_packed,
+                           int p_H, int N, int K, void* stream);
+
+/*
+ * y = x . W_hat^T for M rows of x, each row at its own precision.
+ *
+ *   x        device, fp16 [M][K] row-major, 16-byte aligned.
+ *   planes   device, packed planes from bcq_pack_planes (p_H, N, K).
+ *   alpha    HOST array of 4 device pointers; alpha[q-1] -> fp16 [N][K/128][q],
+ *            the scales of precision q (alpha^(q)[n][g][i], i = plane).  It must
+ *            be non-NULL for every precision used by the call; the others may
+ *            be NULL.  2-byte aligned.
+ *   z        device, fp16 [N][K/128] per-(row, group) offset, or NULL (= 0).
+ *   p        uniform precision 1..p_H for every row, or 0 to use p_row.
+ *   p_row    HOST array int32 [M] of precisions 1..p_H (read during the call
+ *            only), or NULL when p > 0.
+ *   M        rows of x, 0..BCQ_MAX_M (0 = nothing to do, returns BCQ_OK).
+ *   N, K     weight shape; K % 128 == 0, K >= 128, N >= 1.
+ *   p_H      planes stored in `planes` (1..4).
+ *   group    must be 128 (other sizes -> BCQ_ERR_UNSUPPORTED).
+ *   y        device, fp16 [M][N] row-major, overwritten; 2-byte aligned.
+ * The call reads planes 0..max_m(p_m)-1 only.  Accumulation is fp32; each
+ * output is rounded once to fp16 (round to nearest even).  For a given launch
+ * configuration the summation order is fixed, so results are reproducible.
+ */
+bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes,
+                    const uint16_t* const alpha[4], const uint16_t* z,
+                    int p, const int32_t* p_row, int M, int N, int K, int p_H,
+                    int group, uint16_t* y, void* stream);
+
+/*
+ * bcq_gemm with x and y in HOST memory: enqueues the copy of x_host into
+ * x_dev, the matmul, and the copy of y_dev back into y_host, all on `stream`
+ * (pinned host buffers make the copies asynchronous).  x_dev (fp16 [M][K],
+ * 16-byte aligned) and y_dev (fp16 [M][N]) are caller-owned device staging
+ * buffers.  The caller synchronises `stream` before reading y_host.
+ * Errors as bcq_gemm, plus BCQ_ERR_NULL for missing host or staging buffers.
+ */
+bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
+                         const uint16_t* const alpha[4], const uint16_t* z,
+                         int p, const int32_t* p_row, int M, int N, int K,
+                         int p_H, int group, uint16_t* y_host,
+                         uint16_t* x_dev, uint16_t* y_dev, void* stream);
+
+/*
+ * The lookup table and group sums exactly as the GEMV kernel builds them in
+ * shared memory (AnyBCQ page, "直接bit-plane运算的CUDA内核": cached signed
+ * partial sums of x).  For test and inspection.
+ *
+ *   x           device, fp16 [M][K], 16-byte aligned; 1 <= M <= 4.
+ *   lut         device, fp32 [M][K/8][256]:
+ *               lut[m][c][b] = sum_{j<8} (2*bit_j(b) - 1) * x[m][8c + j].
+ *   group_sums  device, fp32 [M][K/128]: sum of x[m] over each group; may be NULL.
+ */
+bcq_status bcq_build_lut(const uint16_t* x, int M, int K, float* lut,
+                         float* group_sums, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of
+ * the current device: BCQ_OK when no kernel reported a problem, otherwise
+ * the status a kernel recorded (BCQ_ERR_TIMEOUT for a wait that ran out).
+ * Returns BCQ_ERR_CUDA if the synchronisation or the read fails.
+ */
+bcq_status bcq_device_error(void* stream);
+
+/*
+ * Test hook for the bounded waits: launches one CTA that waits on a
+ * shared-memory barrier nothing will complete, using the same bounded-wait
+ * routine as the GEMV kernel, with a limit of `limit_us` microseconds
+ * (1..1000000).  The kernel records BCQ_ERR_TIMEOUT in the device error word
+ * and returns; read it with bcq_device_error().  Faults nothing.
+ */
+bcq_status bcq_debug_wait_timeout(int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BCQ_H_ */

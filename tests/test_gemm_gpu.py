@@ -1,0 +1,236 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar (stated with the target): every output within
+    |y - y_ref| <= 1e-2 + 2e-3 |y_ref|
+for fp16 outputs with fp32 accumulation.  Inputs are the seeded synthetic
+recipe of bit_gemv_bcq_b200/synth.py.  Sizes: the five workload shapes (some
+at full size, the 70B-like ones on sampled output rows), plus small and
+ragged shapes spanning several row-blocks, K-blocks and split-K CTAs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_gemv_bcq_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    api.lib()
+    yield
+    assert api.device_error() == api.BCQ_OK
+
+
+def _weights(prob):
+    return api.BcqWeights.from_canonical(prob.planes, prob.alphas, prob.z)
+
+
+def _x(prob):
+    return torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).cuda()
+
+
+def _check(y_gpu, y_ref, what=""):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    err = np.abs(y - y_ref)
+    bound = ATOL + RTOL * np.abs(y_ref)
+    bad = err > bound
+    assert not bad.any(), (
+        f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst "
+        f"err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}")
+    return float(err.max())
+
+
+def _run(prob, w=None, p=None, p_row=None):
+    w = _weights(prob) if w is None else w
+    y = w.gemm(_x(prob), p=p, p_row=p_row)
+    torch.cuda.synchronize()
+    return y
+
+
+# --------------------------------------------------------------- small / ragged
+
+@pytest.mark.parametrize("N,K", [(1, 128), (31, 384), (33, 640), (100, 1024),
+                                 (256, 512), (1000, 2048), (64, 128 * 33)])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+def test_parity_small_and_ragged(N, K, M):
+    prob = synth.make_problem(N, K, M, seed=N + K + M, precisions=(1, 2, 3, 4))
+    w = _weights(prob)
+    for p in (1, 2, 3, 4):
+        y = _run(prob, w, p=p)
+        _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p),
+               f"N={N} K={K} M={M} p={p}")
+
+
+def test_parity_tiny_config_all_precisions():
+    """256 x 512, M = 1, p = 2, 3, 4, seed 0 (the tiny workload)."""
+    prob = synth.make_problem(256, 512, 1, seed=0)
+    w = _weights(prob)
+    for p in (2, 3, 4):
+        _check(_run(prob, w, p=p), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p))
+
+
+def test_parity_attention_projection_full():
+    """4096 x 4096, M = 1, p = 2, 3, 4 (every output)."""
+    prob = synth.make_problem(4096, 4096, 1, seed=1)
+    w = _weights(prob)
+    for p in (2, 3, 4):
+        _check(_run(prob, w, p=p), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p),
+               f"p={p}")
+
+
+@pytest.mark.parametrize("N,K", [(14336, 4096), (4096, 14336)])
+def test_parity_mlp_decode_with_outliers_full(N, K):
+    """Llama-3.1-8B MLP shapes, M = 1, 0.1 % outlier channels x 20."""
+    prob = synth.make_problem(N, K, 1, seed=2, outliers=True)
+    w = _weights(prob)
+    for p in (2, 3, 4):
+        _check(_run(prob, w, p=p), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p),
+               f"{N}x{K} p={p}")
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096)])
+def test_parity_batch_sweep(N, K):
+    """M in {1, 2, 4, 8, 16}, p = 2, 3, 4, all outputs."""
+    prob = synth.make_problem(N, K, 16, seed=3)
+    w = _weights(prob)
+    for M in (1, 2, 4, 8, 16):
+        sub = synth.Problem(x=prob.x[:M], planes=prob.planes, alphas=prob.alphas, z=prob.z)
+        for p in (2, 3, 4):
+            y = _run(sub, w, p=p)
+            _check(y, oracle.gemm(sub.x, prob.planes, prob.alphas, prob.z, p=p), f"M={M} p={p}")
+
+
+@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
+def test_parity_mixed_precision_70b_sampled(N, K):
+    """M = 8 rows with p drawn from {2,3,4}; outputs checked on 1024 sampled
+    rows plus the first and last row-blocks."""
+    prob = synth.make_problem(N, K, 8, seed=4, mixed=True)
+    assert set(prob.p_row.tolist()) <= {2, 3, 4}
+    y = _run(prob, p_row=prob.p_row)
+    rng = np.random.default_rng(40)
+    rows = np.unique(np.concatenate([np.arange(32), np.arange(N - 32, N),
+                                     rng.choice(N, 1024, replace=False)])).astype(np.int32)
+    ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row, rows=rows)
+    _check(y[:, torch.from_numpy(rows).long().cuda()], ref, f"{N}x{K} mixed")
+
+
+# ------------------------------------------------------------------ invariants
+
+def test_p_prefix_poisoned_planes_are_never_read():
+    """Planes p..p_H-1 replaced by random bits: bitwise identical output."""
+    prob = synth.make_problem(1000, 2048, 3, seed=5)
+    w = _weights(prob)
+    rng = np.random.default_rng(50)
+    for p in (1, 2, 3):
+        y1 = _run(prob, w, p=p)
+        poisoned = prob.planes.copy()
+        poisoned[p:] = rng.integers(0, 2**32, size=poisoned[p:].shape, dtype=np.uint32)
+        w2 = api.BcqWeights.from_canonical(poisoned, prob.alphas, prob.z)
+        y2 = _run(prob, w2, p=p)
+        assert torch.equal(y1, y2), f"p={p}"
+
+
+def test_results_are_reproducible():
+    prob = synth.make_problem(14336, 4096, 2, seed=6)
+    w = _weights(prob)
+    ys = [_run(prob, w, p=3) for _ in range(3)]
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+
+
+def test_mixed_rows_match_uniform_calls():
+    prob = synth.make_problem(4096, 4096, 8, seed=7, mixed=True)
+    prob.p_row[:] = [4, 2, 3, 3, 2, 4, 2, 3]
+    w = _weights(prob)
+    y = _run(prob, w, p_row=prob.p_row)
+    for m, q in enumerate(prob.p_row):
+        one = synth.Problem(x=prob.x[m:m + 1], planes=prob.planes, alphas=prob.alphas, z=prob.z)
+        ym = _run(one, w, p=int(q))
+        assert (y[m].float() - ym[0].float()).abs().max().item() <= 2 * ATOL
+    _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row))
+
+
+def test_sign_symmetry():
+    prob = synth.make_problem(512, 1024, 1, seed=8)
+    y = _run(prob, p=4)
+    flipped = prob.planes.copy()
+    flipped[1] = ~flipped[1]
+    al = {q: a.copy() for q, a in prob.alphas.items()}
+    al[4][:, :, 1] = -al[4][:, :, 1]
+    y2 = _run(synth.Problem(x=prob.x, planes=flipped, alphas=al, z=prob.z), p=4)
+    assert (y.float() - y2.float()).abs().max().item() <= 2 * ATOL
+
+
+def test_fewer_stored_planes_and_no_offset():
+    prob = synth.make_problem(300, 768, 2, seed=9, p_H=2, precisions=(1, 2))
+    w = api.BcqWeights.from_canonical(prob.planes, prob.alphas, None)
+    for p in (1, 2):
+        y = _run(prob, w, p=p)
+        _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, None, p=p), f"p={p}")
+
+
+def test_hand_example_through_the_gpu():
+    """The BiLoCo hand example: x = [0.5, -1.2, 2.0, 0.3], v = [+1,-1,+1,-1],
+    v.x = 3.4 (K = 128, p = 1, alpha = 1, z = 0)."""
+    x = np.zeros((1, 128), dtype=np.float16)
+    x[0, :4] = [0.5, -1.2, 2.0, 0.3]
+    planes = np.zeros((1, 1, 4), dtype=np.uint32)
+    planes[0, 0, 0] = 0b0101
+    alphas = {1: np.ones((1, 1, 1), dtype=np.float16)}
+    prob = synth.Problem(x=x, planes=planes, alphas=alphas, z=np.zeros((1, 1), np.float16))
+    y = _run(prob, p=1)
+    assert abs(float(y[0, 0]) - 3.4) < 2e-3
+
+
+def test_empty_batch():
+    prob = synth.make_problem(64, 256, 1, seed=10)
+    w = _weights(prob)
+    y = w.gemm(torch.empty((0, 256), dtype=torch.float16, device="cuda"), p=2)
+    assert y.shape == (0, 64)
+
+
+# -------------------------------------------------- steps of the path (a1, a2)
+
+@pytest.mark.parametrize("M,K", [(1, 128), (1, 4096), (2, 640), (3, 384), (4, 1024)])
+def test_lut_and_group_sums_match_oracle(M, K):
+    x = synth.make_x(M, K, seed=K + M)
+    lut, gs = api.build_lut(torch.from_numpy(x.view(np.int16)).view(torch.float16).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.lut(x)
+    # each entry is a sum of 8 fp16 values in fp32: a few ulps of |sum|
+    err = np.abs(lut.cpu().numpy().astype(np.float64) - ref)
+    assert err.max() <= 1e-5 * (1 + np.abs(ref).max())
+    gref = oracle.group_sums(x)
+    assert np.abs(gs.cpu().numpy() - gref).max() <= 1e-4 * (1 + np.abs(gref).max())
+
+
+# ---------------------------------------------------------------- host path
+
+def test_host_buffers_path_matches_device_path():
+    prob = synth.make_problem(4096, 4096, 4, seed=11)
+    w = _weights(prob)
+    y_dev_ref = _run(prob, w, p=3)
+    x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).pin_memory()
+    y_host = torch.empty((4, 4096), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty((4, 4096), dtype=torch.float16, device="cuda")
+    y_dev = torch.empty((4, 4096), dtype=torch.float16, device="cuda")
+    api.gemm_host(x_host, w, y_host, x_dev, y_dev, p=3)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, y_dev_ref.cpu())
+
+
+# ------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert api.device_error() == api.BCQ_OK
+    api.debug_wait_timeout(20000)          # 20 ms on a barrier nothing completes
+    assert api.device_error() == api.BCQ_ERR_TIMEOUT
+    assert api.device_error() == api.BCQ_OK   # read clears it
+    prob = synth.make_problem(256, 512, 1, seed=12)
+    _check(_run(prob, p=2), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=2))

@@ -132,6 +132,9 @@ def run_gpu(args, rank, world, local_rank):
     x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).to(dev)
     ys = {M: torch.empty((M, N_OUT), dtype=torch.float16, device=dev) for M in BATCHES}
     cases = [(p, M) for p in PRECISIONS for M in BATCHES]
+    if args.cases:
+        want = {tuple(int(v) for v in c.split(":")) for c in args.cases.split(",")}
+        cases = [(p, M) for p, M in cases if (M, p) in want]
     bytes_step = sum(algo_bytes(N_OUT, K_IN, M, p) for p, M in cases)
     launches_per_step = sum(math.ceil(M / 4) for _, M in cases)
 
@@ -290,6 +293,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-rows", type=int, default=14336,
                     help="output rows per call in the oracle's timed sample")
+    ap.add_argument("--cases", default="",
+                    help="restrict the step to these M:p pairs (profiling only), e.g. 1:2,1:3")
     ap.add_argument("--profile", action="store_true",
                     help="GPU timing only (no e2e or CPU legs), for profiler runs")
     args = ap.parse_args()

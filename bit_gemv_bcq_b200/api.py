@@ -63,6 +63,14 @@ def lib():
         L.bcq_packed_planes_bytes.argtypes = [I, I, I]
         L.bcq_pack_planes.restype = I
         L.bcq_pack_planes.argtypes = [P, P, I, I, I, P]
+        L.bcq_packed_scales_bytes.restype = S
+        L.bcq_packed_scales_bytes.argtypes = [I, I, I]
+        L.bcq_pack_scales.restype = I
+        L.bcq_pack_scales.argtypes = [P, I, I, I, P, P]
+        L.bcq_set_pdl.restype = I
+        L.bcq_set_pdl.argtypes = [I]
+        L.bcq_plan_query.restype = I
+        L.bcq_plan_query.argtypes = [I, I, I, I, I, I, I, I, P]
         L.bcq_gemm.restype = I
         L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
         L.bcq_gemm_host.restype = I
@@ -78,7 +86,8 @@ def lib():
 
 
 EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
-            "bcq_pack_planes", "bcq_gemm", "bcq_gemm_host", "bcq_build_lut",
+            "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
+            "bcq_gemm", "bcq_plan_query", "bcq_set_pdl", "bcq_gemm_host", "bcq_build_lut",
             "bcq_device_error", "bcq_debug_wait_timeout")
 
 
@@ -142,13 +151,52 @@ def pack_planes(planes_canon: torch.Tensor, stream=None) -> torch.Tensor:
     return out
 
 
+def packed_scales_bytes(q: int, N: int, K: int) -> int:
+    return int(lib().bcq_packed_scales_bytes(q, N, K))
+
+
+def pack_scales(src: torch.Tensor, q: int, stream=None) -> torch.Tensor:
+    """Canonical fp16 per-(row, group) array [N][K/128][q] (or [N][K/128] for
+    q = 1) -> packed streaming order (fp16 CUDA tensor)."""
+    _need_cuda(src, "scales", torch.float16)
+    N, G = src.shape[0], src.shape[1]
+    if src.numel() != N * G * q:
+        raise ValueError("scales must hold q values per (row, group)")
+    K = G * GROUP
+    nbytes = packed_scales_bytes(q, N, K)
+    if nbytes == 0:
+        raise BcqError(BCQ_ERR_SHAPE, "bcq_packed_scales_bytes")
+    out = torch.empty(nbytes // 2, dtype=torch.float16, device=src.device)
+    _check(lib().bcq_pack_scales(_ptr(src), int(q), N, K, _ptr(out), _stream(stream)),
+           "bcq_pack_scales")
+    return out
+
+
+PLAN_FIELDS = ("S", "C", "W", "NP", "D", "dyn_bytes", "stage_bytes", "row_groups")
+
+
+def plan_query(M: int, N: int, K: int, p_load: int, q0: int, q1: int = 0,
+               has_z: bool = True, use_device: bool = False) -> dict:
+    """Launch plan of one GEMV launch (see bcq_plan_query)."""
+    out = (ctypes.c_int * 8)()
+    _check(lib().bcq_plan_query(M, N, K, p_load, q0, q1, int(has_z), int(use_device),
+                                ctypes.cast(out, ctypes.c_void_p)), "bcq_plan_query")
+    return dict(zip(PLAN_FIELDS, list(out)))
+
+
+def set_pdl(mode: int) -> None:
+    """Programmatic dependent launch for later GEMV launches (see bcq_set_pdl)."""
+    _check(lib().bcq_set_pdl(int(mode)), "bcq_set_pdl")
+
+
 @dataclass
 class BcqWeights:
     """One BCQ weight matrix on the device: packed +-1 planes shared by every
-    precision, the scales alpha^(q) of each precision q, and the offset z."""
+    precision, the scales alpha^(q) of each precision q and the offsets z,
+    all in the library's streaming order (bcq_pack_planes, bcq_pack_scales)."""
     packed: torch.Tensor        # int32, library layout
-    alphas: dict                # {q: fp16 [N][G][q]}
-    z: torch.Tensor | None      # fp16 [N][G] or None
+    alphas: dict                # {q: packed alpha^(q), fp16}
+    z: torch.Tensor | None      # packed offsets (fp16) or None
     N: int
     K: int
     p_H: int
@@ -165,11 +213,12 @@ class BcqWeights:
         al = {}
         for q, a in alphas.items():
             a = torch.as_tensor(a) if isinstance(a, np.ndarray) else a
-            al[int(q)] = a.to(device=device, dtype=torch.float16).contiguous()
+            al[int(q)] = pack_scales(a.to(device=device, dtype=torch.float16).contiguous(),
+                                     int(q), stream)
         zz = None
         if z is not None:
             zz = (torch.as_tensor(z) if isinstance(z, np.ndarray) else z)
-            zz = zz.to(device=device, dtype=torch.float16).contiguous()
+            zz = pack_scales(zz.to(device=device, dtype=torch.float16).contiguous(), 1, stream)
         return cls(packed=packed, alphas=al, z=zz, N=N, K=KW * 32, p_H=p_H)
 
     def gemm(self, x, p=None, p_row=None, out=None, stream=None):

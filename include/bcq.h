@@ -92,15 +92,41 @@ bcq_status bcq_pack_planes(const uint32_t* planes_canon, uint32_t* planes_packed
                            int p_H, int N, int K, void* stream);
 
 /*
+ * Size in bytes of a packed per-(row, group) array with q values per entry
+ * (q = 1..4), or 0 for invalid arguments (same shape rules as above).
+ */
+size_t bcq_packed_scales_bytes(int q, int N, int K);
+
+/*
+ * Repack a per-(row, group) fp16 array into the streaming order bcq_gemm
+ * reads, next to the planes of the same rows and groups.  Offline, once per
+ * weight matrix.  Used for the scales of each precision (AnyBCQ page,
+ * "渐进式精度扩展": every precision p has its own alpha^(p)) with q = p, and
+ * for the asymmetric offsets z ("训练策略") with q = 1.
+ *
+ *   src   device, fp16 [N][K/128][q] (entry (n, g) holds q values), 2-byte
+ *         aligned, read only.
+ *   dst   device, bcq_packed_scales_bytes(q, N, K) bytes, 16-byte aligned,
+ *         written entirely (zero padding outside the matrix).
+ * Errors: NULL -> BCQ_ERR_NULL; q outside 1..4 -> BCQ_ERR_PRECISION; shape ->
+ * BCQ_ERR_SHAPE; misaligned -> BCQ_ERR_ALIGN.
+ */
+bcq_status bcq_pack_scales(const uint16_t* src, int q, int N, int K,
+                           uint16_t* dst, void* stream);
+
+/*
  * y = x . W_hat^T for M rows of x, each row at its own precision.
  *
  *   x        device, fp16 [M][K] row-major, 16-byte aligned.
  *   planes   device, packed planes from bcq_pack_planes (p_H, N, K).
- *   alpha    HOST array of 4 device pointers; alpha[q-1] -> fp16 [N][K/128][q],
- *            the scales of precision q (alpha^(q)[n][g][i], i = plane).  It must
- *            be non-NULL for every precision used by the call; the others may
- *            be NULL.  2-byte aligned.
- *   z        device, fp16 [N][K/128] per-(row, group) offset, or NULL (= 0).
+ *   alpha    HOST array of 4 device pointers; alpha[q-1] -> the scales of
+ *            precision q (alpha^(q)[n][g][i], i = plane, canonically fp16
+ *            [N][K/128][q]) packed by bcq_pack_scales(.., q, ..).  It must be
+ *            non-NULL for every precision used by the call; the others may be
+ *            NULL.  16-byte aligned.
+ *   z        device, the per-(row, group) offsets (canonically fp16
+ *            [N][K/128]) packed by bcq_pack_scales(.., 1, ..), or NULL (= 0).
+ *            16-byte aligned.
  *   p        uniform precision 1..p_H for every row, or 0 to use p_row.
  *   p_row    HOST array int32 [M] of precisions 1..p_H (read during the call
  *            only), or NULL when p > 0.
@@ -117,6 +143,32 @@ bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes,
                     const uint16_t* const alpha[4], const uint16_t* z,
                     int p, const int32_t* p_row, int M, int N, int K, int p_H,
                     int group, uint16_t* y, void* stream);
+
+/*
+ * The launch plan bcq_gemm would use for one launch of M (1..2) activation
+ * rows: p_load planes streamed, precisions q0 (and q1, 0 = none) among the
+ * rows, offsets present (has_z).  use_device = 1 plans for the current
+ * device; 0 (or no usable device) plans for a nominal 148-SM B200 without
+ * touching CUDA.  out[8] receives: cluster size S (K splits), clusters C,
+ * consumer warps, producer warps, ring stages, dynamic shared memory bytes,
+ * stage bytes, row groups per cluster.  For inspection and tests.
+ */
+int bcq_plan_query(int M, int N, int K, int p_load, int q0, int q1, int has_z,
+                   int use_device, int* out);
+
+/*
+ * Launch option for the GEMV kernels of this process (all devices):
+ *   0  plain stream order (default);
+ *   1  programmatic dependent launch: a GEMV kernel may be scheduled while the
+ *      preceding kernel in its stream finishes; it touches no global memory
+ *      before that kernel has completed;
+ *   2  as 1, but the kernel may start streaming its planes and packed scales
+ *      before the preceding kernel has completed (x and y still wait).  Only
+ *      valid when no kernel immediately before it in the stream writes the
+ *      weights it reads.
+ * Returns BCQ_OK, or BCQ_ERR_UNSUPPORTED for another mode.
+ */
+int bcq_set_pdl(int mode);
 
 /*
  * bcq_gemm with x and y in HOST memory: enqueues the copy of x_host into

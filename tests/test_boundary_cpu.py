@@ -42,12 +42,48 @@ def test_version_and_status_strings(L):
 
 
 def test_packed_bytes_formula(L):
-    # ceil(N/32) row-blocks x p_H x ceil(K/256) K-blocks x 1 KiB
-    assert api.packed_planes_bytes(4, 14336, 4096) == 448 * 4 * 16 * 1024
+    # chunks of 512 columns x row groups of 4 row-blocks (128 rows) x p_H x 8 KiB
+    assert api.packed_planes_bytes(4, 14336, 4096) == 8 * 112 * 4 * 8192
     assert api.packed_planes_bytes(4, 14336, 4096) == 14336 * 4096 * 4 // 8
-    assert api.packed_planes_bytes(2, 33, 384) == 2 * 2 * 2 * 1024
+    assert api.packed_planes_bytes(2, 33, 384) == 1 * 1 * 2 * 8192     # padded
     for bad in [(0, 32, 256), (5, 32, 256), (4, 0, 256), (4, 32, 100), (4, 32, 0)]:
         assert api.packed_planes_bytes(*bad) == 0
+    # chunks x row-blocks (padded to groups of 4) x 2 K-blocks x 2 passes x 32 lanes x q halves
+    assert api.packed_scales_bytes(3, 14336, 4096) == 8 * 448 * 128 * 3 * 2
+    assert api.packed_scales_bytes(3, 14336, 4096) == 14336 * 32 * 3 * 2
+    assert api.packed_scales_bytes(1, 33, 384) == 1 * 4 * 128 * 1 * 2
+    assert api.packed_scales_bytes(0, 32, 256) == 0
+
+
+@pytest.mark.parametrize("M,N,K,p,q1", [(1, 14336, 4096, 2, 0), (1, 14336, 4096, 4, 0),
+                                        (1, 4096, 14336, 3, 0), (2, 4096, 4096, 2, 0),
+                                        (2, 28672, 8192, 3, 2), (1, 256, 512, 4, 0),
+                                        (1, 1, 128, 1, 0), (2, 33, 640, 2, 0)])
+def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, q1):
+    """Plans for a nominal 148-SM B200 (no GPU needed): every launch fits the
+    227 KiB of shared memory, splits K into at most the chunks there are,
+    and keeps the ring depth a multiple of both the consumer groups and the
+    producer warps (the stage-ownership rule of the pipeline)."""
+    pl = api.plan_query(M, N, K, p, p, q1, has_z=True, use_device=False)
+    KC = -(-(-(-K // 256)) // 2)
+    assert 1 <= pl["S"] <= min(8, KC)
+    assert pl["dyn_bytes"] <= 232448
+    G = pl["W"] // 4
+    assert pl["W"] % 4 == 0 and pl["D"] % G == 0 and pl["D"] % pl["NP"] == 0
+    assert 2 <= pl["D"] <= 8
+    assert pl["C"] * pl["S"] <= 148
+    RBG = -(-(-(-N // 32)) // 4)
+    assert pl["row_groups"] * pl["C"] <= RBG + pl["C"]
+    assert pl["stage_bytes"] == 4 * (p * 2048 + 256 * (p + q1) + 256)
+
+
+def test_plan_query_rejects_bad_arguments(L):
+    with pytest.raises(api.BcqError):
+        api.plan_query(3, 64, 256, 2, 2)          # at most two rows per launch
+    with pytest.raises(api.BcqError):
+        api.plan_query(1, 64, 200, 2, 2)          # K % 128
+    with pytest.raises(api.BcqError):
+        api.plan_query(1, 64, 256, 5, 2)          # p_load
 
 
 FAKE = 0x10000   # never dereferenced: every call below fails validation first
@@ -92,7 +128,8 @@ def test_gemm_rejects_before_launch(L):
     assert _gemm(L, y=FAKE + 1) == api.BCQ_ERR_ALIGN
     assert _gemm(L, z=FAKE + 1) == api.BCQ_ERR_ALIGN
     assert _gemm(L, alpha=_alpha(2, base=FAKE + 2), p=2) == api.BCQ_ERR_ALIGN
-    assert _gemm(L, alpha=_alpha(4, base=FAKE + 4), p=4) == api.BCQ_ERR_ALIGN
+    assert _gemm(L, alpha=_alpha(4, base=FAKE + 8), p=4) == api.BCQ_ERR_ALIGN
+    assert _gemm(L, z=FAKE + 8) == api.BCQ_ERR_ALIGN
 
 
 def test_pack_and_lut_reject_before_launch(L):
@@ -104,6 +141,14 @@ def test_pack_and_lut_reject_before_launch(L):
     assert L.bcq_build_lut(FAKE, 5, 256, FAKE, None, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_build_lut(FAKE, 1, 250, FAKE, None, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_build_lut(FAKE + 8, 1, 256, FAKE, None, None) == api.BCQ_ERR_ALIGN
+    assert L.bcq_pack_scales(None, 2, 64, 256, FAKE, None) == api.BCQ_ERR_NULL
+    assert L.bcq_pack_scales(FAKE, 0, 64, 256, FAKE, None) == api.BCQ_ERR_PRECISION
+    assert L.bcq_pack_scales(FAKE, 5, 64, 256, FAKE, None) == api.BCQ_ERR_PRECISION
+    assert L.bcq_pack_scales(FAKE, 2, 64, 200, FAKE, None) == api.BCQ_ERR_SHAPE
+    assert L.bcq_pack_scales(FAKE + 1, 2, 64, 256, FAKE, None) == api.BCQ_ERR_ALIGN
+    assert L.bcq_pack_scales(FAKE, 2, 64, 256, FAKE + 8, None) == api.BCQ_ERR_ALIGN
+    assert L.bcq_set_pdl(3) == api.BCQ_ERR_UNSUPPORTED
+    assert L.bcq_set_pdl(0) == api.BCQ_OK
     assert L.bcq_debug_wait_timeout(0, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_debug_wait_timeout(2000000, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_gemm_host(None, FAKE, _alpha(2), None, 2, None, 1, 64, 256, 4, 128,

@@ -125,7 +125,7 @@ def test_parity_mixed_precision_70b_sampled(N, K):
 
 def test_p_prefix_poisoned_planes_are_never_read():
     """Planes p..p_H-1 replaced by random bits: bitwise identical output."""
-    prob = synth.make_problem(1000, 2048, 3, seed=5)
+    prob = synth.make_problem(1000, 2048, 3, seed=5, precisions=(1, 2, 3, 4))
     w = _weights(prob)
     rng = np.random.default_rng(50)
     for p in (1, 2, 3):

@@ -136,7 +136,8 @@ def run_gpu(args, rank, world, local_rank):
         want = {tuple(int(v) for v in c.split(":")) for c in args.cases.split(",")}
         cases = [(p, M) for p, M in cases if (M, p) in want]
     bytes_step = sum(algo_bytes(N_OUT, K_IN, M, p) for p, M in cases)
-    launches_per_step = sum(math.ceil(M / 4) for _, M in cases)
+    api.set_pdl(args.pdl)
+    launches_per_step = sum(launches_per_call(M) for p, M in cases)
 
     stream = torch.cuda.Stream(device=dev)
     # eager pass: plans and caches every launch shape before capture
@@ -260,6 +261,11 @@ def run_gpu(args, rank, world, local_rank):
     return result
 
 
+def launches_per_call(M):
+    """GEMV kernel launches of one bcq_gemm call: one per two activation rows."""
+    return -(-M // 2)
+
+
 # ------------------------------------------------------------- CPU oracle arm
 
 def run_oracle_sample(seed, rows_per_call, prob=None):
@@ -293,8 +299,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-rows", type=int, default=14336,
                     help="output rows per call in the oracle's timed sample")
+    ap.add_argument("--cpu-reps", type=int, default=4,
+                    help="repetitions of the oracle's sample (about 10-30 s of CPU work)")
     ap.add_argument("--cases", default="",
                     help="restrict the step to these M:p pairs (profiling only), e.g. 1:2,1:3")
+    ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
+                    help="bcq_set_pdl mode for the GEMV launches (2: weights may stream "
+                         "while the previous kernel drains; no kernel of the step writes them)")
     ap.add_argument("--profile", action="store_true",
                     help="GPU timing only (no e2e or CPU legs), for profiler runs")
     args = ap.parse_args()
@@ -357,7 +368,8 @@ def main():
                    "l2": f"inputs larger than L2: {res['R']} rotating weight copies of "
                          f"{res['per_copy_bytes'] / 2**20:.1f} MiB",
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "timing": "CUDA graph per step, CUDA events on the launching stream"},
+                   "timing": "CUDA graph per step, CUDA events on the launching stream",
+                   "pdl": args.pdl},
         "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
                      "peak_kind": peak_kind, "traffic": None,
@@ -376,11 +388,15 @@ def main():
                        "ms_per_step": round(e["ms"] / e["steps"], 4),
                        "path": "bcq_gemm_host (pinned host x/y, copies on the stream)"}
     if rank == 0 and world == 1 and not args.profile:
-        secs, by, thr = run_oracle_sample(args.seed, args.cpu_rows)
+        secs, by, thr = 0.0, 0.0, 1
+        for k in range(max(1, args.cpu_reps)):
+            s_k, b_k, thr = run_oracle_sample(args.seed + k, args.cpu_rows)
+            secs += s_k
+            by += b_k
         line["cpu_baseline"] = {"value": round(by / secs / 1e9, 4), "unit": "GB/s", "cores": thr,
                                 "kind": "oracle",
                                 "sample": f"{args.cpu_rows} of {N_OUT} output rows of each of the "
-                                          f"15 calls ({secs:.1f} s)"}
+                                          f"15 calls, {max(1, args.cpu_reps)} times ({secs:.1f} s)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

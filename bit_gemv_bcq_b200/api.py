@@ -5,9 +5,11 @@ current torch stream becomes the CUDA stream, and every step of the matmul
 runs in the library's kernels.  There is no CPU fallback: a missing
 ``libbcq.so`` raises ``BcqLibraryError`` on first use.
 
-The same names as the C ABI: ``pack_planes``, ``gemm``, ``gemm_host``,
-``build_lut``, ``device_error``, ``debug_wait_timeout``; ``BcqWeights`` bundles
-the packed planes with their scales and offsets.
+The same names as the C ABI: ``pack_planes``, ``pack_scales``,
+``workspace_bytes``, ``gemm``, ``gemm_host``, ``build_lut``, ``device_error``,
+``debug_wait_timeout``; ``BcqWeights`` bundles the packed planes with their
+scales and offsets.  The split-K workspace bcq_gemm needs is kept here, one
+zero-filled buffer per (device, stream), grown on demand.
 """
 from __future__ import annotations
 
@@ -69,12 +71,14 @@ def lib():
         L.bcq_pack_scales.argtypes = [P, I, I, I, P, P]
         L.bcq_set_pdl.restype = I
         L.bcq_set_pdl.argtypes = [I]
+        L.bcq_workspace_bytes.restype = S
+        L.bcq_workspace_bytes.argtypes = [I, I, I]
         L.bcq_plan_query.restype = I
-        L.bcq_plan_query.argtypes = [I, I, I, I, I, I, I, I, P]
+        L.bcq_plan_query.argtypes = [I, I, I, I, I, I, P]
         L.bcq_gemm.restype = I
-        L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
+        L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, S, P]
         L.bcq_gemm_host.restype = I
-        L.bcq_gemm_host.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, P, P]
+        L.bcq_gemm_host.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, P, P, S, P]
         L.bcq_build_lut.restype = I
         L.bcq_build_lut.argtypes = [P, I, I, P, P, P]
         L.bcq_device_error.restype = I
@@ -87,7 +91,7 @@ def lib():
 
 EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
-            "bcq_gemm", "bcq_plan_query", "bcq_set_pdl", "bcq_gemm_host", "bcq_build_lut",
+            "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl", "bcq_gemm_host", "bcq_build_lut",
             "bcq_device_error", "bcq_debug_wait_timeout")
 
 
@@ -172,16 +176,48 @@ def pack_scales(src: torch.Tensor, q: int, stream=None) -> torch.Tensor:
     return out
 
 
-PLAN_FIELDS = ("S", "C", "W", "NP", "D", "dyn_bytes", "stage_bytes", "row_groups")
+PLAN_FIELDS = ("C", "consumer_warps", "NP", "D", "dyn_bytes", "stage_bytes", "units_max",
+               "KB")
 
 
-def plan_query(M: int, N: int, K: int, p_load: int, q0: int, q1: int = 0,
-               has_z: bool = True, use_device: bool = False) -> dict:
+def plan_query(M: int, N: int, K: int, p_load: int, mixed: bool = False,
+               use_device: bool = False) -> dict:
     """Launch plan of one GEMV launch (see bcq_plan_query)."""
     out = (ctypes.c_int * 8)()
-    _check(lib().bcq_plan_query(M, N, K, p_load, q0, q1, int(has_z), int(use_device),
+    _check(lib().bcq_plan_query(M, N, K, p_load, int(mixed), int(use_device),
                                 ctypes.cast(out, ctypes.c_void_p)), "bcq_plan_query")
     return dict(zip(PLAN_FIELDS, list(out)))
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bcq_workspace_bytes(M, N, K))
+
+
+_WS: dict = {}
+
+
+def workspace(M: int, N: int, K: int, device, stream=None) -> torch.Tensor | None:
+    """The zero-filled workspace of (device, stream), at least
+    bcq_workspace_bytes(M, N, K) bytes; None when none is needed.  Every call
+    that completes leaves it zero-filled again."""
+    need = workspace_bytes(M, N, K)
+    if need == 0:
+        return None
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    key = (torch.device(device).index, s.cuda_stream)
+    ws = _WS.get(key)
+    if ws is None or ws.numel() < need:
+        with torch.cuda.stream(s):
+            ws = torch.zeros(max(need, 2 * ws.numel() if ws is not None else need),
+                             dtype=torch.uint8, device=device)
+        _WS[key] = ws
+    return ws
+
+
+def drop_workspaces() -> None:
+    """Forget the cached workspaces (after a device error they may hold
+    stale counters; new ones are zero-filled)."""
+    _WS.clear()
 
 
 def set_pdl(mode: int) -> None:
@@ -249,9 +285,11 @@ def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
     else:
         _need_cuda(out, "out", torch.float16)
     alpha = _alpha_array(w.alphas)
+    ws = workspace(M, w.N, w.K, x.device, stream)
     st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
                         _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                        _ptr(out), _stream(stream))
+                        _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                        _stream(stream))
     _check(st, "bcq_gemm")
     del pr_keep
     return out
@@ -267,9 +305,11 @@ def gemm_host(x_host: torch.Tensor, w: BcqWeights, y_host: torch.Tensor,
     M = x_host.shape[0]
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
     alpha = _alpha_array(w.alphas)
+    ws = workspace(M, w.N, w.K, x_dev.device, stream)
     st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
                              _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                             _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _stream(stream))
+                             _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(ws),
+                             0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "bcq_gemm_host")
     del pr_keep
 
@@ -287,8 +327,12 @@ def build_lut(x: torch.Tensor, stream=None):
 
 
 def device_error(stream=None) -> int:
-    """Synchronise the stream, return and clear the device error word."""
-    return int(lib().bcq_device_error(_stream(stream)))
+    """Synchronise the stream, return and clear the device error word.  After
+    an error the cached workspaces are dropped (their counters may be stale)."""
+    st = int(lib().bcq_device_error(_stream(stream)))
+    if st != BCQ_OK:
+        drop_workspaces()
+    return st
 
 
 def debug_wait_timeout(limit_us: int, stream=None) -> None:

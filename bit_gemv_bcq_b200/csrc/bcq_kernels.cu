@@ -2,10 +2,12 @@
 //
 //   pack_planes_kernel   canonical planes -> streaming layout (offline)
 //   pack_scales_kernel   per-(row, group) scales/offsets -> streaming order
-//   gemv_lut_kernel      LUT build + plane/scale streaming (producer warp,
-//                        bulk copies) + lookup-accumulate + alpha/z fusion +
-//                        cluster split-K reduction + fp16 out
-//   lut_dump_kernel      the same LUT build, written out for inspection
+//   gemv_lut_kernel      producer warps stream plane stages by bulk copy;
+//                        consumer warps build the K-block's lookup table,
+//                        look up and accumulate, fuse alpha and z, and write
+//                        split-K partial sums; the last CTA to finish a
+//                        row-block sums its partials in K order -> fp16 y
+//   lut_dump_kernel      the same table build, written out for inspection
 //   wait_probe_kernel    exercises the bounded mbarrier wait
 //
 // Method (page title, section): "AnyBCQ: Hardware Efficient Flexible
@@ -15,7 +17,6 @@
 // table of cached partial sums; scale by alpha_i, accumulate; output after
 // p planes; a p-bit call loads only p planes.  Group size 128, asymmetric
 // offset: same page, "训练策略".
-#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -23,8 +24,6 @@
 #include "bcq_device.cuh"
 #include "bcq_launch.h"
 #include "bcq_layout.h"
-
-namespace cg = cooperative_groups;
 
 namespace bcq {
 
@@ -36,24 +35,22 @@ __device__ int g_device_error = 0;
 
 // One thread per packed word; see bcq_layout.h for the layout.
 __global__ void pack_planes_kernel(const uint32_t* __restrict__ canon,
-                                   uint32_t* __restrict__ packed, int p_H,
-                                   int N, int K, int RBG, size_t total_words) {
+                                   uint32_t* __restrict__ packed, int p_H, int N, int K,
+                                   int RG, size_t total_words) {
   const int KW = K / 32;
   for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < total_words;
        w += (size_t)gridDim.x * blockDim.x) {
     const int u = (int)(w & 3);
     const int lane = (int)((w >> 2) & 31);
     const int pass = (int)((w >> 7) & 1);
-    const int kbi = (int)((w >> 8) & 1);
-    size_t rest = w >> 9;
+    size_t rest = w >> 8;
     const int r = (int)(rest % kRowGroup);
     rest /= kRowGroup;
     const int i = (int)(rest % p_H);
     rest /= p_H;
-    const size_t rg = rest % RBG;
-    const size_t chunk = rest / RBG;
+    const size_t rg = rest % RG;
+    const size_t kb = rest / RG;
     const size_t rb = rg * kRowGroup + r;
-    const size_t kb = chunk * kChunkBlocks + kbi;
     const size_t n = rb * kRowBlock + lane;
     const int h = (lane >> 4) ^ pass;
     uint32_t out = 0;
@@ -77,20 +74,19 @@ __global__ void pack_planes_kernel(const uint32_t* __restrict__ canon,
 
 // One thread per packed half; see bcq_layout.h for the layout.
 __global__ void pack_scales_kernel(const uint16_t* __restrict__ src,
-                                   uint16_t* __restrict__ dst, int q, int N,
-                                   int G, int RBP, size_t total) {
+                                   uint16_t* __restrict__ dst, int q, int N, int G,
+                                   int RB, size_t total) {
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
     const int i = (int)(e % q);
     const size_t slot = e / q;
-    const int lane = (int)(slot & 31);
-    const int pass = (int)((slot >> 5) & 1);
-    const int kbi = (int)((slot >> 6) & 1);
-    const size_t rest = slot >> 7;
-    const size_t rb = rest % RBP;
-    const size_t chunk = rest / RBP;
+    const int pass = (int)(slot & 1);
+    const int lane = (int)((slot >> 1) & 31);
+    const size_t rest = slot >> 6;
+    const size_t rb = rest % RB;
+    const size_t kb = rest / RB;
     const size_t n = rb * kRowBlock + lane;
-    const size_t g = 2 * (chunk * kChunkBlocks + kbi) + ((lane >> 4) ^ pass);
+    const size_t g = 2 * kb + ((lane >> 4) ^ pass);
     uint16_t v = 0;
     if (n < (size_t)N && g < (size_t)G) v = src[(n * G + g) * q + i];
     dst[e] = v;
@@ -99,522 +95,735 @@ __global__ void pack_scales_kernel(const uint16_t* __restrict__ src,
 
 // ============================================================ LUT build
 
-// First 64 KiB boundary of the shared window above the CTA's low region.
-__device__ __forceinline__ uint32_t lut_base_of(uint32_t sbase) {
-  return (sbase & ~(kLutAlign - 1u)) + kLutAlign;
-}
-
-// Shared address of the table of slot s (= m * NKB + kb).
-template <int NKB>
-__device__ __forceinline__ uint32_t lut_table_addr(uint32_t lut_base, int m, int kbp) {
-  const int s = m * NKB + kbp;
-  return lut_base + (uint32_t)(s >> 1) * kLutTableBytes + (uint32_t)(s & 1) * 128u;
-}
-
-// Builds the tables of K-blocks [kb_first, kb_first + nkb) for the M rows of
-// x (fp16 [M][K]) into the LUT at lut_base, and the group sums into
-// gsum[m * 2 * NKB + g_local].  Columns beyond K read as zero.  All threads
-// of the first nwarps warps take part; the caller synchronises afterwards.
-//
-// Entry b of a chunk with values x0..x7 is sum_j (2 bit_j(b) - 1) x_j,
-// formed as L[b & 15] + H[b >> 4], L from x0..x3 and H from x4..x7.
-template <int M, int NKB>
-__device__ void build_lut_phase(const uint16_t* __restrict__ x, int K, int KB,
-                                int kb_first, int nkb, uint32_t lut_base, float* gsum,
-                                int nwarps) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int h = lane >> 4, c = lane & 15;
-  const int ntask = M * nkb * 8;  // (m, kb, eighth of the high nibbles)
-  for (int t = warp; t < ntask; t += nwarps) {
-    const int q8 = t & 7;
-    const int mk = t >> 3;
-    const int m = mk / nkb;
-    const int kbp = mk % nkb;
-    const int kbg = kb_first + kbp;
-    const int k = kbg * kKBlock + h * kGroup + c * 8;
-    float v[8];
-    if (kbg < KB && k < K) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)m * K + k));
-      const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+// Loads this lane's 8 activations of K-block kb for rows 0..M-1: the chunk
+// c = lane % 16 of group h = lane / 16 (zero past K).  x was written before
+// this grid started (or by a grid it waited for), so it is read through L2.
+template <int M>
+__device__ __forceinline__ void load_x(const uint16_t* x, int K, int kb, int lane,
+                                       uint4 (&xv)[M]) {
+  const int k = kb * kKBlock + (lane >> 4) * kGroup + (lane & 15) * 8;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = h2f((uint16_t)(r[e] & 0xFFFFu));
-        v[2 * e + 1] = h2f((uint16_t)(r[e] >> 16));
-      }
+  for (int m = 0; m < M; ++m) {
+    if (k < K) {
+      const uint16_t* p = x + (size_t)m * K + k;
+      asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(xv[m].x), "=r"(xv[m].y), "=r"(xv[m].z), "=r"(xv[m].w)
+                   : "l"(p));
     } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
-    }
-    // signed sums of pairs: index bit 0 -> sign of the first, bit 1 -> second
-    const float a3 = v[0] + v[1], a1 = v[0] - v[1];
-    const float a[4] = {-a3, a1, -a1, a3};
-    const float b3 = v[2] + v[3], b1 = v[2] - v[3];
-    const float bb[4] = {-b3, b1, -b1, b3};
-    // signed sum of x4..x7 for high nibble hi (computed per hi below)
-    const float x4 = v[4], x5 = v[5], x6 = v[6], x7 = v[7];
-    float L[16];
-#pragma unroll
-    for (int lo = 0; lo < 16; ++lo) L[lo] = a[lo & 3] + bb[lo >> 2];
-    const uint32_t tab = lut_table_addr<NKB>(lut_base, m, kbp) + (uint32_t)lane * 4u;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int hi = q8 * 2 + hh;
-      const float H = ((hi & 1) ? x4 : -x4) + ((hi & 2) ? x5 : -x5) +
-                      (((hi & 4) ? x6 : -x6) + ((hi & 8) ? x7 : -x7));
-#pragma unroll
-      for (int lo = 0; lo < 16; ++lo)
-        sts_f32(tab + (uint32_t)(hi * 16 + lo) * 256u, L[lo] + H);
+      xv[m] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  // group sums: one warp per (m, kb, group half)
-  const int ngs = M * nkb * 2;
-  for (int t = warp; t < ngs; t += nwarps) {
-    const int hh = t & 1;
-    const int m = (t >> 1) / nkb;
-    const int kbp = (t >> 1) % nkb;
-    const int kbg = kb_first + kbp;
-    const int k = kbg * kKBlock + hh * kGroup + lane * 4;
-    float s = 0.f;
-    if (kbg < KB && k < K) {
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + (size_t)m * K + k));
-      s = (h2f((uint16_t)(raw.x & 0xFFFFu)) + h2f((uint16_t)(raw.x >> 16))) +
-          (h2f((uint16_t)(raw.y & 0xFFFFu)) + h2f((uint16_t)(raw.y >> 16)));
-    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4& r, float (&v)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (lane == 0) gsum[m * 2 * NKB + kbp * 2 + hh] = s;
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = h2f((uint16_t)(w[e] & 0xFFFFu));
+    v[2 * e + 1] = h2f((uint16_t)(w[e] >> 16));
+  }
+}
+
+// Signed sums of the low nibble: L[lo] = sum_{j<4} (bit_j(lo) ? +v_j : -v_j).
+__device__ __forceinline__ void low_sums(const float (&v)[8], float (&L)[16]) {
+  const float a3 = v[0] + v[1], a1 = v[0] - v[1];
+  const float b3 = v[2] + v[3], b1 = v[2] - v[3];
+  const float a[4] = {-a3, a1, -a1, a3};
+  const float b[4] = {-b3, b1, -b1, b3};
+#pragma unroll
+  for (int lo = 0; lo < 16; ++lo) L[lo] = a[lo & 3] + b[lo >> 2];
+}
+
+// Signed sum of the high nibble hi over v4..v7.
+__device__ __forceinline__ float high_sum(const float (&v)[8], int hi) {
+  return (((hi & 1) ? v[4] : -v[4]) + ((hi & 2) ? v[5] : -v[5])) +
+         (((hi & 4) ? v[6] : -v[6]) + ((hi & 8) ? v[7] : -v[7]));
+}
+
+// Stores entries (hi0 * 16 + lo) (and, with HH = 2, (hi0 * 16 + 16 + lo)),
+// lo = LO..15, of one column: offsets are compile-time immediates.
+template <int LO, int HH>
+struct LutRows1 {
+  static __device__ __forceinline__ void run(uint32_t tb, const float (&L)[16], float H0,
+                                             float H1) {
+    sts_f32_at<(uint32_t)LO * 256u>(tb, L[LO] + H0);
+    if (HH > 1) sts_f32_at<(uint32_t)(16 + LO) * 256u>(tb, L[LO] + H1);
+    LutRows1<LO + 1, HH>::run(tb, L, H0, H1);
+  }
+};
+template <int HH>
+struct LutRows1<16, HH> {
+  static __device__ __forceinline__ void run(uint32_t, const float (&)[16], float, float) {}
+};
+
+// The same for entry pairs (two activation rows).
+template <int LO, int HH>
+struct LutRows2 {
+  static __device__ __forceinline__ void run(uint32_t tb, const float (&L0)[16],
+                                             const float (&L1)[16], float H00, float H01,
+                                             float H10, float H11) {
+    sts_f32x2_at<(uint32_t)LO * 256u>(tb, L0[LO] + H00, L1[LO] + H10);
+    if (HH > 1) sts_f32x2_at<(uint32_t)(16 + LO) * 256u>(tb, L0[LO] + H01, L1[LO] + H11);
+    LutRows2<LO + 1, HH>::run(tb, L0, L1, H00, H01, H10, H11);
+  }
+};
+template <int HH>
+struct LutRows2<16, HH> {
+  static __device__ __forceinline__ void run(uint32_t, const float (&)[16], const float (&)[16],
+                                             float, float, float, float) {}
+};
+
+// Builds the table of one K-block at shared address lut (layout in
+// bcq_layout.h): 16 / HH warps of the caller each write the entries of high
+// nibbles HH * warp .. HH * warp + HH - 1 for all 32 columns (lane = column).
+// Entry b of a column with activations v0..v7 is sum_j (2 bit_j(b) - 1) v_j,
+// formed as L[b & 15] + H[b >> 4].  Also returns the group sums of this
+// lane's pass-0 group (gs[m][0]) and of the other group (gs[m][1]).  The
+// caller synchronises before the table is read.
+template <int M, int HH>
+__device__ __forceinline__ void build_lut(const uint4 (&xv)[M], int slot, uint32_t lut,
+                                          int warp, int lane, float (&gs)[M][2]) {
+  float v[M][8];
+#pragma unroll
+  for (int m = 0; m < M; ++m) unpack8(xv[m], v[m]);
+  float L[M][16];
+#pragma unroll
+  for (int m = 0; m < M; ++m) low_sums(v[m], L[m]);
+  const int hi0 = warp * HH;
+  const int hi1 = HH > 1 ? hi0 + 1 : hi0;
+  if (M == 1) {
+    const uint32_t tb = lut + (uint32_t)(hi0 * 16) * 256u + (uint32_t)slot * 128u +
+                        (uint32_t)lane * 4u;
+    LutRows1<0, HH>::run(tb, L[0], high_sum(v[0], hi0), high_sum(v[0], hi1));
+  } else {
+    const uint32_t tb = lut + (uint32_t)(hi0 * 16) * 256u + (uint32_t)lane * 8u;
+    LutRows2<0, HH>::run(tb, L[0], L[M - 1], high_sum(v[0], hi0), high_sum(v[0], hi1),
+                         high_sum(v[M - 1], hi0), high_sum(v[M - 1], hi1));
+  }
+  // group sums: lanes 0-15 hold group A, 16-31 group B
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    float s = ((v[m][0] + v[m][1]) + (v[m][2] + v[m][3])) +
+              ((v[m][4] + v[m][5]) + (v[m][6] + v[m][7]));
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    gs[m][0] = s;
+    gs[m][1] = __shfl_xor_sync(0xFFFFFFFFu, s, 16);
   }
 }
 
 // ============================================================ GEMV
 
-// prmt selectors for byte j of a plane word: result byte 0 <- column offset
+// prmt selectors for byte j of a plane word: result byte 0 <- column byte
 // (byte j & 1 of the column register), byte 1 <- plane byte j, bytes 2-3 <-
-// bytes 2-3 of the column register (the upper half of lut_base).  The result
-// is lut_base + b * 256 + column * 4.
+// bytes 2-3 of the column register (zero).  The result is b * 256 + column
+// byte, the table offset of entry b of that column.
 __device__ __forceinline__ constexpr uint32_t sel_of(int j) {
   return (4u + (uint32_t)(j & 1)) | ((uint32_t)j << 4) | 0x7600u;
 }
 
-template <int M, int KBI, int MM>
-struct LutAcc {
-  static __device__ __forceinline__ void run(uint32_t a, float (&p)[M]) {
-    constexpr int s = MM * kChunkBlocks + KBI;
-    constexpr uint32_t off = (uint32_t)(s / 2) * kLutTableBytes + (uint32_t)(s % 2) * 128u;
-    p[MM] += lds_f32<off>(a);
-    LutAcc<M, KBI, MM + 1>::run(a, p);
+// Column registers of this lane: cr0[u][q] holds the column bytes of bytes
+// 2q and 2q + 1 of word u in pass 0; cr1 the same for pass 1 (other group).
+template <int M>
+__device__ __forceinline__ void column_regs(int lane, uint32_t (&cr0)[4][2],
+                                            uint32_t (&cr1)[4][2]) {
+  const uint32_t h0 = (uint32_t)(lane >> 4);
+  const uint32_t flip = M == 1 ? 0x4040u : 0x8080u;  // group bit of each byte
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t r = 0;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t c = (uint32_t)((4 * u + 2 * q + e + lane) & 15);
+        const uint32_t col = h0 * 16u + c;
+        r |= (M == 1 ? col * 4u : col * 8u) << (8 * e);
+      }
+      cr0[u][q] = r;
+      cr1[u][q] = r ^ flip;
+    }
   }
-};
-template <int M, int KBI>
-struct LutAcc<M, KBI, M> {
-  static __device__ __forceinline__ void run(uint32_t, float (&)[M]) {}
+}
+
+// Sum of the 16 table entries one lane's 16 plane bytes select (M = 1).
+__device__ __forceinline__ float plane_sum1(const uint4& w, const uint32_t (&cr)[4][2]) {
+  const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      s[j] += lds_f32<kDynBase>(prmt(wd[u], cr[u][j >> 1], sel_of(j)));
+  }
+  return (s[0] + s[1]) + (s[2] + s[3]);
+}
+
+// The same for two activation rows (entries are pairs).
+__device__ __forceinline__ void plane_sum2(const uint4& w, const uint32_t (&cr)[4][2],
+                                           float& r0, float& r1) {
+  const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+  float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 e = lds_f32x2<kDynBase>(prmt(wd[u], cr[u][j >> 1], sel_of(j)));
+      s0[j & 1] += e.x;
+      s1[j & 1] += e.y;
+    }
+  }
+  r0 = s0[0] + s0[1];
+  r1 = s1[0] + s1[1];
+}
+
+// Scales and offsets of one unit for this lane: a[m][r] holds halves
+// 2r, 2r + 1 of the lane's 2P values (pass 0: planes 0..P-1, then pass 1);
+// z holds the offsets of the pass-0 and pass-1 groups.
+template <int M, int P>
+struct ScaleSet {
+  uint32_t a[M][P];
+  uint32_t z;
 };
 
-// Lookup-accumulate of one pass of one K-block of 32 rows.  planes_at is
-// this lane's 16 bytes of plane 0; plane i is plane_stride bytes further.
-//   acc[m] += sum_{i < p_load} ae[m][i] * P_i[m]  +  zv * gs[m]
-template <int M, int KBI>
-__device__ __forceinline__ void unit_body(uint32_t planes_at, uint32_t plane_stride,
-                                          int p_load, const uint32_t (&cr)[4][2],
-                                          const float (&ae)[M][4], float zv,
-                                          const float (&gs)[M], float (&acc)[M]) {
+template <int M, int P, bool MIXED>
+__device__ __forceinline__ void load_scales(const GemvParams& prm, int kb, int rb, int lane,
+                                            ScaleSet<M, P>& s) {
+  const size_t e = ((size_t)kb * prm.RB + rb) * kRowBlock + lane;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (i < p_load) {
-      const uint4 wv = lds_v4(planes_at + (uint32_t)i * plane_stride);
-      const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-      float pa[M], pb[M];
+  for (int m = 0; m < M; ++m) {
+    if (!MIXED) {
+      if (m > 0) {
 #pragma unroll
-      for (int m = 0; m < M; ++m) pa[m] = pb[m] = 0.f;
+        for (int r = 0; r < P; ++r) s.a[m][r] = s.a[0][r];  // same precision, same scales
+        continue;
+      }
+      const uint16_t* a = prm.alpha[0] + e * (2 * P);
+      if (P == 1) {
+        s.a[m][0] = ldg_nc_u32(a);
+      } else if (P == 2) {
+        const uint2 r = ldg_nc_v2(a);
+        s.a[m][0] = r.x;
+        s.a[m][P > 1 ? 1 : 0] = r.y;
+      } else if (P == 3) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+        for (int r = 0; r < P; ++r) s.a[m][r] = ldg_nc_u32(a + 2 * r);
+      } else {
+        const uint4 r = ldg_nc_v4(a);
+        s.a[m][0] = r.x;
+        s.a[m][P > 1 ? 1 : 0] = r.y;
+        s.a[m][P > 2 ? 2 : 0] = r.z;
+        s.a[m][P > 3 ? 3 : 0] = r.w;
+      }
+    } else {
+      const int q = prm.q[m];
+      const uint16_t* a = prm.alpha[m] + e * (size_t)(2 * q);
 #pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-          const uint32_t a0 = prmt(wd[u], cr[u][j >> 1], sel_of(j));
-          const uint32_t a1 = prmt(wd[u], cr[u][j >> 1], sel_of(j + 1));
-          LutAcc<M, KBI, 0>::run(a0, pa);
-          LutAcc<M, KBI, 0>::run(a1, pb);
+      for (int r = 0; r < P; ++r) s.a[m][r] = 0u;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+          const int hidx = pass * P + i;
+          const uint32_t v = i < q ? (uint32_t)ldg_nc_u16(a + pass * q + i) : 0u;
+          s.a[m][hidx >> 1] |= v << (16 * (hidx & 1));
         }
       }
-#pragma unroll
-      for (int m = 0; m < M; ++m) acc[m] = fmaf(ae[m][i], pa[m] + pb[m], acc[m]);
     }
   }
-#pragma unroll
-  for (int m = 0; m < M; ++m) acc[m] = fmaf(zv, gs[m], acc[m]);
+  s.z = prm.z ? ldg_nc_u32(prm.z + e * 2) : 0u;
 }
 
-// Reads q scale values of this lane from a staged span of packed scales.
-__device__ __forceinline__ void read_scales(uint32_t at, int q, float (&a)[4]) {
-  a[0] = a[1] = a[2] = a[3] = 0.f;
-  if (q == 4) {
-    uint32_t v0, v1;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(at));
-    a[0] = h2f((uint16_t)(v0 & 0xFFFFu));
-    a[1] = h2f((uint16_t)(v0 >> 16));
-    a[2] = h2f((uint16_t)(v1 & 0xFFFFu));
-    a[3] = h2f((uint16_t)(v1 >> 16));
-  } else if (q == 2) {
-    uint32_t v0;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v0) : "r"(at));
-    a[0] = h2f((uint16_t)(v0 & 0xFFFFu));
-    a[1] = h2f((uint16_t)(v0 >> 16));
+template <int M, int P>
+__device__ __forceinline__ void zero_scales(ScaleSet<M, P>& s) {
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int r = 0; r < P; ++r) s.a[m][r] = 0u;
+  s.z = 0u;
+}
+
+__device__ __forceinline__ float half_at(uint32_t r, int hi) {
+  return h2f((uint16_t)(hi ? (r >> 16) : (r & 0xFFFFu)));
+}
+
+// The units of one CTA: [u0, u1) in kb-major order, cut into groups: the
+// row-blocks of one K-block inside one row group (at most kRowGroup).  When
+// the CTAs divide evenly among the K-blocks, each CTA keeps to one K-block;
+// otherwise the units are shared out evenly (the first U mod C CTAs take one
+// more).
+struct CtaRange {
+  int u0, u1, NG, kb0, kb_last;
+};
+
+__device__ __forceinline__ void make_range(const GemvParams& p, CtaRange& R) {
+  const int c = (int)blockIdx.x;
+  if (p.C >= p.KB && p.C % p.KB == 0) {
+    // whole K-blocks: C / KB CTAs share the row-blocks of each K-block
+    const int cpk = p.C / p.KB, kb = c / cpk, j = c - kb * cpk;
+    const int q = p.RB / cpk, r = p.RB % cpk;
+    R.u0 = kb * p.RB + j * q + min(j, r);
+    R.u1 = R.u0 + q + (j < r ? 1 : 0);
   } else {
-    uint16_t h0, h1 = 0, h2 = 0;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h0) : "r"(at));
-    if (q == 3) {
-      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h1) : "r"(at + 2u));
-      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h2) : "r"(at + 4u));
-    }
-    a[0] = h2f(h0);
-    a[1] = h2f(h1);
-    a[2] = h2f(h2);
+    const int q = p.U / p.C, r = p.U % p.C;
+    R.u0 = c * q + min(c, r);
+    R.u1 = R.u0 + q + (c < r ? 1 : 0);
+  }
+  int ng = 0;
+  for (int u = R.u0; u < R.u1;) {
+    const int kb = u / p.RB;
+    const int end = min(R.u1, (kb + 1) * p.RB);
+    const int a = u - kb * p.RB, b = end - kb * p.RB;  // row-blocks [a, b) of kb
+    ng += (b + kRowGroup - 1) / kRowGroup - a / kRowGroup;
+    u = end;
+  }
+  R.NG = ng;
+  R.kb0 = R.u0 / p.RB;
+  R.kb_last = R.u1 > R.u0 ? (R.u1 - 1) / p.RB : R.kb0;
+}
+
+// Walks the groups of a CTA in order: K-block kb, first row-block rb0, n
+// row-blocks (all in row group rb0 / kRowGroup); seg_end bounds the
+// row-blocks of kb inside the CTA's range.
+struct GroupCursor {
+  int kb, rb0, n, seg_end;
+};
+
+__device__ __forceinline__ void cursor_init(GroupCursor& c, int u0, int u1, int RB) {
+  c.kb = u0 / RB;
+  c.rb0 = u0 - c.kb * RB;
+  c.seg_end = min(RB, u1 - c.kb * RB);
+  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
+}
+
+__device__ __forceinline__ void cursor_next(GroupCursor& c, int u1, int RB) {
+  c.rb0 += c.n;
+  if (c.rb0 >= c.seg_end) {
+    ++c.kb;
+    c.rb0 = 0;
+    c.seg_end = min(RB, u1 - c.kb * RB);
+  }
+  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
+}
+
+// Waits for phase `parity` of a stage barrier: a non-blocking test first
+// (the common case: the stage has landed), then bounded waiting that gives
+// up when the CTA aborts.
+__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity,
+                                           volatile int* abort_flag,
+                                           unsigned long long limit_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+  while (true) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
-// Both passes of K-block KBI of the chunk for this warp's row-block j of
-// the task staged at st.
-template <int M, int KBI>
-__device__ __forceinline__ void task_kbi(const GemvParams& P, uint32_t st, int j, int lane,
-                                         uint32_t plane_stride, const uint32_t (&cr0)[4][2],
-                                         const uint32_t (&cr1)[4][2], const float* gsum,
-                                         float (&acc)[M]) {
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int sub = (KBI * 2 + pass) * 32 + lane;
-    float ae[M][4];
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const int d = P.d_of[m];
-      const int q = P.q_of[d];
-      read_scales(st + P.st_scale[d] + (uint32_t)(j * 256 * q + sub * q * 2), q, ae[m]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (i >= P.p_m[m]) ae[m][i] = 0.f;
-    }
-    float zv = 0.f;
-    if (P.has_z) {
-      uint16_t zh;
-      asm volatile("ld.shared.u16 %0, [%1];"
-                   : "=h"(zh)
-                   : "r"(st + P.st_scale[2] + (uint32_t)(j * 256 + sub * 2)));
-      zv = h2f(zh);
-    }
-    const int h = (lane >> 4) ^ pass;
-    float gs[M];
-#pragma unroll
-    for (int m = 0; m < M; ++m) gs[m] = gsum[m * 4 + KBI * 2 + h];
-    uint32_t cr[4][2];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      cr[u][0] = pass ? cr1[u][0] : cr0[u][0];
-      cr[u][1] = pass ? cr1[u][1] : cr0[u][1];
-    }
-    const uint32_t at = st + (uint32_t)(j * kPlaneChunkBytes + KBI * 1024 +
-                                        pass * kUnitBytesPerPlane + lane * 16);
-    unit_body<M, KBI>(at, plane_stride, P.p_load, cr, ae, zv, gs, acc);
-  }
-}
+template <int J>
+struct Slot {
+  static constexpr int value = J;
+};
 
-__device__ __forceinline__ void consumer_sync(int nthreads) {
-  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
-// Stage s address: offsets with bit 31 set count from the end of the LUT,
-// the others from the dynamic shared memory base.
-__device__ __forceinline__ uint32_t stage_addr(const GemvParams& P, int s, uint32_t sbase,
-                                               uint32_t lut_end) {
-  const uint32_t o = P.stage_off[s];
-  return (o & 0x80000000u) ? lut_end + (o & 0x7FFFFFFFu) : sbase + o;
-}
-
-// One CTA: K-range [c0, c1) in chunks of 512 columns (one LUT phase per chunk)
-// times the row-blocks of its cluster.  Warps 0..W-1 consume, warp W produces.
-// A task is T consecutive row-blocks of one chunk; its planes, scales and
-// offsets arrive by bulk copy in one ring stage; consumer group (task mod G)
-// takes it, one row-block per warp.
-template <int M>
-__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + kMaxProducerWarps), 1)
-    gemv_lut_kernel(const __grid_constant__ GemvParams P) {
-  extern __shared__ __align__(128) unsigned char smem[];
+// One CTA per SM: units [u0, u1) of the launch in kb-major order.  Warps
+// 0..15 consume, in two teams of 8 that take alternate groups; the NP warps
+// after them produce.  Stage g of the CTA holds the P planes of group g
+// (plane i at i * 8 KiB, row-block rb0 + w at w KiB); it lands in ring slot
+// g mod D and is read by the team of its group (team warp w takes
+// row-block rb0 + w).  The teams share the lookup table: each K-block's
+// table is built by all 16 warps together.
+//   M      activation rows of the launch (1 or 2)
+//   P      planes streamed (the largest precision among the rows)
+//   MIXED  rows may use precisions below P (scales loaded per row)
+template <int M, int P, bool MIXED>
+__global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
+    gemv_lut_kernel(const __grid_constant__ GemvParams prm) {
+  extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int W = P.W, D = P.D, NP = P.NP;
-  constexpr int T = kRowGroup;  // row-blocks per task: one per warp of a group
-  const int G = W / T;
+  const int D = prm.D, NP = prm.NP, RB = prm.RB;
+  constexpr uint32_t kStage = gemv_stage_bytes(P);
+  const uint32_t full0 = sbase + gemv_off_bar(D, P);
+  const uint32_t empty0 = full0 + 8u * (uint32_t)D;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + gemv_off_misc(D, P));
+  int* nlist = reinterpret_cast<int*>(smem + gemv_off_misc(D, P) + 4);
+  int* list = reinterpret_cast<int*>(smem + gemv_off_misc(D, P) + 16);
+  constexpr int kConsumers = kConsumerWarps * 32;
 
-  const int S = P.S;
-  const int rank = (int)(blockIdx.x % (unsigned)S);
-  const int cl = (int)(blockIdx.x / (unsigned)S);
-  const int rg0 = cl * P.rg_base + (cl < P.rg_rem ? cl : P.rg_rem);
-  const int nrg = P.rg_base + (cl < P.rg_rem ? 1 : 0);
-  const int rb0 = rg0 * kRowGroup;
-  const int nrb = nrg * kRowGroup;
-  const int c0 = (int)(((long long)rank * P.KC) / S);
-  const int c1 = (int)(((long long)(rank + 1) * P.KC) / S);
-  const int nphase = c1 - c0;
-  const int ntask = nrg;
-  const int ktot = nphase * ntask;
-
-  float* accr = reinterpret_cast<float*>(smem + P.off_acc);    // [M][part_rows]
-  float* gsum = reinterpret_cast<float*>(smem + P.off_gsum);   // [M][4]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P.off_flag);
-  const uint32_t full0 = sbase + P.off_bar;                    // D full barriers
-  const uint32_t empty0 = full0 + 8u * kMaxStages;             // D empty barriers
-  const uint32_t lut_base = lut_base_of(sbase);
-  const uint32_t lut_end = lut_base + P.lut_bytes;
-
-  // The LUT and the stages must lie inside this CTA's dynamic shared memory
-  // (and a ring depth that is a multiple of the consumer groups: see the
-  // stage rule in the planner).
-  const uint32_t pad = lut_base - sbase;
-  const bool layout_ok = pad >= P.low_bytes && pad + P.lut_bytes <= P.dyn_bytes &&
-                         D >= 1 && D <= kMaxStages && NP >= 1 && NP <= kMaxProducerWarps &&
-                         D % G == 0 && D % NP == 0 && W % T == 0 && W <= kMaxConsumerWarps;
-  const uint32_t recv_bar = full0 + 16u * kMaxStages;
-  const int rows_c = nrb * kRowBlock;
-  const int own0 = rank * P.own_rows;
-  const int own_n = max(0, min(rows_c, own0 + P.own_rows) - own0);
-  const int nthreads = (W + NP) * 32;
-  if (warp >= W) {
-    // ------------------------------------------------------------ producers
-    // Producer pw issues tasks k = pw, pw + NP, ... (their stages
-    // s = k mod D are its own).  Barrier set-up (one barrier per lane of
-    // producer 0) overlaps the consumers' LUT build; everyone waits for it
-    // (named barrier 2) before the first barrier access.
-    const int pw = warp - W;
-    if (pw == 0) {
-      if (lane == 0) {
-        *abort_flag = layout_ok ? 0 : 1;
-        if (!layout_ok) record_error(&g_device_error, BCQ_ERR_UNSUPPORTED);
-      }
-      if (layout_ok) {
-        if (lane < D) {
-          mbar_init(full0 + 8u * lane, 1);
-          mbar_init(empty0 + 8u * lane, (uint32_t)T);
-        }
-        if (lane == 31) {
-          mbar_init(recv_bar, 1);
-          mbar_arrive_expect_tx(recv_bar, (uint32_t)((S - 1) * M * own_n * 4));
-        }
-        fence_mbar_init();
-      }
-      __syncwarp();
-      asm volatile("bar.arrive 2, %0;" ::"r"(nthreads) : "memory");
-    } else {
-      asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
+  // The table is addressed through load immediates: the dynamic shared
+  // memory must start where they assume.  A stage's team must have consumed
+  // the stage D earlier (D even: teams alternate), and each producer refills
+  // only its own slots (D a multiple of NP).
+  const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 &&
+                      D % NP == 0 && D % 2 == 0 &&
+                      (int)blockDim.x == 32 * (kConsumerWarps + NP);
+  if (warp == 0) {
+    if (cfg_ok && lane < D) {  // one lane per ring slot
+      mbar_init(full0 + 8u * lane, 1);
+      mbar_init(empty0 + 8u * lane, kTeamWarps);
     }
-    if (!P.early_weights) grid_dependency_wait();
-    const int nreq = 1 + P.nq + P.has_z;
-    const uint32_t stage_bytes = P.stage_bytes;
-    int issued = 0;  // one past the last task this producer issued
-    for (int k = pw; layout_ok && k < ktot; k += NP) {
-      const int s = k % D;
-      bool ok = true;
-      if (k >= D && lane == 0)
-        ok = mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((k / D) - 1) & 1), P.timeout_ns);
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      if (!ok) {
-        if (lane == 0) {
+    if (lane == 0) {
+      *abort_flag = cfg_ok ? 0 : 1;
+      if (!cfg_ok) record_error(&g_device_error, BCQ_ERR_UNSUPPORTED);
+    }
+    if (cfg_ok) fence_mbar_init();
+  }
+  __syncthreads();
+  launch_dependents();
+  if (*abort_flag) return;  // set before the barrier: uniform
+
+  CtaRange R;
+  make_range(prm, R);
+
+  if (warp >= kConsumerWarps) {
+    // ------------------------------------------------------------ producers
+    // Producer pw issues stages (groups) k = pw, pw + NP, ...; with D a
+    // multiple of NP it alone refills its ring slots, so the empty-barrier
+    // phase it waits for is never two phases behind.  A whole row group is
+    // one bulk copy of its first P planes; a partial one (at the ends of the
+    // CTA's range) one copy per plane.
+    const int pw = warp - kConsumerWarps;
+    if (!prm.early_weights) grid_dependency_wait();
+    if (lane == 0) {
+      int issued = 0;
+      GroupCursor gc;
+      cursor_init(gc, R.u0, R.u1, RB);
+      for (int k = 0; k < R.NG; ++k, cursor_next(gc, R.u1, RB)) {
+        if (k % NP != pw) continue;
+        const int s = k % D;
+        if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((k / D) - 1) & 1),
+                                         prm.timeout_ns)) {
           record_error(&g_device_error, BCQ_ERR_TIMEOUT);
           *abort_flag = 1;
         }
-        break;
-      }
-      if (*abort_flag) break;
-      const int ph = k / ntask;
-      const int t = k % ntask;
-      const size_t chunk = (size_t)(c0 + ph);
-      const size_t rg = (size_t)(rg0 + t);
-      const uint32_t dst = stage_addr(P, s, sbase, lut_end);
-      if (lane == 0) mbar_arrive_expect_tx(full0 + 8u * s, stage_bytes);
-      __syncwarp();
-      // one bulk copy per lane, all issued by one instruction: the first
-      // p_load planes of the row group (contiguous), the scales of each
-      // distinct precision, the offsets
-      if (lane < nreq) {
-        const void* src;
-        uint32_t to, bytes;
-        if (lane == 0) {
-          src = P.planes + ((chunk * P.RBG + rg) * P.p_H) * (kRowGroup * kPlaneChunkBytes / 4);
-          to = 0;
-          bytes = (uint32_t)P.p_load * kRowGroup * kPlaneChunkBytes;
-        } else if (lane <= P.nq) {
-          const int d = lane - 1;
-          const int q = P.q_of[d];
-          src = P.scale[d] + (chunk * P.RBG + rg) * (512 * q);
-          to = P.st_scale[d];
-          bytes = 1024u * q;
+        if (*abort_flag) break;
+        const uint32_t bar = full0 + 8u * s;
+        const uint32_t dst = sbase + kLutBytes + (uint32_t)s * kStage;
+        const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
+        const uint32_t* src = prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H *
+                                               (kRowGroup * kWordsPerUnitPlane);
+        mbar_arrive_expect_tx(bar, (uint32_t)(P * gc.n) * kUnitPlaneBytes);
+        if (gc.n == kRowGroup) {
+          bulk_g2s(dst, src, kStage, bar);
         } else {
-          src = P.scale[2] + (chunk * P.RBG + rg) * 512;
-          to = P.st_scale[2];
-          bytes = 1024u;
+#pragma unroll
+          for (int i = 0; i < P; ++i)
+            bulk_g2s(dst + (uint32_t)i * kPlaneGroupBytes,
+                     src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
+                     (uint32_t)gc.n * kUnitPlaneBytes, bar);
         }
-        bulk_g2s(dst + to, src, bytes, full0 + 8u * s);
+        issued = k + 1;
       }
-      issued = k + 1;
-    }
-    if (P.early_weights) grid_dependency_wait();
-    launch_dependents();
-    if (S > 1) cluster_arrive_relaxed();  // off the path to the first copies
-    // copies still in flight must land before the CTA releases its memory
-    if (lane == 0) {
-      for (int s = pw; s < D; s += NP) {
-        if (s >= issued) break;
+      // every copy this warp issued lands before the CTA may exit
+      for (int s = pw; s < D && s < issued; s += NP) {
         const int klast = issued - 1 - ((issued - 1 - s) % D);
-        (void)mbar_wait_bounded(full0 + 8u * s, (uint32_t)((klast / D) & 1), P.timeout_ns);
+        (void)mbar_wait_bounded(full0 + 8u * s, (uint32_t)((klast / D) & 1), prm.timeout_ns);
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ consumers
-    grid_dependency_wait();
-    const int grp = warp / T;
-    const int j = warp % T;
-    // per-lane column registers for the two passes: [u][j/2] holds the column
-    // offsets of bytes 2*(j/2), 2*(j/2)+1 and lut_base >> 16
-    uint32_t cr0[4][2], cr1[4][2];
-    {
-      const uint32_t hi = lut_base & 0xFFFF0000u;
-      const uint32_t h0 = (uint32_t)(lane >> 4), h1 = h0 ^ 1u;
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  grid_dependency_wait();  // x, y and the workspace may belong to earlier work
+  const int team = warp / kTeamWarps;
+  const int tw = warp % kTeamWarps;  // row-block of a stage
+  GroupCursor gc;                    // this team's next group
+  cursor_init(gc, R.u0, R.u1, RB);
+  uint4 xv[M];                       // activations of the first table, first of all
+  load_x<M>(prm.x, prm.K, gc.kb, lane, xv);
+  uint32_t cr0[4][2], cr1[4][2];
+  column_regs<M>(lane, cr0, cr1);
+  int cr_slot = 0;
+  int cur_kb = -1, xn_kb = -1;
+  uint4 xn[M];
+  float gs[M][2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+  for (int m = 0; m < M; ++m) {
+    xn[m] = make_uint4(0u, 0u, 0u, 0u);
+    gs[m][0] = gs[m][1] = 0.f;
+  }
+  int g = team;  // team t takes groups t, t + 2, ...
+  if (team) cursor_next(gc, R.u1, RB);
+  // ring position of the team's next stage (stage = group; D >= 2)
+  int s = team;
+  uint32_t ph = 0;
+  // Scales and offsets are loaded PF team-groups ahead into pf[j mod PF];
+  // the loop is unrolled by PF so no register with a load in flight is
+  // ever copied.
+  constexpr int PF = 2;
+  ScaleSet<M, P> pf[PF];
+  GroupCursor pc = gc;
+  int gp = g;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t r0 = hi, r1 = hi;
+  for (int j = 0; j < PF; ++j) {
+    zero_scales(pf[j]);
+    if (gp < R.NG && tw < pc.n) load_scales<M, P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, pf[j]);
+    cursor_next(pc, R.u1, RB);
+    cursor_next(pc, R.u1, RB);
+    gp += 2;
+  }
+  const size_t part_stride = (size_t)RB * kRowBlock;
+  // Results of a group are used (offset term, store) only after the team's
+  // next group has issued its first lookups, so no warp stalls on its own
+  // loads: acc[J] / pend*[J] hold the group in slot J until then.
+  float acc[PF][M];
+  bool pend[PF];
+  int pend_row[PF] = {0, 0}, pend_kb[PF] = {0, 0};
+  uint32_t pend_z[PF] = {0u, 0u};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const uint32_t c = (uint32_t)((4 * u + 2 * q + e + lane) & 15);
-            r0 |= ((h0 * 16u + c) * 4u) << (8 * e);
-            r1 |= ((h1 * 16u + c) * 4u) << (8 * e);
-          }
-          cr0[u][q] = r0;
-          cr1[u][q] = r1;
+  for (int j = 0; j < PF; ++j) pend[j] = false;
+
+  auto finish = [&](auto slot_tag) {
+    constexpr int J = decltype(slot_tag)::value;
+    if (!pend[J]) return;
+    pend[J] = false;
+    if (*abort_flag) return;
+    const float z0 = half_at(pend_z[J], 0), z1 = half_at(pend_z[J], 1);
+    float r[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) r[m] = fmaf(z0, gs[m][0], fmaf(z1, gs[m][1], acc[J][m]));
+    const int row = pend_row[J];
+    if (prm.KB > 1) {
+#pragma unroll
+      for (int m = 0; m < M; ++m)
+        prm.part[((size_t)pend_kb[J] * M + m) * part_stride + (size_t)row] = r[m];
+    } else if (row < prm.N) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) prm.y[(size_t)m * prm.N + row] = f2h_rn(r[m]);
+    }
+  };
+
+  // Tables of every K-block up to kbt, in order; all 16 consumer warps take
+  // part in each (the teams meet at the barriers), so both teams go through
+  // the same K-blocks even when one has no group in some of them.
+  auto advance_tables = [&](int kbt) {
+    if (cur_kb >= kbt) return;
+    finish(Slot<0>{});  // group sums change with the table
+    finish(Slot<1>{});
+    while (cur_kb < kbt) {
+      const int kbn = cur_kb < 0 ? R.kb0 : cur_kb + 1;
+      if (cur_kb >= 0) {
+        if (xn_kb == kbn) {
+#pragma unroll
+          for (int m = 0; m < M; ++m) xv[m] = xn[m];
+        } else {
+          load_x<M>(prm.x, prm.K, kbn, lane, xv);
         }
       }
-    }
-    const uint32_t plane_stride = (uint32_t)T * kPlaneChunkBytes;
-    if (nphase == 0) {
-      asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
-      if (S > 1) cluster_arrive_relaxed();
-    }
-    for (int ph = 0; ph < nphase; ++ph) {
-      if (layout_ok)
-        build_lut_phase<M, kChunkBlocks>(P.x, P.K, P.KB, (c0 + ph) * kChunkBlocks,
-                                         kChunkBlocks, lut_base, gsum, W);
-      if (ph == 0) {
-        asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");  // barriers ready
-        if (S > 1) cluster_arrive_relaxed();
+      if (kbn < R.kb_last) {
+        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn);
+        xn_kb = kbn + 1;
       }
-      consumer_sync(W * 32);
-      for (int t = grp; layout_ok && t < ntask; t += G) {
-        if (*abort_flag) break;
-        const int k = ph * ntask + t;
-        const int s = k % D;
-        const bool ok = mbar_wait_bounded(full0 + 8u * s, (uint32_t)((k / D) & 1), P.timeout_ns);
-        if (!ok) {
-          if (lane == 0) {
-            record_error(&g_device_error, BCQ_ERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          break;
-        }
-        const int rbl = t * T + j;
-        if (rbl < nrb) {
-          const uint32_t st = stage_addr(P, s, sbase, lut_end);
-          float acc[M];
+      // M = 2 has one table: every warp must be done with the old one.
+      // M = 1 alternates two slots; the one rebuilt was last read two
+      // K-blocks ago, before the previous build's barrier.
+      if (M == 2 && cur_kb >= 0) named_barrier_sync(1, kConsumers);
+      const int slot = M == 1 ? (kbn & 1) : 0;
+      build_lut<M, 1>(xv, slot, sbase, warp, lane, gs);
+      if (M == 1 && slot != cr_slot) {
 #pragma unroll
-          for (int m = 0; m < M; ++m) acc[m] = 0.f;
-          task_kbi<M, 0>(P, st, j, lane, plane_stride, cr0, cr1, gsum, acc);
-          task_kbi<M, 1>(P, st, j, lane, plane_stride, cr0, cr1, gsum, acc);
+        for (int u = 0; u < 4; ++u)
 #pragma unroll
-          for (int m = 0; m < M; ++m) {
-            float* dstp = accr + (size_t)m * P.part_rows + rbl * kRowBlock + lane;
-            *dstp = (ph == 0 ? 0.f : *dstp) + acc[m];
+          for (int q = 0; q < 2; ++q) {
+            cr0[u][q] ^= 0x8080u;
+            cr1[u][q] ^= 0x8080u;
           }
+        cr_slot = slot;
+      }
+      named_barrier_sync(1, kConsumers);
+      cur_kb = kbn;
+    }
+  };
+
+  auto group = [&](auto slot_tag) {
+    constexpr int J = decltype(slot_tag)::value;
+    constexpr int JP = (J + PF - 1) % PF;  // slot of the team's previous group
+    advance_tables(gc.kb);
+    const bool active = tw < gc.n;
+    const ScaleSet<M, P>& sc = pf[J];
+#pragma unroll
+    for (int m = 0; m < M; ++m) acc[J][m] = 0.f;
+    const bool ok = wait_stage(full0 + 8u * s, ph, abort_flag, prm.timeout_ns);
+    if (!ok && lane == 0 && *abort_flag == 0) {
+      record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    const bool live = ok && active;
+    const uint32_t st = sbase + kLutBytes + (uint32_t)s * kStage +
+                        (uint32_t)tw * kUnitPlaneBytes + (uint32_t)lane * 16u;
+    // planes in batches of two: their plane words, then the lookups of both;
+    // the stage is released once all its words are in registers
+#pragma unroll
+    for (int i0 = 0; i0 < P; i0 += 2) {
+      constexpr int kB = 2;
+      uint4 w[kB][2];
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        if (i0 + t < P && live) {
+          w[t][0] = lds_v4(st + (uint32_t)(i0 + t) * kPlaneGroupBytes);
+          w[t][1] = lds_v4(st + (uint32_t)(i0 + t) * kPlaneGroupBytes + 512u);
+        } else {
+          w[t][0] = w[t][1] = make_uint4(0u, 0u, 0u, 0u);
         }
+      }
+      if (i0 + kB >= P) {
         __syncwarp();
         if (lane == 0) mbar_arrive_cta(empty0 + 8u * s);
       }
-      consumer_sync(W * 32);
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const int i = i0 + t;
+        if (i < P && live) {
+          // half (pass * P + i) of the lane's scales of row m
+          if (M == 1) {
+            const float p0 = plane_sum1(w[t][0], cr0);
+            const float p1 = plane_sum1(w[t][1], cr1);
+            acc[J][0] = fmaf(half_at(sc.a[0][i >> 1], i & 1), p0, acc[J][0]);
+            acc[J][0] = fmaf(half_at(sc.a[0][(P + i) >> 1], (P + i) & 1), p1, acc[J][0]);
+          } else {
+            float a0, a1, b0, b1;
+            plane_sum2(w[t][0], cr0, a0, a1);
+            plane_sum2(w[t][1], cr1, b0, b1);
+            acc[J][0] = fmaf(half_at(sc.a[0][i >> 1], i & 1), a0, acc[J][0]);
+            acc[J][0] = fmaf(half_at(sc.a[0][(P + i) >> 1], (P + i) & 1), b0, acc[J][0]);
+            acc[J][M - 1] = fmaf(half_at(sc.a[M - 1][i >> 1], i & 1), a1, acc[J][M - 1]);
+            acc[J][M - 1] =
+                fmaf(half_at(sc.a[M - 1][(P + i) >> 1], (P + i) & 1), b1, acc[J][M - 1]);
+          }
+        }
+      }
+      if (i0 == 0) finish(Slot<JP>{});  // the previous group's loads are long done
     }
-  }
-  __syncthreads();
+    pend[J] = active;
+    pend_row[J] = (gc.rb0 + tw) * kRowBlock + lane;
+    pend_kb[J] = gc.kb;
+    pend_z[J] = sc.z;
+    // this slot's scales now take the team's group PF ahead
+    zero_scales(pf[J]);
+    if (gp < R.NG && tw < pc.n) load_scales<M, P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, pf[J]);
+    cursor_next(pc, R.u1, RB);
+    cursor_next(pc, R.u1, RB);
+    gp += 2;
+    // the team's next group is two stages on (D even: no slot is skipped)
+    cursor_next(gc, R.u1, RB);
+    cursor_next(gc, R.u1, RB);
+    s += 2;
+    if (s >= D) {
+      s -= D;
+      ph ^= 1u;
+    }
+    g += 2;
+  };
 
-  // Split-K reduction over the CTAs of the cluster: rank r finishes rows
-  // [r * own_rows, (r + 1) * own_rows) of the cluster.  Every other rank
-  // stores its sums for those rows into r's receive buffer (distributed
-  // shared memory, counted on r's receive barrier); r adds them in rank
-  // order and rounds once to fp16.
-  float* recv = reinterpret_cast<float*>(smem + P.off_recv);   // [S][M][own_rows]
-  if (S > 1) cluster_wait();  // every CTA of the cluster has its receive barrier ready
-  if (S > 1 && layout_ok) {
-    for (int e = tid; e < M * rows_c; e += nthreads) {
-      const int m = e / rows_c;
-      const int rl = e % rows_c;
-      const int owner = rl / P.own_rows;
-      if (owner == rank) continue;
-      const uint32_t slot = smem_u32(recv + ((size_t)rank * M + m) * P.own_rows + (rl - owner * P.own_rows));
-      st_async_f32(mapa_shared(slot, (uint32_t)owner), accr[(size_t)m * P.part_rows + rl],
-                   mapa_shared(recv_bar, (uint32_t)owner));
-    }
-    if (layout_ok && !mbar_wait_bounded(recv_bar, 0, P.timeout_ns)) {
-      if (tid == 0) record_error(&g_device_error, BCQ_ERR_TIMEOUT);
-    }
+  while (g < R.NG) {
+    group(Slot<0>{});
+    if (g < R.NG) group(Slot<1>{});
   }
-  for (int e = tid; e < M * own_n; e += nthreads) {
-    const int m = e / own_n;
-    const int i = e % own_n;
-    const int rl = own0 + i;
-    const int n = rb0 * kRowBlock + rl;
-    if (n >= P.N) continue;
-    float sum = 0.f;
-    for (int rk = 0; rk < S; ++rk)
-      sum += rk == rank ? accr[(size_t)m * P.part_rows + rl]
-                        : recv[((size_t)rk * M + m) * P.own_rows + i];
-    P.y[(size_t)m * P.N + n] = f2h_rn(sum);
+  finish(Slot<0>{});
+  finish(Slot<1>{});
+  advance_tables(R.kb_last);  // the same barriers in both teams
+
+  // Split-K: every unit's partial sums are in the workspace.  Each CTA
+  // counts its arrivals (release), then reduces the row-blocks it is
+  // designated for -- row-block rb belongs to the CTA that computed its unit
+  // in K-block rb mod KB, so the work is spread evenly whatever the order in
+  // which CTAs finish.  The reducer waits (bounded) until all KB partials of
+  // rb have arrived, adds them in K-block order (the result does not depend
+  // on scheduling) and clears them and the counter, so the whole workspace
+  // is zero again for the next call, whatever its shape.
+  if (prm.KB > 1) {
+    __threadfence();
+    named_barrier_sync(1, kConsumers);
+    if (*abort_flag == 0) {
+      for (int u = R.u0 + tid; u < R.u1; u += kConsumers) red_add_release(prm.cnt + u % RB, 1u);
+    }
+    // this CTA's row-blocks to reduce: units (kb, rb) with kb == rb mod KB,
+    // taken kReduceBatch units at a time (the list holds one batch)
+    for (int base = R.u0; base < R.u1; base += kReduceBatch) {
+      if (tid == 0) *nlist = 0;
+      named_barrier_sync(1, kConsumers);
+      if (tid < kReduceBatch && base + tid < R.u1) {
+        const int u = base + tid;
+        const int rbx = u % RB;
+        if (u / RB == rbx % prm.KB) list[atomicAdd(nlist, 1)] = rbx;
+      }
+      named_barrier_sync(1, kConsumers);
+      const int nl = *abort_flag == 0 ? *reinterpret_cast<volatile int*>(nlist) : 0;
+      for (int e = warp; e < nl; e += kConsumerWarps) {
+        const int rbx = list[e];
+        bool ready = true;
+        if (lane == 0)
+          ready = wait_count(prm.cnt + rbx, (unsigned int)prm.KB, abort_flag, prm.timeout_ns);
+        ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
+        if (!ready) {
+          if (lane == 0 && *abort_flag == 0) {
+            record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          continue;
+        }
+        const int row = rbx * kRowBlock + lane;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
+          float sum = 0.f;
+#pragma unroll 8
+          for (int k = 0; k < prm.KB; ++k) sum += ldg_cg_f32(pp + (size_t)k * M * part_stride);
+          if (row < prm.N) prm.y[(size_t)m * prm.N + row] = f2h_rn(sum);
+        }
+        // the workspace is left zero-filled for any later shape
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
+          for (int k = 0; k < prm.KB; ++k) stg_cg_zero(pp + (size_t)k * M * part_stride);
+        }
+        __syncwarp();
+        if (lane == 0) *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
+      }
+      named_barrier_sync(1, kConsumers);
+    }
   }
 }
 
 // ============================================================ LUT dump
 
-template <int M, int NKB>
-__global__ void __launch_bounds__(256, 1) lut_dump_kernel(const __grid_constant__ LutParams P) {
-  extern __shared__ __align__(128) unsigned char smem[];
+// One CTA per K-block: the table exactly as the GEMV kernel builds it, read
+// back to global memory in the canonical [M][K/8][256] order.
+template <int M>
+__global__ void __launch_bounds__(256) lut_dump_kernel(const __grid_constant__ LutParams P) {
+  extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
-  float* gsum = reinterpret_cast<float*>(smem);
-  const uint32_t lut_base = lut_base_of(sbase);
-  if (lut_base - sbase < 64 || lut_base - sbase + 2u * kLutTableBytes > P.dyn_bytes) {
-    if (threadIdx.x == 0) record_error(&g_device_error, BCQ_ERR_UNSUPPORTED);
-    return;
-  }
-  const int kb_first = blockIdx.x * NKB;
-  const int nkb = min(NKB, P.KB - kb_first);
-  build_lut_phase<M, NKB>(P.x, P.K, P.KB, kb_first, nkb, lut_base, gsum,
-                          (int)(blockDim.x >> 5));
+  const int kb = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  uint4 xv[M];
+  load_x<M>(P.x, P.K, kb, lane, xv);
+  float gs[M][2];
+  const int slot = M == 1 ? (kb & 1) : 0;
+  build_lut<M, 2>(xv, slot, sbase, warp, lane, gs);
   __syncthreads();
-  const int C = P.K / 8;
-  const int total = M * nkb * 32 * 256;
-  for (int e = threadIdx.x; e < total; e += blockDim.x) {
+  const int C8 = P.K / 8;
+  for (int e = threadIdx.x; e < M * 32 * 256; e += blockDim.x) {
     const int col = e & 31;
     const int b = (e >> 5) & 255;
-    const int mk = e >> 13;
-    const int m = mk / nkb, kbp = mk % nkb;
-    const int k = (kb_first + kbp) * kKBlock + (col >> 4) * kGroup + (col & 15) * 8;
+    const int m = e >> 13;
+    const int k = kb * kKBlock + (col >> 4) * kGroup + (col & 15) * 8;
     if (k >= P.K) continue;
-    const float v = lds_f32_dyn(lut_table_addr<NKB>(lut_base, m, kbp) + (uint32_t)b * 256u +
-                                (uint32_t)col * 4u);
-    P.lut[((size_t)m * C + k / 8) * 256 + b] = v;
+    const uint32_t a = sbase + (uint32_t)b * 256u +
+                       (M == 1 ? (uint32_t)slot * 128u + (uint32_t)col * 4u
+                               : (uint32_t)col * 8u + (uint32_t)m * 4u);
+    P.lut[((size_t)m * C8 + k / 8) * 256 + b] = lds_f32_dyn(a);
   }
-  if (P.gsum) {
-    for (int e = threadIdx.x; e < M * nkb * 2; e += blockDim.x) {
-      const int m = e / (nkb * 2);
-      const int gl = e % (nkb * 2);
-      const int g = kb_first * 2 + gl;
-      if (g < P.G) P.gsum[(size_t)m * P.G + g] = gsum[m * 2 * NKB + gl];
+  if (P.gsum && warp == 0 && (lane & 15) == 0) {
+    const int g = 2 * kb + (lane >> 4);  // lane 0: group A, lane 16: group B
+    if (g < P.G) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) P.gsum[(size_t)m * P.G + g] = gs[m][0];
     }
   }
 }
@@ -629,64 +838,77 @@ __global__ void wait_probe_kernel(unsigned long long limit_ns) {
     fence_mbar_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0 && !mbar_wait_bounded(a, 0, limit_ns)) record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+  if (threadIdx.x == 0 && !mbar_wait_bounded(a, 0, limit_ns))
+    record_error(&g_device_error, BCQ_ERR_TIMEOUT);
 }
 
 // ============================================================ launchers
 
-cudaError_t launch_pack(const uint32_t* canon, uint32_t* packed, int p_H, int N,
-                        int K, cudaStream_t st) {
-  const int KB = (K + kKBlock - 1) / kKBlock;
-  const size_t KC = ((size_t)KB + kChunkBlocks - 1) / kChunkBlocks;
+cudaError_t launch_pack(const uint32_t* canon, uint32_t* packed, int p_H, int N, int K,
+                        cudaStream_t st) {
+  const size_t KB = ((size_t)K + kKBlock - 1) / kKBlock;
   const int RB = (N + kRowBlock - 1) / kRowBlock;
-  const int RBG = (RB + kRowGroup - 1) / kRowGroup;
-  const size_t total = KC * (size_t)RBG * p_H * kRowGroup * kChunkBlocks * kWordsPerPlaneBlock;
+  const int RG = (RB + kRowGroup - 1) / kRowGroup;
+  const size_t total = KB * (size_t)RG * p_H * kRowGroup * kWordsPerUnitPlane;
   const int threads = 256;
   size_t blocks = (total + threads - 1) / threads;
   if (blocks > 148u * 64u) blocks = 148u * 64u;
-  pack_planes_kernel<<<(unsigned)blocks, threads, 0, st>>>(canon, packed, p_H, N, K, RBG, total);
+  pack_planes_kernel<<<(unsigned)blocks, threads, 0, st>>>(canon, packed, p_H, N, K, RG, total);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pack_scales(const uint16_t* src, uint16_t* dst, int q, int N,
-                               int K, cudaStream_t st) {
-  const int KB = (K + kKBlock - 1) / kKBlock;
-  const size_t KC = ((size_t)KB + kChunkBlocks - 1) / kChunkBlocks;
+cudaError_t launch_pack_scales(const uint16_t* src, uint16_t* dst, int q, int N, int K,
+                               cudaStream_t st) {
+  const size_t KB = ((size_t)K + kKBlock - 1) / kKBlock;
   const int G = K / kGroup;
   const int RB = (N + kRowBlock - 1) / kRowBlock;
-  const int RBP = (RB + kRowGroup - 1) / kRowGroup * kRowGroup;
-  const size_t total = KC * (size_t)RBP * 128 * q;
+  const size_t total = KB * (size_t)RB * kRowBlock * 2 * q;
   const int threads = 256;
   size_t blocks = (total + threads - 1) / threads;
   if (blocks > 148u * 64u) blocks = 148u * 64u;
-  pack_scales_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, dst, q, N, G, RBP, total);
+  pack_scales_kernel<<<(unsigned)blocks, threads, 0, st>>>(src, dst, q, N, G, RB, total);
   return cudaGetLastError();
 }
 
-GemvKernel gemv_kernel_for(int M) {
-  switch (M) {
-    case 1: return gemv_lut_kernel<1>;
-    case 2: return gemv_lut_kernel<2>;
-    default: return nullptr;
+GemvKernel gemv_kernel_for(int M, int P, bool mixed) {
+  if (M == 1) {
+    switch (P) {
+      case 1: return gemv_lut_kernel<1, 1, false>;
+      case 2: return gemv_lut_kernel<1, 2, false>;
+      case 3: return gemv_lut_kernel<1, 3, false>;
+      case 4: return gemv_lut_kernel<1, 4, false>;
+      default: return nullptr;
+    }
   }
+  if (M == 2 && !mixed) {
+    switch (P) {
+      case 1: return gemv_lut_kernel<2, 1, false>;
+      case 2: return gemv_lut_kernel<2, 2, false>;
+      case 3: return gemv_lut_kernel<2, 3, false>;
+      case 4: return gemv_lut_kernel<2, 4, false>;
+      default: return nullptr;
+    }
+  }
+  if (M == 2) {
+    switch (P) {
+      case 2: return gemv_lut_kernel<2, 2, true>;
+      case 3: return gemv_lut_kernel<2, 3, true>;
+      case 4: return gemv_lut_kernel<2, 4, true>;
+      default: return nullptr;
+    }
+  }
+  return nullptr;
 }
 
-cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, int C, int W,
-                        size_t dyn, bool pdl, cudaStream_t st) {
+cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,
+                        cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(C * p.S), 1, 1);
-  cfg.blockDim = dim3((unsigned)(32 * (W + p.NP)), 1, 1);
+  cfg.gridDim = dim3((unsigned)p.C, 1, 1);
+  cfg.blockDim = dim3((unsigned)(32 * (kConsumerWarps + p.NP)), 1, 1);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   int na = 0;
-  if (p.S > 1) {
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = (unsigned)p.S;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-  }
   if (pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -697,19 +919,10 @@ cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, int C, int W,
   return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
-cudaError_t max_active_clusters(GemvKernel fn, int S, int nthreads, size_t dyn, int* out) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)S, 1, 1);
-  cfg.blockDim = dim3((unsigned)nthreads, 1, 1);
-  cfg.dynamicSmemBytes = dyn;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaOccupancyMaxActiveClusters(out, fn, &cfg);
+cudaError_t blocks_per_sm(GemvKernel fn, int nthreads, size_t dyn, int* out) {
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, nthreads, dyn);
 }
 
 cudaError_t launch_lut_dump(const uint16_t* x, int M, int K, float* lut, float* gsum,
@@ -722,21 +935,16 @@ cudaError_t launch_lut_dump(const uint16_t* x, int M, int K, float* lut, float* 
   p.K = K;
   p.KB = (K + kKBlock - 1) / kKBlock;
   p.G = K / kGroup;
-  const int NKB = 4 / M;  // M * NKB <= 4 -> at most 2 tables of 64 KiB
-  const size_t dyn = kLutAlign + 2u * kLutTableBytes;
-  p.dyn_bytes = (uint32_t)dyn;
-  const unsigned blocks = (unsigned)((p.KB + NKB - 1) / NKB);
+  const size_t dyn = kLutBytes;
   void (*fn)(LutParams) = nullptr;
   switch (M) {
-    case 1: fn = lut_dump_kernel<1, 4>; break;
-    case 2: fn = lut_dump_kernel<2, 2>; break;
-    case 3: fn = lut_dump_kernel<3, 1>; break;
-    case 4: fn = lut_dump_kernel<4, 1>; break;
+    case 1: fn = lut_dump_kernel<1>; break;
+    case 2: fn = lut_dump_kernel<2>; break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
   if (e != cudaSuccess) return e;
-  fn<<<blocks, 256, dyn, st>>>(p);
+  fn<<<(unsigned)p.KB, 256, dyn, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -35,7 +35,8 @@
  *   - Kernels never wait without a limit.  A wait that runs out sets a device
  *     error word (read with bcq_device_error) and the kernel returns early;
  *     its outputs are then unspecified.
- *   - The library allocates no device memory.
+ *   - The library allocates no device memory.  Calls whose split-K partial
+ *     sums need room take a caller-owned workspace (bcq_workspace_bytes).
  */
 #ifndef BCQ_H_
 #define BCQ_H_
@@ -70,7 +71,8 @@ int bcq_version(void);
 
 /*
  * Size in bytes of the packed plane buffer for p_H planes of an N x K weight
- * (rows padded to a multiple of 32, columns to a multiple of 256).  Returns 0
+ * (rows padded to a multiple of 32, columns to a multiple of 256): exactly
+ * 1 KiB per (plane, 32 rows, 256 columns).  Returns 0
  * for invalid shapes (p_H outside 1..4, N < 1, K < 128 or K % 128 != 0).
  */
 size_t bcq_packed_planes_bytes(int p_H, int N, int K);
@@ -93,7 +95,8 @@ bcq_status bcq_pack_planes(const uint32_t* planes_canon, uint32_t* planes_packed
 
 /*
  * Size in bytes of a packed per-(row, group) array with q values per entry
- * (q = 1..4), or 0 for invalid arguments (same shape rules as above).
+ * (q = 1..4; rows padded to a multiple of 32, groups to an even count), or 0
+ * for invalid arguments (same shape rules as above).
  */
 size_t bcq_packed_scales_bytes(int q, int N, int K);
 
@@ -113,6 +116,14 @@ size_t bcq_packed_scales_bytes(int q, int N, int K);
  */
 bcq_status bcq_pack_scales(const uint16_t* src, int q, int N, int K,
                            uint16_t* dst, void* stream);
+
+/*
+ * Bytes of workspace bcq_gemm needs for M rows of x and an N x K weight: 0
+ * when K <= 256 (no split over K), else room for the arrival counters of the
+ * row-blocks and the fp32 partial sums of every (256-column K-block, row) for
+ * up to two rows.  0 for invalid shapes as well.
+ */
+size_t bcq_workspace_bytes(int M, int N, int K);
 
 /*
  * y = x . W_hat^T for M rows of x, each row at its own precision.
@@ -135,26 +146,38 @@ bcq_status bcq_pack_scales(const uint16_t* src, int q, int N, int K,
  *   p_H      planes stored in `planes` (1..4).
  *   group    must be 128 (other sizes -> BCQ_ERR_UNSUPPORTED).
  *   y        device, fp16 [M][N] row-major, overwritten; 2-byte aligned.
+ *   workspace, workspace_bytes
+ *            device scratch of at least bcq_workspace_bytes(M, N, K) bytes,
+ *            16-byte aligned (NULL allowed when that is 0).  Zero-fill it once
+ *            before its first use; every call that completes without a device
+ *            error leaves it zero-filled again (zero it again after
+ *            BCQ_ERR_TIMEOUT).  Calls that may run at the same time (other
+ *            streams) need workspaces of their own; calls in one stream may
+ *            share one.
  * The call reads planes 0..max_m(p_m)-1 only.  Accumulation is fp32; each
- * output is rounded once to fp16 (round to nearest even).  For a given launch
- * configuration the summation order is fixed, so results are reproducible.
+ * output is rounded once to fp16 (round to nearest even).  Partial sums over
+ * 256-column K-blocks are added in K order, so for a given device and shape
+ * the result does not depend on scheduling: results are reproducible.
+ * Errors: as listed above; workspace too small or NULL -> BCQ_ERR_NULL;
+ * misaligned workspace -> BCQ_ERR_ALIGN.
  */
 bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes,
                     const uint16_t* const alpha[4], const uint16_t* z,
                     int p, const int32_t* p_row, int M, int N, int K, int p_H,
-                    int group, uint16_t* y, void* stream);
+                    int group, uint16_t* y, void* workspace, size_t workspace_bytes,
+                    void* stream);
 
 /*
  * The launch plan bcq_gemm would use for one launch of M (1..2) activation
- * rows: p_load planes streamed, precisions q0 (and q1, 0 = none) among the
- * rows, offsets present (has_z).  use_device = 1 plans for the current
- * device; 0 (or no usable device) plans for a nominal 148-SM B200 without
- * touching CUDA.  out[8] receives: cluster size S (K splits), clusters C,
- * consumer warps, producer warps, ring stages, dynamic shared memory bytes,
- * stage bytes, row groups per cluster.  For inspection and tests.
+ * rows streaming p_load planes (mixed = 1: the rows use different
+ * precisions).  use_device = 1 plans for the current device; 0 (or no usable
+ * device) plans for a nominal 148-SM B200 without touching CUDA.  out[8]
+ * receives: CTAs, consumer warps, producer warps, ring stages, dynamic shared
+ * memory bytes, bytes per ring stage, largest number of units (K-block x
+ * row-block pairs) of one CTA, K-blocks (partial sums per output).  For
+ * inspection and tests.
  */
-int bcq_plan_query(int M, int N, int K, int p_load, int q0, int q1, int has_z,
-                   int use_device, int* out);
+int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, int* out);
 
 /*
  * Launch option for the GEMV kernels of this process (all devices):
@@ -162,10 +185,10 @@ int bcq_plan_query(int M, int N, int K, int p_load, int q0, int q1, int has_z,
  *   1  programmatic dependent launch: a GEMV kernel may be scheduled while the
  *      preceding kernel in its stream finishes; it touches no global memory
  *      before that kernel has completed;
- *   2  as 1, but the kernel may start streaming its planes and packed scales
- *      before the preceding kernel has completed (x and y still wait).  Only
- *      valid when no kernel immediately before it in the stream writes the
- *      weights it reads.
+ *   2  as 1, but the kernel may start streaming its planes before the
+ *      preceding kernel has completed (x, y, scales and the workspace still
+ *      wait).  Only valid when no kernel immediately before it in the stream
+ *      writes the planes it reads.
  * Returns BCQ_OK, or BCQ_ERR_UNSUPPORTED for another mode.
  */
 int bcq_set_pdl(int mode);
@@ -175,14 +198,16 @@ int bcq_set_pdl(int mode);
  * x_dev, the matmul, and the copy of y_dev back into y_host, all on `stream`
  * (pinned host buffers make the copies asynchronous).  x_dev (fp16 [M][K],
  * 16-byte aligned) and y_dev (fp16 [M][N]) are caller-owned device staging
- * buffers.  The caller synchronises `stream` before reading y_host.
+ * buffers; workspace as for bcq_gemm.  The caller synchronises `stream`
+ * before reading y_host.
  * Errors as bcq_gemm, plus BCQ_ERR_NULL for missing host or staging buffers.
  */
 bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
                          const uint16_t* const alpha[4], const uint16_t* z,
                          int p, const int32_t* p_row, int M, int N, int K,
                          int p_H, int group, uint16_t* y_host,
-                         uint16_t* x_dev, uint16_t* y_dev, void* stream);
+                         uint16_t* x_dev, uint16_t* y_dev, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /*
  * The lookup table and group sums exactly as the GEMV kernel builds them in

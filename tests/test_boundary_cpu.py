@@ -35,55 +35,77 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert api.lib().bcq_version() == 100
+    assert api.lib().bcq_version() == 200
     for s in range(8):
         assert api.status_string(s).startswith("BCQ_")
     assert api.status_string(99) == "BCQ_ERR_UNKNOWN"
 
 
 def test_packed_bytes_formula(L):
-    # chunks of 512 columns x row groups of 4 row-blocks (128 rows) x p_H x 8 KiB
-    assert api.packed_planes_bytes(4, 14336, 4096) == 8 * 112 * 4 * 8192
+    # 8 KiB per (plane, 256 rows, 256 columns), rows and columns padded
+    assert api.packed_planes_bytes(4, 14336, 4096) == 16 * 56 * 4 * 8192
     assert api.packed_planes_bytes(4, 14336, 4096) == 14336 * 4096 * 4 // 8
-    assert api.packed_planes_bytes(2, 33, 384) == 1 * 1 * 2 * 8192     # padded
+    assert api.packed_planes_bytes(2, 33, 384) == 2 * 1 * 2 * 8192     # padded
     for bad in [(0, 32, 256), (5, 32, 256), (4, 0, 256), (4, 32, 100), (4, 32, 0)]:
         assert api.packed_planes_bytes(*bad) == 0
-    # chunks x row-blocks (padded to groups of 4) x 2 K-blocks x 2 passes x 32 lanes x q halves
-    assert api.packed_scales_bytes(3, 14336, 4096) == 8 * 448 * 128 * 3 * 2
+    # K-blocks x row-blocks x 32 lanes x 2 groups x q halves
+    assert api.packed_scales_bytes(3, 14336, 4096) == 16 * 448 * 32 * 2 * 3 * 2
     assert api.packed_scales_bytes(3, 14336, 4096) == 14336 * 32 * 3 * 2
-    assert api.packed_scales_bytes(1, 33, 384) == 1 * 4 * 128 * 1 * 2
+    assert api.packed_scales_bytes(1, 33, 384) == 2 * 2 * 32 * 2 * 1 * 2
     assert api.packed_scales_bytes(0, 32, 256) == 0
 
 
-@pytest.mark.parametrize("M,N,K,p,q1", [(1, 14336, 4096, 2, 0), (1, 14336, 4096, 4, 0),
-                                        (1, 4096, 14336, 3, 0), (2, 4096, 4096, 2, 0),
-                                        (2, 28672, 8192, 3, 2), (1, 256, 512, 4, 0),
-                                        (1, 1, 128, 1, 0), (2, 33, 640, 2, 0)])
-def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, q1):
-    """Plans for a nominal 148-SM B200 (no GPU needed): every launch fits the
-    227 KiB of shared memory, splits K into at most the chunks there are,
-    and keeps the ring depth a multiple of both the consumer groups and the
-    producer warps (the stage-ownership rule of the pipeline)."""
-    pl = api.plan_query(M, N, K, p, p, q1, has_z=True, use_device=False)
-    KC = -(-(-(-K // 256)) // 2)
-    assert 1 <= pl["S"] <= min(8, KC)
+def test_workspace_bytes_formula(L):
+    # one K-block: no split over K, no workspace
+    assert api.workspace_bytes(1, 4096, 256) == 0
+    assert api.workspace_bytes(4, 4096, 128) == 0
+    # counters (row-blocks x 4 B, rounded to 256 B) + KB x min(M, 2) x rows x 4 B
+    assert api.workspace_bytes(1, 14336, 4096) == 1792 + 16 * 1 * 14336 * 4
+    assert api.workspace_bytes(8, 14336, 4096) == 1792 + 16 * 2 * 14336 * 4
+    assert api.workspace_bytes(2, 33, 640) == 256 + 3 * 2 * 64 * 4
+    assert api.workspace_bytes(0, 64, 512) == 0
+    assert api.workspace_bytes(1, 64, 100) == 0
+
+
+@pytest.mark.parametrize("M,N,K,p,mixed", [(1, 14336, 4096, 2, False), (1, 14336, 4096, 4, False),
+                                           (1, 4096, 14336, 3, False), (2, 4096, 4096, 2, False),
+                                           (2, 28672, 8192, 4, True), (1, 256, 512, 4, False),
+                                           (1, 1, 128, 1, False), (2, 33, 640, 2, False)])
+def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
+    """Plans for a nominal 148-SM B200 (no GPU needed): one CTA per SM at
+    most (never more CTAs than units), whole K-blocks per CTA when the CTAs
+    divide among them, the 227 KiB of shared memory, and an even ring depth
+    (teams alternate stages: a stage's team consumed the stage one ring
+    earlier) that is a multiple of the producer warps (each refills only its
+    own slots)."""
+    pl = api.plan_query(M, N, K, p, mixed=mixed, use_device=False)
+    RB, KB = -(-N // 32), -(-K // 256)
+    U = RB * KB
+    if KB <= 148:
+        assert pl["C"] == min(U, KB * min(RB, 148 // KB))   # whole K-blocks per CTA group
+        assert pl["C"] % KB == 0 or pl["C"] == U
+    else:
+        assert pl["C"] == 148
+    assert pl["KB"] == KB
+    assert pl["units_max"] == -(-U // pl["C"])
     assert pl["dyn_bytes"] <= 232448
-    G = pl["W"] // 4
-    assert pl["W"] % 4 == 0 and pl["D"] % G == 0 and pl["D"] % pl["NP"] == 0
-    assert 2 <= pl["D"] <= 8
-    assert pl["C"] * pl["S"] <= 148
-    RBG = -(-(-(-N // 32)) // 4)
-    assert pl["row_groups"] * pl["C"] <= RBG + pl["C"]
-    assert pl["stage_bytes"] == 4 * (p * 2048 + 256 * (p + q1) + 256)
+    assert pl["stage_bytes"] == 8192 * p    # the p planes of one row group
+    assert pl["dyn_bytes"] >= 65536 + pl["D"] * pl["stage_bytes"]
+    assert pl["D"] % 2 == 0 and pl["D"] % pl["NP"] == 0 and 2 <= pl["D"] <= 20
+    # as deep as the shared memory allows
+    assert pl["D"] == 20 or 65536 + (pl["D"] + 2) * pl["stage_bytes"] + 1024 > 232448
+    assert pl["consumer_warps"] == 16
 
 
 def test_plan_query_rejects_bad_arguments(L):
     with pytest.raises(api.BcqError):
-        api.plan_query(3, 64, 256, 2, 2)          # at most two rows per launch
+        api.plan_query(3, 64, 256, 2)             # at most two rows per launch
     with pytest.raises(api.BcqError):
-        api.plan_query(1, 64, 200, 2, 2)          # K % 128
+        api.plan_query(1, 64, 200, 2)             # K % 128
     with pytest.raises(api.BcqError):
-        api.plan_query(1, 64, 256, 5, 2)          # p_load
+        api.plan_query(1, 64, 256, 5)             # p_load
+    with pytest.raises(api.BcqError):
+        api.plan_query(1, 64, 256, 3, mixed=True)  # one row cannot mix
 
 
 FAKE = 0x10000   # never dereferenced: every call below fails validation first
@@ -97,16 +119,18 @@ def _alpha(*present, base=FAKE):
 
 
 def _gemm(L, x=FAKE, planes=FAKE, alpha=None, z=None, p=2, p_row=None, M=1,
-          N=64, K=256, p_H=4, group=128, y=FAKE):
+          N=64, K=256, p_H=4, group=128, y=FAKE, ws=None, ws_bytes=0):
     alpha = _alpha(2, 3, 4) if alpha is None else alpha
-    return L.bcq_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, group, y, None)
+    return L.bcq_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, group, y, ws, ws_bytes,
+                      None)
 
 
 def test_gemm_rejects_before_launch(L):
     assert _gemm(L, x=None) == api.BCQ_ERR_NULL
     assert _gemm(L, y=None) == api.BCQ_ERR_NULL
     assert _gemm(L, planes=None) == api.BCQ_ERR_NULL
-    assert L.bcq_gemm(FAKE, FAKE, None, None, 2, None, 1, 64, 256, 4, 128, FAKE, None) == api.BCQ_ERR_NULL
+    assert L.bcq_gemm(FAKE, FAKE, None, None, 2, None, 1, 64, 256, 4, 128, FAKE, None, 0,
+                      None) == api.BCQ_ERR_NULL
     assert _gemm(L, K=100) == api.BCQ_ERR_SHAPE
     assert _gemm(L, K=0) == api.BCQ_ERR_SHAPE
     assert _gemm(L, N=0) == api.BCQ_ERR_SHAPE
@@ -130,6 +154,12 @@ def test_gemm_rejects_before_launch(L):
     assert _gemm(L, alpha=_alpha(2, base=FAKE + 2), p=2) == api.BCQ_ERR_ALIGN
     assert _gemm(L, alpha=_alpha(4, base=FAKE + 8), p=4) == api.BCQ_ERR_ALIGN
     assert _gemm(L, z=FAKE + 8) == api.BCQ_ERR_ALIGN
+    # K > 256 splits over K: a workspace of bcq_workspace_bytes is required
+    need = api.workspace_bytes(1, 64, 512)
+    assert need > 0
+    assert _gemm(L, K=512) == api.BCQ_ERR_NULL
+    assert _gemm(L, K=512, ws=FAKE, ws_bytes=need - 1) == api.BCQ_ERR_NULL
+    assert _gemm(L, K=512, ws=FAKE + 8, ws_bytes=need) == api.BCQ_ERR_ALIGN
 
 
 def test_pack_and_lut_reject_before_launch(L):
@@ -152,7 +182,7 @@ def test_pack_and_lut_reject_before_launch(L):
     assert L.bcq_debug_wait_timeout(0, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_debug_wait_timeout(2000000, None) == api.BCQ_ERR_SHAPE
     assert L.bcq_gemm_host(None, FAKE, _alpha(2), None, 2, None, 1, 64, 256, 4, 128,
-                           FAKE, FAKE, FAKE, None) == api.BCQ_ERR_NULL
+                           FAKE, FAKE, FAKE, None, 0, None) == api.BCQ_ERR_NULL
 
 
 def test_empty_batch_is_a_no_op(L):

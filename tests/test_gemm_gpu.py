@@ -234,3 +234,63 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert api.device_error() == api.BCQ_OK   # read clears it
     prob = synth.make_problem(256, 512, 1, seed=12)
     _check(_run(prob, p=2), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=2))
+
+
+# ------------------------------------------------- launch shapes and workspace
+
+@pytest.mark.parametrize("C,D,NP", [(1, 2, 1), (3, 4, 2), (7, 6, 2), (13, 2, 2), (148, 8, 2)])
+def test_forced_launch_shapes(monkeypatch, C, D, NP):
+    """Few CTAs (each spanning several K-blocks, groups cut at K-block
+    boundaries), shallow and deep rings, one or two producer warps."""
+    monkeypatch.setenv("BCQ_FORCE_C", str(C))
+    monkeypatch.setenv("BCQ_FORCE_D", str(D))
+    monkeypatch.setenv("BCQ_FORCE_NP", str(NP))
+    prob = synth.make_problem(1000, 2048, 3, seed=20 + C, mixed=True)
+    prob.p_row[:] = [4, 2, 3]
+    w = _weights(prob)
+    _check(_run(prob, w, p_row=prob.p_row),
+           oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row), f"C={C}")
+    for p in (2, 4):
+        _check(_run(prob, w, p=p), oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p),
+               f"C={C} p={p}")
+
+
+def test_workspace_is_left_zero_filled():
+    prob = synth.make_problem(4096, 4096, 2, seed=21)
+    w = _weights(prob)
+    for p in (2, 3):
+        _run(prob, w, p=p)
+    ws = api.workspace(2, 4096, 4096, "cuda")
+    torch.cuda.synchronize()
+    assert ws is not None and int(ws.count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_programmatic_dependent_launch_gives_the_same_bits(mode):
+    """Back-to-back calls with PDL (and early plane streaming) equal the plain
+    stream-ordered results bit for bit."""
+    prob = synth.make_problem(14336, 4096, 2, seed=22)
+    w = _weights(prob)
+    x = _x(prob)
+    ref = [w.gemm(x[:1], p=2), w.gemm(x, p=3), w.gemm(x[1:], p=4)]
+    torch.cuda.synchronize()
+    try:
+        api.set_pdl(mode)
+        for _ in range(3):
+            got = [w.gemm(x[:1], p=2), w.gemm(x, p=3), w.gemm(x[1:], p=4)]
+        torch.cuda.synchronize()
+    finally:
+        api.set_pdl(0)
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+
+
+def test_workspace_shared_across_shapes():
+    """One workspace serves calls of different shapes in turn: a smaller N
+    leaves no partial sums where a larger N keeps its arrival counters."""
+    a = synth.make_problem(4096, 4096, 2, seed=23)
+    b = synth.make_problem(14336, 4096, 1, seed=24)
+    wa, wb = _weights(a), _weights(b)
+    for _ in range(2):
+        _check(_run(a, wa, p=3), oracle.gemm(a.x, a.planes, a.alphas, a.z, p=3), "4096")
+        _check(_run(b, wb, p=2), oracle.gemm(b.x, b.planes, b.alphas, b.z, p=2), "14336")

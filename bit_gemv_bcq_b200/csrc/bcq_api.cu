@@ -138,10 +138,10 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, Plan* out) {
   // With no more K-blocks than SMs, every K-block gets the same number of
   // CTAs and no CTA spans two K-blocks (a second table build would make it
   // the slowest CTA, and the last to arrive for all of its row-blocks).
-  long long C = std::min<long long>(U, dc->sm_count);
-  if (KB <= dc->sm_count) C = std::min<long long>(U, KB * std::min<long long>(RB, dc->sm_count / KB));
+  long long C = std::min<long long>(U, std::min(dc->sm_count, kMaxCtas));
+  if (KB <= C) C = std::min<long long>(U, KB * std::min<long long>(RB, C / KB));
   const int force_C = env_int("BCQ_FORCE_C", 0);
-  if (force_C > 0) C = std::min<long long>(U, force_C);
+  if (force_C > 0) C = std::min<long long>(U, std::min(force_C, kMaxCtas));
   pl.C = (int)C;
   pl.units_max = (U + C - 1) / C;
   if (U >= (1ll << 31)) return BCQ_ERR_UNSUPPORTED;  // units are counted in 32 bits
@@ -186,6 +186,39 @@ bcq_status validate_gemm(const uint16_t* x, const uint32_t* planes,
 
 std::atomic<int> g_pdl_mode{0};  // 0 off, 1 PDL, 2 PDL + early plane streaming
 
+// Splits the U = RB * KB units (kb-major) over C CTAs: when the CTAs divide
+// evenly among the K-blocks, C / KB CTAs share the row-blocks of each
+// K-block and no CTA builds two tables; otherwise every CTA takes an equal
+// share (the first U mod C one unit more).  Groups: per K-block, the row
+// groups of 8 row-blocks the CTA touches.
+void plan_units(int RB, int KB, int C, CtaWork* work) {
+  const long long U = (long long)RB * KB;
+  for (int c = 0; c < C; ++c) {
+    long long u0, u1;
+    if (C >= KB && C % KB == 0) {
+      const int cpk = C / KB, kb = c / cpk, j = c - kb * cpk;
+      const int q = RB / cpk, r = RB % cpk;
+      u0 = (long long)kb * RB + (long long)j * q + std::min(j, r);
+      u1 = u0 + q + (j < r ? 1 : 0);
+    } else {
+      const long long q = U / C, r = U % C;
+      u0 = c * q + std::min<long long>(c, r);
+      u1 = u0 + q + (c < r ? 1 : 0);
+    }
+    int ng = 0;
+    for (long long u = u0; u < u1;) {
+      const long long kb = u / RB;
+      const long long end = std::min(u1, (kb + 1) * RB);
+      const long long a = u - kb * RB, b = end - kb * RB;
+      ng += (int)((b + kRowGroup - 1) / kRowGroup - a / kRowGroup);
+      u = end;
+    }
+    const int kb0 = (int)(u0 / RB);
+    const int kb1 = u1 > u0 ? (int)((u1 - 1) / RB) : kb0;
+    work[c] = CtaWork{(int)u0, (int)u1, ng, kb0 | (kb1 << 16)};
+  }
+}
+
 // Launches of at most two rows, in order; two rows with different
 // precisions share one launch (planes streamed up to the larger one).
 bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
@@ -226,6 +259,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
     g.q[1] = q[1];
     g.U = (int)((long long)RB * KB);
     g.C = pl.C;
+    plan_units(RB, KB, pl.C, g.work);
     g.D = pl.D;
     g.NP = pl.NP;
     g.early_weights = pdl_mode == 2 ? 1 : 0;

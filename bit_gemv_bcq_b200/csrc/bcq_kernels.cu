@@ -347,39 +347,20 @@ __device__ __forceinline__ float half_at(uint32_t r, int hi) {
   return h2f((uint16_t)(hi ? (r >> 16) : (r & 0xFFFFu)));
 }
 
-// The units of one CTA: [u0, u1) in kb-major order, cut into groups: the
-// row-blocks of one K-block inside one row group (at most kRowGroup).  When
-// the CTAs divide evenly among the K-blocks, each CTA keeps to one K-block;
-// otherwise the units are shared out evenly (the first U mod C CTAs take one
-// more).
+// The units of one CTA: [u0, u1) in kb-major order (the host's split: see
+// plan_units), cut into groups: the row-blocks of one K-block inside one row
+// group (at most kRowGroup).
 struct CtaRange {
   int u0, u1, NG, kb0, kb_last;
 };
 
 __device__ __forceinline__ void make_range(const GemvParams& p, CtaRange& R) {
-  const int c = (int)blockIdx.x;
-  if (p.C >= p.KB && p.C % p.KB == 0) {
-    // whole K-blocks: C / KB CTAs share the row-blocks of each K-block
-    const int cpk = p.C / p.KB, kb = c / cpk, j = c - kb * cpk;
-    const int q = p.RB / cpk, r = p.RB % cpk;
-    R.u0 = kb * p.RB + j * q + min(j, r);
-    R.u1 = R.u0 + q + (j < r ? 1 : 0);
-  } else {
-    const int q = p.U / p.C, r = p.U % p.C;
-    R.u0 = c * q + min(c, r);
-    R.u1 = R.u0 + q + (c < r ? 1 : 0);
-  }
-  int ng = 0;
-  for (int u = R.u0; u < R.u1;) {
-    const int kb = u / p.RB;
-    const int end = min(R.u1, (kb + 1) * p.RB);
-    const int a = u - kb * p.RB, b = end - kb * p.RB;  // row-blocks [a, b) of kb
-    ng += (b + kRowGroup - 1) / kRowGroup - a / kRowGroup;
-    u = end;
-  }
-  R.NG = ng;
-  R.kb0 = R.u0 / p.RB;
-  R.kb_last = R.u1 > R.u0 ? (R.u1 - 1) / p.RB : R.kb0;
+  const CtaWork w = p.work[blockIdx.x];
+  R.u0 = w.u0;
+  R.u1 = w.u1;
+  R.NG = w.ng;
+  R.kb0 = w.kb & 0xFFFF;
+  R.kb_last = w.kb >> 16;
 }
 
 // Walks the groups of a CTA in order: K-block kb, first row-block rb0, n
@@ -389,8 +370,8 @@ struct GroupCursor {
   int kb, rb0, n, seg_end;
 };
 
-__device__ __forceinline__ void cursor_init(GroupCursor& c, int u0, int u1, int RB) {
-  c.kb = u0 / RB;
+__device__ __forceinline__ void cursor_init(GroupCursor& c, int u0, int u1, int kb0, int RB) {
+  c.kb = kb0;
   c.rb0 = u0 - c.kb * RB;
   c.seg_end = min(RB, u1 - c.kb * RB);
   c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
@@ -450,8 +431,6 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   const uint32_t full0 = sbase + gemv_off_bar(D, P);
   const uint32_t empty0 = full0 + 8u * (uint32_t)D;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + gemv_off_misc(D, P));
-  int* nlist = reinterpret_cast<int*>(smem + gemv_off_misc(D, P) + 4);
-  int* list = reinterpret_cast<int*>(smem + gemv_off_misc(D, P) + 16);
   constexpr int kConsumers = kConsumerWarps * 32;
 
   // The table is addressed through load immediates: the dynamic shared
@@ -459,8 +438,16 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   // the stage D earlier (D even: teams alternate), and each producer refills
   // only its own slots (D a multiple of NP).
   const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 &&
-                      D % NP == 0 && D % 2 == 0 &&
-                      (int)blockDim.x == 32 * (kConsumerWarps + NP);
+                      (D & 1) == 0 && (int)blockDim.x == 32 * (kConsumerWarps + NP);
+  CtaRange R;
+  make_range(prm, R);
+  // consumers: activations of the first table first of all (x may come
+  // from the preceding grid: wait for it)
+  uint4 xv[M];
+  if (warp < kConsumerWarps) {
+    grid_dependency_wait();
+    load_x<M>(prm.x, prm.K, R.kb0, lane, xv);
+  }
   if (warp == 0) {
     if (cfg_ok && lane < D) {  // one lane per ring slot
       mbar_init(full0 + 8u * lane, 1);
@@ -476,9 +463,6 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   launch_dependents();
   if (*abort_flag) return;  // set before the barrier: uniform
 
-  CtaRange R;
-  make_range(prm, R);
-
   if (warp >= kConsumerWarps) {
     // ------------------------------------------------------------ producers
     // Producer pw issues stages (groups) k = pw, pw + NP, ...; with D a
@@ -491,12 +475,12 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     if (lane == 0) {
       int issued = 0;
       GroupCursor gc;
-      cursor_init(gc, R.u0, R.u1, RB);
-      for (int k = 0; k < R.NG; ++k, cursor_next(gc, R.u1, RB)) {
-        if (k % NP != pw) continue;
-        const int s = k % D;
-        if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, (uint32_t)(((k / D) - 1) & 1),
-                                         prm.timeout_ns)) {
+      cursor_init(gc, R.u0, R.u1, R.kb0, RB);
+      if (pw) cursor_next(gc, R.u1, RB);
+      int s = pw;          // ring slot of stage k (incremental: no division)
+      uint32_t eph = 1;    // parity of the empty phase that frees slot s (k - D)
+      for (int k = pw; k < R.NG; k += NP) {
+        if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, eph, prm.timeout_ns)) {
           record_error(&g_device_error, BCQ_ERR_TIMEOUT);
           *abort_flag = 1;
         }
@@ -517,6 +501,12 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
                      (uint32_t)gc.n * kUnitPlaneBytes, bar);
         }
         issued = k + 1;
+        for (int t = 0; t < NP; ++t) cursor_next(gc, R.u1, RB);
+        s += NP;
+        if (s >= D) {
+          s -= D;
+          eph ^= 1u;
+        }
       }
       // every copy this warp issued lands before the CTA may exit
       for (int s = pw; s < D && s < issued; s += NP) {
@@ -529,13 +519,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   }
 
   // -------------------------------------------------------------- consumers
-  grid_dependency_wait();  // x, y and the workspace may belong to earlier work
   const int team = warp / kTeamWarps;
   const int tw = warp % kTeamWarps;  // row-block of a stage
   GroupCursor gc;                    // this team's next group
-  cursor_init(gc, R.u0, R.u1, RB);
-  uint4 xv[M];                       // activations of the first table, first of all
-  load_x<M>(prm.x, prm.K, gc.kb, lane, xv);
+  cursor_init(gc, R.u0, R.u1, R.kb0, RB);
   uint32_t cr0[4][2], cr1[4][2];
   column_regs<M>(lane, cr0, cr1);
   int cr_slot = 0;
@@ -729,33 +716,30 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   advance_tables(R.kb_last);  // the same barriers in both teams
 
   // Split-K: every unit's partial sums are in the workspace.  Each CTA
-  // counts its arrivals (release), then reduces the row-blocks it is
-  // designated for -- row-block rb belongs to the CTA that computed its unit
-  // in K-block rb mod KB, so the work is spread evenly whatever the order in
-  // which CTAs finish.  The reducer waits (bounded) until all KB partials of
-  // rb have arrived, adds them in K-block order (the result does not depend
-  // on scheduling) and clears them and the counter, so the whole workspace
-  // is zero again for the next call, whatever its shape.
+  // counts its arrivals (fence, then release), then reduces the row-blocks
+  // it is designated for -- row-block rb belongs to the CTA that computed its
+  // unit in K-block rb mod KB, so the work is spread evenly whatever the
+  // order in which CTAs finish.  The reducer waits (bounded) until all KB
+  // partials of rb have arrived, adds them in K-block order (the result does
+  // not depend on scheduling) and clears them and the counter, so the whole
+  // workspace is zero again for the next call, whatever its shape.
   if (prm.KB > 1) {
-    __threadfence();
-    named_barrier_sync(1, kConsumers);
-    if (*abort_flag == 0) {
-      for (int u = R.u0 + tid; u < R.u1; u += kConsumers) red_add_release(prm.cnt + u % RB, 1u);
-    }
-    // this CTA's row-blocks to reduce: units (kb, rb) with kb == rb mod KB,
-    // taken kReduceBatch units at a time (the list holds one batch)
-    for (int base = R.u0; base < R.u1; base += kReduceBatch) {
-      if (tid == 0) *nlist = 0;
-      named_barrier_sync(1, kConsumers);
-      if (tid < kReduceBatch && base + tid < R.u1) {
-        const int u = base + tid;
-        const int rbx = u % RB;
-        if (u / RB == rbx % prm.KB) list[atomicAdd(nlist, 1)] = rbx;
+    named_barrier_sync(1, kConsumers);  // every partial of the CTA is stored
+    const bool live = *abort_flag == 0;
+    for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
+      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+      for (int rb = a + tid; rb < b; rb += kConsumers) {
+        __threadfence();  // cumulative over the barrier: the CTA's stores
+        red_add_release(prm.cnt + rb, 1u);
       }
-      named_barrier_sync(1, kConsumers);
-      const int nl = *abort_flag == 0 ? *reinterpret_cast<volatile int*>(nlist) : 0;
-      for (int e = warp; e < nl; e += kConsumerWarps) {
-        const int rbx = list[e];
+    }
+    for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
+      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+      int first = kb;  // designated row-blocks: kb, kb + KB, ...
+      if (first < a) first += (a - first + prm.KB - 1) / prm.KB * prm.KB;
+      for (int rbx = first + warp * prm.KB; rbx < b; rbx += kConsumerWarps * prm.KB) {
         bool ready = true;
         if (lane == 0)
           ready = wait_count(prm.cnt + rbx, (unsigned int)prm.KB, abort_flag, prm.timeout_ns);
@@ -785,7 +769,6 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
         __syncwarp();
         if (lane == 0) *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
       }
-      named_barrier_sync(1, kConsumers);
     }
   }
 }

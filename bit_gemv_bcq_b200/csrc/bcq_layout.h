@@ -85,6 +85,13 @@ __host__ __device__ constexpr uint32_t gemv_dyn_bytes(int D, int P) {
   return gemv_off_misc(D, P) + 16u + 4u * kReduceBatch;
 }
 
+// Units of one CTA, computed on the host: [u0, u1), its group count and
+// first and last K-blocks (no integer division on the device).
+struct CtaWork {
+  int u0, u1, ng, kb;  // kb: first K-block (bits 0-15), last K-block (16-31)
+};
+constexpr int kMaxCtas = 256;
+
 struct GemvParams {
   const uint16_t* x;         // fp16 [M][K] (rows of this launch)
   const uint32_t* planes;    // packed planes
@@ -100,6 +107,7 @@ struct GemvParams {
   int D, NP;                 // ring stages, producer warps
   int early_weights;         // with PDL: stream weights before the grid wait
   unsigned long long timeout_ns;
+  CtaWork work[kMaxCtas];    // per CTA (C entries)
 };
 
 struct LutParams {

@@ -47,6 +47,30 @@ def algo_bytes(N, K, M, p):
     return N * K * p // 8 + N * G * p * 2 + N * G * 2 + M * K * 2 + M * N * 2
 
 
+def csrc_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "bit_gemv_bcq_b200", "csrc")
+    for f in sorted(os.listdir(src)):
+        h.update(f.encode())
+        with open(os.path.join(src, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu launch list, or None when
+    the kernel sources changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        if t.get("csrc_sha256") != csrc_sha256():
+            return None
+        return t
+    except Exception:
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -378,6 +402,12 @@ def main():
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
     }
+    tr = recorded_traffic()
+    if tr is not None:
+        line["roofline"]["traffic"] = round(tr["dram_bytes_per_launch"])
+        line["roofline"]["traffic_per"] = "launch (mean over one step's launches, ncu launch list)"
+        line["roofline"]["algorithmic_bytes_per_launch"] = round(tr["algorithmic_bytes_per_launch"])
+        line["roofline"]["traffic_source"] = tr["source"]
     m1 = [c for c in res["per_case"] if c["M"] == 1]
     line["headline_m1"] = {f"p{c['p']}": {"us": c["us"], "GBps": c["GBps"],
                                           "frac": round(c["GBps"] / peak, 4)} for c in m1}

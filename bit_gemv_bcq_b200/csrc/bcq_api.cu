@@ -21,6 +21,8 @@ constexpr int kVersion = 200;                // 0.2.0
 constexpr size_t kMaxDynSmem = 232448;       // 227 KiB per CTA on sm_100
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
 constexpr int kDefaultProducers = 2;
+// Calls with at least this many rows take the tensor-core path.
+constexpr int kDefaultMmaMinRows = 3;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -39,12 +41,12 @@ size_t k_blocks(int K) { return ((size_t)K + kKBlock - 1) / kKBlock; }
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace: arrival counters [RB] (256-byte aligned), then fp32 partial
-// sums [KB][min(M, 2)][RB * 32].
+// sums [KB][min(M, 16)][RB * 32] (the rows of the largest launch).
 size_t counter_bytes(int N) { return align256(row_blocks(N) * sizeof(unsigned int)); }
 size_t workspace_bytes(int M, int N, int K) {
   const size_t KB = k_blocks(K);
   if (M < 1 || KB <= 1) return 0;
-  const size_t ml = (size_t)std::min(M, kMaxMPerLaunch);
+  const size_t ml = (size_t)std::min(M, kMmaRows);
   return counter_bytes(N) + KB * ml * row_blocks(N) * kRowBlock * sizeof(float);
 }
 
@@ -99,13 +101,14 @@ struct Plan {
 // of one K-block) fed by NP producer warps, as deep as shared memory allows
 // beside the 64 KiB table; D is even (a stage's team consumed the stage D
 // earlier) and a multiple of NP (a producer refills only its own slots).
-bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, Plan* out) {
+bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, bool mma, Plan* out) {
   DeviceCache* dc = nullptr;
   bcq_status st = get_device(&dc);
   if (st != BCQ_OK) return st;
   Plan pl;
-  pl.fn = gemv_kernel_for(M, P, mixed);
+  pl.fn = mma ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P) : gemv_kernel_for(M, P, mixed);
   if (!pl.fn) return BCQ_ERR_UNSUPPORTED;
+  auto dyn_of = [&](int d) { return mma ? mma_dyn_bytes(d, P) : gemv_dyn_bytes(d, P); };
   const long long RB = (long long)row_blocks(N);
   const long long KB = (long long)k_blocks(K);
   const long long U = RB * KB;
@@ -115,10 +118,10 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, Plan* out) {
   int D = env_int("BCQ_FORCE_D", kMaxStages);
   D = std::min(kMaxStages, D) / step * step;
   if (D < step) D = step;
-  while (D > step && gemv_dyn_bytes(D, P) > kMaxDynSmem) D -= step;
+  while (D > step && dyn_of(D) > kMaxDynSmem) D -= step;
   const int nthreads = 32 * (kConsumerWarps + pl.NP);
   while (true) {
-    pl.dyn = gemv_dyn_bytes(D, P);
+    pl.dyn = dyn_of(D);
     int per_sm = 0;
     if (pl.dyn <= kMaxDynSmem) {
       if (t_virtual) {
@@ -219,15 +222,65 @@ void plan_units(int RB, int KB, int C, CtaWork* work) {
   }
 }
 
-// Launches of at most two rows, in order; two rows with different
-// precisions share one launch (planes streamed up to the larger one).
+// Fills the fields every launch shares.
+void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const uint16_t* z,
+                 int N, int K, int p_H, void* ws, int pdl_mode, int wait_us) {
+  const int RB = (int)row_blocks(N);
+  const int KB = (int)k_blocks(K);
+  g.planes = planes;
+  g.z = z;
+  g.cnt = KB > 1 ? static_cast<unsigned int*>(ws) : nullptr;
+  g.part = KB > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + counter_bytes(N))
+                  : nullptr;
+  g.N = N;
+  g.K = K;
+  g.KB = KB;
+  g.RB = RB;
+  g.RG = (RB + kRowGroup - 1) / kRowGroup;
+  g.p_H = p_H;
+  g.U = (int)((long long)RB * KB);
+  g.C = pl.C;
+  plan_units(RB, KB, pl.C, g.work);
+  g.D = pl.D;
+  g.NP = pl.NP;
+  g.early_weights = pdl_mode == 2 ? 1 : 0;
+  g.timeout_ns = wait_us > 0 ? (unsigned long long)wait_us * 1000ull : kDefaultWaitNs;
+}
+
+// Small batches: lookup-table launches of at most two rows, in order; two
+// rows with different precisions share one launch (planes streamed up to
+// the larger one).  Larger batches: tensor-core launches of up to 16 rows of
+// one precision each (rows grouped by precision, in order).
 bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
                     const uint16_t* z, int p, const int32_t* p_row, int M, int N, int K,
                     int p_H, uint16_t* y, void* ws, cudaStream_t st) {
   const int pdl_mode = g_pdl_mode.load();
   const int wait_us = env_int("BCQ_WAIT_LIMIT_US", 0);
-  const int RB = (int)row_blocks(N);
-  const int KB = (int)k_blocks(K);
+  const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
+  if (M >= mma_min) {
+    for (int q = 1; q <= 4; ++q) {
+      int rows[BCQ_MAX_M];
+      int n = 0;
+      for (int m = 0; m < M; ++m)
+        if ((p > 0 ? p : p_row[m]) == q) rows[n++] = m;
+      for (int r0 = 0; r0 < n; r0 += kMmaRows) {
+        const int cnt = std::min(kMmaRows, n - r0);
+        Plan pl;
+        bcq_status s = plan_gemv(cnt, N, K, q, false, true, &pl);
+        if (s != BCQ_OK) return s;
+        GemvParams g{};
+        fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
+        g.x = x;
+        g.y = y;
+        g.alpha[0] = g.alpha[1] = alpha[q - 1];
+        g.M = cnt;
+        g.q[0] = g.q[1] = q;
+        for (int j = 0; j < cnt; ++j) g.rows[j] = rows[r0 + j];
+        if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st) != cudaSuccess) return BCQ_ERR_CUDA;
+      }
+    }
+    return BCQ_OK;
+  }
   for (int m0 = 0; m0 < M;) {
     const int rows = std::min(kMaxMPerLaunch, M - m0);
     int q[2];
@@ -236,34 +289,17 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
     const int P = std::max(q[0], q[1]);
     const bool mixed = q[0] != q[1];
     Plan pl;
-    bcq_status s = plan_gemv(rows, N, K, P, mixed, &pl);
+    bcq_status s = plan_gemv(rows, N, K, P, mixed, false, &pl);
     if (s != BCQ_OK) return s;
     GemvParams g{};
+    fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
     g.x = x + (size_t)m0 * K;
-    g.planes = planes;
+    g.y = y + (size_t)m0 * N;
     g.alpha[0] = alpha[q[0] - 1];
     g.alpha[1] = alpha[q[1] - 1];
-    g.z = z;
-    g.y = y + (size_t)m0 * N;
-    g.cnt = KB > 1 ? static_cast<unsigned int*>(ws) : nullptr;
-    g.part = KB > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + counter_bytes(N))
-                    : nullptr;
     g.M = rows;
-    g.N = N;
-    g.K = K;
-    g.KB = KB;
-    g.RB = RB;
-    g.RG = (RB + kRowGroup - 1) / kRowGroup;
-    g.p_H = p_H;
     g.q[0] = q[0];
     g.q[1] = q[1];
-    g.U = (int)((long long)RB * KB);
-    g.C = pl.C;
-    plan_units(RB, KB, pl.C, g.work);
-    g.D = pl.D;
-    g.NP = pl.NP;
-    g.early_weights = pdl_mode == 2 ? 1 : 0;
-    g.timeout_ns = wait_us > 0 ? (unsigned long long)wait_us * 1000ull : kDefaultWaitNs;
     if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st) != cudaSuccess) return BCQ_ERR_CUDA;
     m0 += rows;
   }
@@ -333,15 +369,16 @@ size_t bcq_workspace_bytes(int M, int N, int K) {
 
 int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, int* out) {
   if (!out) return BCQ_ERR_NULL;
-  if (M < 1 || M > kMaxMPerLaunch || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
+  if (M < 1 || M > kMmaRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
   if (p_load < 1 || p_load > 4) return BCQ_ERR_PRECISION;
-  if (mixed && (M < 2 || p_load < 2)) return BCQ_ERR_PRECISION;
+  if (mixed && (M != 2 || p_load < 2)) return BCQ_ERR_PRECISION;
+  const bool mma = M > kMaxMPerLaunch;
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;
   if (t_virtual) (void)cudaGetLastError();
   Plan pl;
-  bcq_status st = plan_gemv(M, N, K, p_load, mixed != 0, &pl);
+  bcq_status st = plan_gemv(M, N, K, p_load, mixed != 0, mma, &pl);
   t_virtual = false;
   if (st != BCQ_OK) return st;
   out[0] = pl.C;

@@ -24,12 +24,10 @@
 #include "bcq_device.cuh"
 #include "bcq_launch.h"
 #include "bcq_layout.h"
+#include "bcq_pipeline.cuh"
 
 namespace bcq {
 
-// Device error word of this library (one per device): kernels record the
-// first problem they hit; bcq_device_error() reads and clears it.
-__device__ int g_device_error = 0;
 
 // ============================================================ pack planes
 
@@ -347,66 +345,6 @@ __device__ __forceinline__ float half_at(uint32_t r, int hi) {
   return h2f((uint16_t)(hi ? (r >> 16) : (r & 0xFFFFu)));
 }
 
-// The units of one CTA: [u0, u1) in kb-major order (the host's split: see
-// plan_units), cut into groups: the row-blocks of one K-block inside one row
-// group (at most kRowGroup).
-struct CtaRange {
-  int u0, u1, NG, kb0, kb_last;
-};
-
-__device__ __forceinline__ void make_range(const GemvParams& p, CtaRange& R) {
-  const CtaWork w = p.work[blockIdx.x];
-  R.u0 = w.u0;
-  R.u1 = w.u1;
-  R.NG = w.ng;
-  R.kb0 = w.kb & 0xFFFF;
-  R.kb_last = w.kb >> 16;
-}
-
-// Walks the groups of a CTA in order: K-block kb, first row-block rb0, n
-// row-blocks (all in row group rb0 / kRowGroup); seg_end bounds the
-// row-blocks of kb inside the CTA's range.
-struct GroupCursor {
-  int kb, rb0, n, seg_end;
-};
-
-__device__ __forceinline__ void cursor_init(GroupCursor& c, int u0, int u1, int kb0, int RB) {
-  c.kb = kb0;
-  c.rb0 = u0 - c.kb * RB;
-  c.seg_end = min(RB, u1 - c.kb * RB);
-  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
-}
-
-__device__ __forceinline__ void cursor_next(GroupCursor& c, int u1, int RB) {
-  c.rb0 += c.n;
-  if (c.rb0 >= c.seg_end) {
-    ++c.kb;
-    c.rb0 = 0;
-    c.seg_end = min(RB, u1 - c.kb * RB);
-  }
-  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
-}
-
-// Waits for phase `parity` of a stage barrier: a non-blocking test first
-// (the common case: the stage has landed), then bounded waiting that gives
-// up when the CTA aborts.
-__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity,
-                                           volatile int* abort_flag,
-                                           unsigned long long limit_ns) {
-  if (mbar_test(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-#pragma unroll 1
-  while (true) {
-    if (*abort_flag) return false;
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-}
-
-template <int J>
-struct Slot {
-  static constexpr int value = J;
-};
 
 // One CTA per SM: units [u0, u1) of the launch in kb-major order.  Warps
 // 0..15 consume, in two teams of 8 that take alternate groups; the NP warps
@@ -464,57 +402,8 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   if (*abort_flag) return;  // set before the barrier: uniform
 
   if (warp >= kConsumerWarps) {
-    // ------------------------------------------------------------ producers
-    // Producer pw issues stages (groups) k = pw, pw + NP, ...; with D a
-    // multiple of NP it alone refills its ring slots, so the empty-barrier
-    // phase it waits for is never two phases behind.  A whole row group is
-    // one bulk copy of its first P planes; a partial one (at the ends of the
-    // CTA's range) one copy per plane.
-    const int pw = warp - kConsumerWarps;
-    if (!prm.early_weights) grid_dependency_wait();
-    if (lane == 0) {
-      int issued = 0;
-      GroupCursor gc;
-      cursor_init(gc, R.u0, R.u1, R.kb0, RB);
-      if (pw) cursor_next(gc, R.u1, RB);
-      int s = pw;          // ring slot of stage k (incremental: no division)
-      uint32_t eph = 1;    // parity of the empty phase that frees slot s (k - D)
-      for (int k = pw; k < R.NG; k += NP) {
-        if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, eph, prm.timeout_ns)) {
-          record_error(&g_device_error, BCQ_ERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        if (*abort_flag) break;
-        const uint32_t bar = full0 + 8u * s;
-        const uint32_t dst = sbase + kLutBytes + (uint32_t)s * kStage;
-        const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
-        const uint32_t* src = prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H *
-                                               (kRowGroup * kWordsPerUnitPlane);
-        mbar_arrive_expect_tx(bar, (uint32_t)(P * gc.n) * kUnitPlaneBytes);
-        if (gc.n == kRowGroup) {
-          bulk_g2s(dst, src, kStage, bar);
-        } else {
-#pragma unroll
-          for (int i = 0; i < P; ++i)
-            bulk_g2s(dst + (uint32_t)i * kPlaneGroupBytes,
-                     src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
-                     (uint32_t)gc.n * kUnitPlaneBytes, bar);
-        }
-        issued = k + 1;
-        for (int t = 0; t < NP; ++t) cursor_next(gc, R.u1, RB);
-        s += NP;
-        if (s >= D) {
-          s -= D;
-          eph ^= 1u;
-        }
-      }
-      // every copy this warp issued lands before the CTA may exit
-      for (int s = pw; s < D && s < issued; s += NP) {
-        const int klast = issued - 1 - ((issued - 1 - s) % D);
-        (void)mbar_wait_bounded(full0 + 8u * s, (uint32_t)((klast / D) & 1), prm.timeout_ns);
-      }
-    }
-    __syncwarp();
+    produce_stages<P>(prm, R, warp - kConsumerWarps, lane, sbase + kLutBytes, full0, empty0,
+                      abort_flag);
     return;
   }
 
@@ -715,63 +604,18 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   finish(Slot<1>{});
   advance_tables(R.kb_last);  // the same barriers in both teams
 
-  // Split-K: every unit's partial sums are in the workspace.  Each CTA
-  // counts its arrivals (fence, then release), then reduces the row-blocks
-  // it is designated for -- row-block rb belongs to the CTA that computed its
-  // unit in K-block rb mod KB, so the work is spread evenly whatever the
-  // order in which CTAs finish.  The reducer waits (bounded) until all KB
-  // partials of rb have arrived, adds them in K-block order (the result does
-  // not depend on scheduling) and clears them and the counter, so the whole
-  // workspace is zero again for the next call, whatever its shape.
+  // split-K reduction (a no-op when the launch has one K-block)
   if (prm.KB > 1) {
     named_barrier_sync(1, kConsumers);  // every partial of the CTA is stored
-    const bool live = *abort_flag == 0;
-    for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
-      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
-      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
-      for (int rb = a + tid; rb < b; rb += kConsumers) {
-        __threadfence();  // cumulative over the barrier: the CTA's stores
-        red_add_release(prm.cnt + rb, 1u);
-      }
-    }
-    for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
-      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
-      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
-      int first = kb;  // designated row-blocks: kb, kb + KB, ...
-      if (first < a) first += (a - first + prm.KB - 1) / prm.KB * prm.KB;
-      for (int rbx = first + warp * prm.KB; rbx < b; rbx += kConsumerWarps * prm.KB) {
-        bool ready = true;
-        if (lane == 0)
-          ready = wait_count(prm.cnt + rbx, (unsigned int)prm.KB, abort_flag, prm.timeout_ns);
-        ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
-        if (!ready) {
-          if (lane == 0 && *abort_flag == 0) {
-            record_error(&g_device_error, BCQ_ERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          continue;
-        }
-        const int row = rbx * kRowBlock + lane;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
-          float sum = 0.f;
-#pragma unroll 8
-          for (int k = 0; k < prm.KB; ++k) sum += ldg_cg_f32(pp + (size_t)k * M * part_stride);
-          if (row < prm.N) prm.y[(size_t)m * prm.N + row] = f2h_rn(sum);
-        }
-        // the workspace is left zero-filled for any later shape
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
-          for (int k = 0; k < prm.KB; ++k) stg_cg_zero(pp + (size_t)k * M * part_stride);
-        }
-        __syncwarp();
-        if (lane == 0) *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
-      }
-    }
+    splitk_tail(prm, R, M, nullptr, tid, kConsumers, abort_flag);
   }
 }
+
+}  // namespace bcq
+
+#include "bcq_mma.cuh"
+
+namespace bcq {
 
 // ============================================================ LUT dump
 
@@ -877,6 +721,28 @@ GemvKernel gemv_kernel_for(int M, int P, bool mixed) {
       case 2: return gemv_lut_kernel<2, 2, true>;
       case 3: return gemv_lut_kernel<2, 3, true>;
       case 4: return gemv_lut_kernel<2, 4, true>;
+      default: return nullptr;
+    }
+  }
+  return nullptr;
+}
+
+GemvKernel gemv_mma_kernel_for(int NT, int P) {
+  if (NT == 1) {
+    switch (P) {
+      case 1: return gemv_mma_kernel<1, 1>;
+      case 2: return gemv_mma_kernel<1, 2>;
+      case 3: return gemv_mma_kernel<1, 3>;
+      case 4: return gemv_mma_kernel<1, 4>;
+      default: return nullptr;
+    }
+  }
+  if (NT == 2) {
+    switch (P) {
+      case 1: return gemv_mma_kernel<2, 1>;
+      case 2: return gemv_mma_kernel<2, 2>;
+      case 3: return gemv_mma_kernel<2, 3>;
+      case 4: return gemv_mma_kernel<2, 4>;
       default: return nullptr;
     }
   }

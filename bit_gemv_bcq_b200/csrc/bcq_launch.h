@@ -21,7 +21,11 @@ cudaError_t launch_pack_scales(const uint16_t* src, uint16_t* dst, int q, int N,
 // the rows use different precisions.  nullptr if there is none.
 GemvKernel gemv_kernel_for(int M, int P, bool mixed);
 
-// p.C CTAs of 32 * (8 + p.NP) threads.
+// The tensor-core GEMV kernel for NT n-tiles of 8 activation rows (1 or 2)
+// streaming P planes (one precision); nullptr if there is none.
+GemvKernel gemv_mma_kernel_for(int NT, int P);
+
+// p.C CTAs of 32 * (16 + p.NP) threads.
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,
                         cudaStream_t st);
 

@@ -92,6 +92,28 @@ struct CtaWork {
 };
 constexpr int kMaxCtas = 256;
 
+// The tensor-core GEMV (bcq_mma.cuh): activations of the current K-block
+// (two slots, 16 rows of 256 columns padded to 264 halves so fragment loads
+// hit distinct banks) and their group sums, then per-warp double buffers of
+// scales and offsets, then the ring.
+constexpr int kMmaRows = 16;                 // activation rows per tensor-core launch (max)
+constexpr int kXPitch = 264;                 // halves per row of the activation tile
+constexpr uint32_t kXTileBytes = kMmaRows * kXPitch * 2;            // 8448
+constexpr uint32_t kMmaGsumOff = 2 * kXTileBytes;                    // 16896
+constexpr uint32_t kMmaScaleOff = kMmaGsumOff + 2 * kMmaRows * 2 * 4; // 17152
+__host__ __device__ constexpr uint32_t mma_scale_buf_bytes(int P) {  // one warp, one group
+  return (uint32_t)32 * (2 * P + 2) * 2;
+}
+__host__ __device__ constexpr uint32_t mma_ring_off(int P) {
+  return (kMmaScaleOff + 16u * 2u * mma_scale_buf_bytes(P) + 1023u) & ~1023u;
+}
+__host__ __device__ constexpr uint32_t mma_off_bar(int D, int P) {
+  return mma_ring_off(P) + (uint32_t)D * gemv_stage_bytes(P);
+}
+__host__ __device__ constexpr uint32_t mma_dyn_bytes(int D, int P) {
+  return mma_off_bar(D, P) + 16u * (uint32_t)D + 16u;
+}
+
 struct GemvParams {
   const uint16_t* x;         // fp16 [M][K] (rows of this launch)
   const uint32_t* planes;    // packed planes
@@ -107,6 +129,7 @@ struct GemvParams {
   int D, NP;                 // ring stages, producer warps
   int early_weights;         // with PDL: stream weights before the grid wait
   unsigned long long timeout_ns;
+  int rows[kMmaRows];        // tensor-core launches: x / y row of launch row m
   CtaWork work[kMaxCtas];    // per CTA (C entries)
 };
 

@@ -1,0 +1,405 @@
+// bcq_mma.cuh -- the tensor-core BCQ GEMV (included by bcq_kernels.cu only).
+//
+// For a batch of up to 16 activation rows the lookup table costs grow with
+// the batch; here each plane is instead expanded in registers into fp16
+// matrix fragments holding +-alpha (alpha^(p)[n][g][i] with the sign of the
+// plane bit: bit 1 -> +alpha, 0 -> -alpha, exact in fp16) and multiplied with
+// the activations on the tensor cores (mma.sync m16n8k16, fp32 accumulate):
+//   y[m][n] = sum_g sum_i sum_{k in g} (+-alpha) x[m][k]  +  sum_g z[n][g] S[m][g]
+// which is the same sum as the lookup path (AnyBCQ Paper-Notes page, 关键设计
+// / 直接bit-plane运算的CUDA内核: plane-by-plane contraction with alpha_i,
+// offsets per group from 训练策略), with no dequantised weight matrix: each
+// plane term is formed from the bits and alpha only, in registers.
+//
+// The planes are read from the same packed layout as the lookup path (one
+// bulk copy per row group and K-block into the ring); the producer warps,
+// the CTA's unit ranges and the split-K reduction are shared with it
+// (bcq_pipeline.cuh).
+#pragma once
+
+#include <cstdint>
+
+#include "bcq_device.cuh"
+#include "bcq_layout.h"
+#include "bcq_pipeline.cuh"
+
+namespace bcq {
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t funnel_r(uint32_t lo, uint32_t hi, uint32_t sh) {
+  uint32_t d;
+  asm("shf.r.clamp.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(lo), "r"(hi), "r"(sh));
+  return d;
+}
+
+// a ^ (~b & c) in one instruction.
+__device__ __forceinline__ uint32_t xor_andnot(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xD2;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Lane l of a warp copies row l's scales (2P halves: pass 0 then pass 1) and
+// offsets (2 halves) of unit (kb, rb) into buf: alpha at l * 4P bytes, z at
+// 128P + 4l.  Packed layouts: bcq_layout.h.
+template <int P>
+__device__ __forceinline__ void stage_scales(const GemvParams& prm, int kb, int rb, int lane,
+                                             uint32_t buf) {
+  const size_t e = ((size_t)kb * prm.RB + rb) * kRowBlock + lane;
+  const uint16_t* a = prm.alpha[0] + e * (2 * P);
+  const uint32_t da = buf + (uint32_t)lane * (4u * P);
+  if (P == 1) {
+    cp_async4(da, a);
+  } else if (P == 2) {
+    cp_async8(da, a);
+  } else if (P == 3) {
+    cp_async4(da, a);
+    cp_async4(da + 4u, a + 2);
+    cp_async4(da + 8u, a + 4);
+  } else {
+    cp_async16(da, a);
+  }
+  if (prm.z) cp_async4(buf + 128u * P + 4u * lane, prm.z + e * 2);
+}
+
+// The 16-row activation tile of K-block kb into slot (kb & 1), rows beyond
+// the launch's M zero, and its group sums gs[slot][m][h].  All 16 consumer
+// warps: warp w loads row w (lane l: columns 8l .. 8l + 7).
+__device__ __forceinline__ void load_x_tile(const GemvParams& prm, int kb, int warp, int lane,
+                                            uint4& v) {
+  const int k = kb * kKBlock + lane * 8;
+  v = make_uint4(0u, 0u, 0u, 0u);
+  if (warp < prm.M && k < prm.K) {
+    const uint16_t* p = prm.x + (size_t)prm.rows[warp] * prm.K + k;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+  }
+}
+
+__device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, int lane,
+                                             const uint4& v) {
+  const uint32_t slot = (uint32_t)(kb & 1);
+  const uint32_t t = sbase + slot * kXTileBytes + (uint32_t)(warp * kXPitch + lane * 8) * 2u;
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(t), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+  float f[8];
+  unpack8(v, f);
+  float s = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if ((lane & 15) == 0)  // lane 0: group A, lane 16: group B
+    sts_f32(sbase + kMmaGsumOff + ((slot * kMmaRows + warp) * 2 + (lane >> 4)) * 4u, s);
+}
+
+// One plane of one row-block for this warp: both 16-row tiles, both groups,
+// all 16 k-steps.  rot: the stage bytes of this row-block and plane;
+// thread (g = lane / 4, q = lane % 4) holds rows g, g + 8, g + 16, g + 24.
+//
+// The packed bytes of row r are rotated by r mod 16 (see bcq_layout.h); the
+// natural 4-byte word v of a pass (chunks 4v .. 4v + 3) starts at rotated
+// byte (4v - rho) mod 16, rho = r mod 16: it is the funnel shift of rotated
+// words (v - R) mod 4 and (v - R + 1) mod 4 by 8 delta bits, with
+// R = ceil(rho / 4) mod 4 and delta = (-rho) mod 4 -- per-thread constants.
+// A fragment element pair (columns 2q, 2q + 1 of an 8-column chunk) becomes
+// +-alpha by moving the two bits to bit 7 of their byte (shifts by 7 - 2q and
+// 6 - 2q), replicating each into a sign byte (prmt) and xoring the fp16 sign
+// bits of alpha2 (lop3).
+template <int NT, int P>
+__device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sbuf, int i,
+                                          int g, int q, uint32_t ra0, uint32_t ra1, uint32_t dsh,
+                                          float (&acc)[2][2][NT][4]) {
+  const uint32_t sh1 = 7u - 2u * (uint32_t)q, sh2 = 6u - 2u * (uint32_t)q;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    // activation fragments of the group's 8 k-steps, off the critical path
+    uint32_t bf[8][NT][2];
+#pragma unroll
+    for (int s8 = 0; s8 < 8; ++s8)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t bx =
+            xt + (uint32_t)((nt * 8 + g) * kXPitch + h * 128 + s8 * 16 + 2 * q) * 2u;
+        bf[s8][nt][0] = lds_u32(bx);
+        bf[s8][nt][1] = lds_u32(bx + 16u);
+      }
+    // natural words of group h for rows g, g + 8, g + 16, g + 24
+    uint32_t nw[4][4];
+    uint32_t al[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = g + 8 * j;          // row in the row-block
+      const int pass = (j >> 1) ^ h;    // rows >= 16 hold group A in pass 1
+      const uint32_t ra = (j & 1) ? ra1 : ra0;  // R of this row's rotation
+      const uint32_t base = rot + (uint32_t)pass * 512u + (uint32_t)r * 16u;
+      uint32_t w[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) w[v] = lds_u32(base + (((uint32_t)v - ra) & 3u) * 4u);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) nw[j][v] = funnel_r(w[v], w[(v + 1) & 3], dsh);
+      // alpha of (row, group h, plane i) in both halves
+      const uint32_t ah = lds_u16(sbuf + ((uint32_t)r * 2u * P + (uint32_t)pass * P + i) * 2u);
+      al[j] = ah | (ah << 16);
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t x1[4], x2[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x1[j] = nw[j][v] << sh1;
+        x2[j] = nw[j][v] << sh2;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {  // k-step s8 = 2v + e: bytes 2e (cols 0-7), 2e + 1 (8-15)
+        const int s8 = 2 * v + e;
+        const uint32_t sel0 = (uint32_t)(((8 + 2 * e) << 4) | ((12 + 2 * e) << 12));
+        const uint32_t sel1 = (uint32_t)(((9 + 2 * e) << 4) | ((13 + 2 * e) << 12));
+        uint32_t a[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          a[j][0] = xor_andnot(al[j], prmt(x1[j], x2[j], sel0), 0x80008000u);  // cols 2q, 2q+1
+          a[j][1] = xor_andnot(al[j], prmt(x1[j], x2[j], sel1), 0x80008000u);  // cols 2q+8, 2q+9
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          // tile f: rows 16 f + g (j = 2f) and 16 f + g + 8 (j = 2f + 1)
+          mma_16816(acc[h][0][nt], a[0][0], a[1][0], a[0][1], a[1][1], bf[s8][nt][0],
+                    bf[s8][nt][1]);
+          mma_16816(acc[h][1][nt], a[2][0], a[3][0], a[2][1], a[3][1], bf[s8][nt][0],
+                    bf[s8][nt][1]);
+        }
+      }
+    }
+  }
+}
+
+// One CTA per SM, the same units, groups, ring and teams as the lookup
+// kernel: warps 0..15 consume in two teams of 8 that take alternate groups
+// (team warp w: row-block rb0 + w of the stage), NP producer warps stream
+// the planes.  Each K-block's activation tile is loaded by all 16 warps
+// (slot kb & 1) between the same kind of barriers as the table build.
+//   NT  n-tiles of 8 activation rows (M <= 8 NT), P  planes (one precision)
+template <int NT, int P>
+__global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
+    gemv_mma_kernel(const __grid_constant__ GemvParams prm) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int D = prm.D, NP = prm.NP, RB = prm.RB;
+  constexpr uint32_t kStage = gemv_stage_bytes(P);
+  const uint32_t ring = sbase + mma_ring_off(P);
+  const uint32_t full0 = sbase + mma_off_bar(D, P);
+  const uint32_t empty0 = full0 + 8u * (uint32_t)D;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + mma_off_bar(D, P) + 16u * D);
+  constexpr int kConsumers = kConsumerWarps * 32;
+
+  const bool cfg_ok = D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 && (D & 1) == 0 &&
+                      prm.M >= 1 && prm.M <= 8 * NT &&
+                      (int)blockDim.x == 32 * (kConsumerWarps + NP);
+  CtaRange R;
+  make_range(prm, R);
+  uint4 xv;  // consumers: the first activation tile's row, first of all
+  if (warp < kConsumerWarps) {
+    grid_dependency_wait();
+    load_x_tile(prm, R.kb0, warp, lane, xv);
+  }
+  if (warp == 0) {
+    if (cfg_ok && lane < D) {
+      mbar_init(full0 + 8u * lane, 1);
+      mbar_init(empty0 + 8u * lane, kTeamWarps);
+    }
+    if (lane == 0) {
+      *abort_flag = cfg_ok ? 0 : 1;
+      if (!cfg_ok) record_error(&g_device_error, BCQ_ERR_UNSUPPORTED);
+    }
+    if (cfg_ok) fence_mbar_init();
+  }
+  __syncthreads();
+  launch_dependents();
+  if (*abort_flag) return;  // set before the barrier: uniform
+
+  if (warp >= kConsumerWarps) {
+    produce_stages<P>(prm, R, warp - kConsumerWarps, lane, ring, full0, empty0, abort_flag);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int team = warp / kTeamWarps;
+  const int tw = warp % kTeamWarps;
+  const int g = lane >> 2, q = lane & 3;
+  // rotation constants of this thread's rows (g and g + 8, mod 16)
+  const uint32_t ra0 = (uint32_t)(((g + 3) >> 2) & 3), ra1 = (uint32_t)(((g + 11) >> 2) & 3);
+  const uint32_t dsh = (uint32_t)((-g) & 3) * 8u;
+  const uint32_t sbuf0 = sbase + kMmaScaleOff + (uint32_t)warp * 2u * mma_scale_buf_bytes(P);
+  const size_t part_stride = (size_t)RB * kRowBlock;
+  int cur_kb = -1;
+  uint4 xn = make_uint4(0u, 0u, 0u, 0u);
+  int xn_kb = -1;
+
+  // tiles of every K-block up to kbt, in order, by all 16 warps
+  auto advance_tiles = [&](int kbt) {
+    while (cur_kb < kbt) {
+      const int kbn = cur_kb < 0 ? R.kb0 : cur_kb + 1;
+      if (cur_kb >= 0) {
+        if (xn_kb == kbn) xv = xn;
+        else load_x_tile(prm, kbn, warp, lane, xv);
+      }
+      if (kbn < R.kb_last) {
+        load_x_tile(prm, kbn + 1, warp, lane, xn);
+        xn_kb = kbn + 1;
+      }
+      // the slot rebuilt was last read two K-blocks ago, before the previous
+      // build's barrier
+      store_x_tile(sbase, kbn, warp, lane, xv);
+      named_barrier_sync(1, kConsumers);
+      cur_kb = kbn;
+    }
+  };
+
+  GroupCursor gc;  // this team's next group
+  cursor_init(gc, R.u0, R.u1, R.kb0, RB);
+  int gg = team;
+  if (team) cursor_next(gc, R.u1, RB);
+  int s = team;
+  uint32_t ph = 0;
+  // scales of the team's groups, staged one group ahead (cp.async, two
+  // buffers per warp)
+  GroupCursor pc = gc;
+  int buf = 0;
+  if (gg < R.NG && tw < pc.n) stage_scales<P>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0);
+  cp_async_commit();
+  cursor_next(pc, R.u1, RB);
+  cursor_next(pc, R.u1, RB);
+
+  while (gg < R.NG) {
+    advance_tiles(gc.kb);
+    const bool active = tw < gc.n;
+    const uint32_t sbuf = sbuf0 + (uint32_t)buf * mma_scale_buf_bytes(P);
+    // stage the next group's scales into the other buffer, then make sure
+    // this group's have landed
+    if (gg + 2 < R.NG && tw < pc.n)
+      stage_scales<P>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0 + (uint32_t)(buf ^ 1) * mma_scale_buf_bytes(P));
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const bool ok = wait_stage(full0 + 8u * s, ph, abort_flag, prm.timeout_ns);
+    if (!ok && lane == 0 && *abort_flag == 0) {
+      record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    float acc[2][2][NT][4];  // [group][tile]: independent accumulator chains
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int f = 0; f < 2; ++f)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[h][f][nt][e] = 0.f;
+    if (ok && active) {
+      const uint32_t xt = sbase + (uint32_t)(gc.kb & 1) * kXTileBytes;
+      const uint32_t st = ring + (uint32_t)s * kStage + (uint32_t)tw * kUnitPlaneBytes;
+#pragma unroll 1
+      for (int i = 0; i < P; ++i)
+        mma_plane<NT, P>(st + (uint32_t)i * kPlaneGroupBytes, xt, sbuf, i, g, q, ra0, ra1, dsh,
+                         acc);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cta(empty0 + 8u * s);
+    if (ok && active && *abort_flag == 0) {
+      // offsets: z[row][group] * S[m][group]; then the unit's partial sums
+      const uint32_t gsl = sbase + kMmaGsumOff + (uint32_t)(gc.kb & 1) * kMmaRows * 8u;
+#pragma unroll
+      for (int f = 0; f < 2; ++f) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int r = 16 * f + g + 8 * hr;
+          float zz[2] = {0.f, 0.f};
+          if (prm.z) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              zz[h] = h2f((uint16_t)lds_u16(sbuf + 128u * P + (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
+          }
+          const int row = (gc.rb0 + tw) * kRowBlock + r;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int m = nt * 8 + 2 * q + c;
+              float v = acc[0][f][nt][2 * hr + c] + acc[1][f][nt][2 * hr + c];
+              const float sA = lds_f32_dyn(gsl + (uint32_t)(m * 2) * 4u);
+              const float sB = lds_f32_dyn(gsl + (uint32_t)(m * 2 + 1) * 4u);
+              v = fmaf(zz[0], sA, fmaf(zz[1], sB, v));
+              if (m < prm.M) {
+                if (prm.KB > 1)
+                  prm.part[((size_t)gc.kb * prm.M + m) * part_stride + (size_t)row] = v;
+                else if (row < prm.N)
+                  prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(v);
+              }
+            }
+          }
+        }
+      }
+    }
+    buf ^= 1;
+    cursor_next(pc, R.u1, RB);
+    cursor_next(pc, R.u1, RB);
+    cursor_next(gc, R.u1, RB);
+    cursor_next(gc, R.u1, RB);
+    s += 2;
+    if (s >= D) {
+      s -= D;
+      ph ^= 1u;
+    }
+    gg += 2;
+  }
+  cp_async_wait<0>();
+  advance_tiles(R.kb_last);  // the same barriers in both teams
+
+  if (prm.KB > 1) {
+    named_barrier_sync(1, kConsumers);  // every partial of the CTA is stored
+    splitk_tail(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
+  }
+}
+
+}  // namespace bcq

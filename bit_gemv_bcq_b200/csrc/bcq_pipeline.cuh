@@ -1,0 +1,202 @@
+// bcq_pipeline.cuh -- pieces shared by the GEMV kernels of libbcq (included
+// by bcq_kernels.cu only): the CTA's share of the (K-block, row-block) units
+// and its groups, the stage wait, the producer warps' bulk-copy ring and the
+// split-K reduction through the caller's workspace.
+#pragma once
+
+#include <cstdint>
+
+#include "bcq_device.cuh"
+#include "bcq_layout.h"
+
+namespace bcq {
+
+// Device error word of this library (one per device): kernels record the
+// first problem they hit; bcq_device_error() reads and clears it.  (This
+// header belongs to the single translation unit bcq_kernels.cu.)
+__device__ int g_device_error = 0;
+
+// The units of one CTA: [u0, u1) in kb-major order (the host's split: see
+// plan_units), cut into groups: the row-blocks of one K-block inside one row
+// group (at most kRowGroup).
+struct CtaRange {
+  int u0, u1, NG, kb0, kb_last;
+};
+
+__device__ __forceinline__ void make_range(const GemvParams& p, CtaRange& R) {
+  const CtaWork w = p.work[blockIdx.x];
+  R.u0 = w.u0;
+  R.u1 = w.u1;
+  R.NG = w.ng;
+  R.kb0 = w.kb & 0xFFFF;
+  R.kb_last = w.kb >> 16;
+}
+
+// Walks the groups of a CTA in order: K-block kb, first row-block rb0, n
+// row-blocks (all in row group rb0 / kRowGroup); seg_end bounds the
+// row-blocks of kb inside the CTA's range.
+struct GroupCursor {
+  int kb, rb0, n, seg_end;
+};
+
+__device__ __forceinline__ void cursor_init(GroupCursor& c, int u0, int u1, int kb0, int RB) {
+  c.kb = kb0;
+  c.rb0 = u0 - c.kb * RB;
+  c.seg_end = min(RB, u1 - c.kb * RB);
+  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
+}
+
+__device__ __forceinline__ void cursor_next(GroupCursor& c, int u1, int RB) {
+  c.rb0 += c.n;
+  if (c.rb0 >= c.seg_end) {
+    ++c.kb;
+    c.rb0 = 0;
+    c.seg_end = min(RB, u1 - c.kb * RB);
+  }
+  c.n = min(kRowGroup - (c.rb0 & (kRowGroup - 1)), c.seg_end - c.rb0);
+}
+
+// Waits for phase `parity` of a stage barrier: a non-blocking test first
+// (the common case: the stage has landed), then bounded waiting that gives
+// up when the CTA aborts.
+__device__ __forceinline__ bool wait_stage(uint32_t bar, uint32_t parity,
+                                           volatile int* abort_flag,
+                                           unsigned long long limit_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+  while (true) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+template <int J>
+struct Slot {
+  static constexpr int value = J;
+};
+
+// Producer warp pw of NP: issues stages (groups) k = pw, pw + NP, ...; with D
+// a multiple of NP it alone refills its ring slots, so the empty-barrier
+// phase it waits for is never two phases behind.  Stage g holds the first P
+// planes of group g (plane i at i * 8 KiB, row-block rb0 + w at w KiB): a
+// whole row group is one bulk copy, a partial one (at the ends of the CTA's
+// range) one copy per plane.  Lane 0 issues; the warp returns when every
+// copy it issued has landed (or the CTA gave up).
+template <int P>
+__device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaRange& R, int pw,
+                                               int lane, uint32_t ring, uint32_t full0,
+                                               uint32_t empty0, volatile int* abort_flag) {
+  constexpr uint32_t kStage = gemv_stage_bytes(P);
+  const int D = prm.D, NP = prm.NP, RB = prm.RB;
+  if (!prm.early_weights) grid_dependency_wait();
+  if (lane == 0) {
+    int issued = 0;
+    GroupCursor gc;
+    cursor_init(gc, R.u0, R.u1, R.kb0, RB);
+    if (pw) cursor_next(gc, R.u1, RB);
+    int s = pw;        // ring slot of stage k (incremental: no division)
+    uint32_t eph = 1;  // parity of the empty phase that frees slot s (stage k - D)
+    for (int k = pw; k < R.NG; k += NP) {
+      if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, eph, prm.timeout_ns)) {
+        record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (*abort_flag) break;
+      const uint32_t bar = full0 + 8u * s;
+      const uint32_t dst = ring + (uint32_t)s * kStage;
+      const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
+      const uint32_t* src =
+          prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H * (kRowGroup * kWordsPerUnitPlane);
+      mbar_arrive_expect_tx(bar, (uint32_t)(P * gc.n) * kUnitPlaneBytes);
+      if (gc.n == kRowGroup) {
+        bulk_g2s(dst, src, kStage, bar);
+      } else {
+#pragma unroll
+        for (int i = 0; i < P; ++i)
+          bulk_g2s(dst + (uint32_t)i * kPlaneGroupBytes,
+                   src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
+                   (uint32_t)gc.n * kUnitPlaneBytes, bar);
+      }
+      issued = k + 1;
+      for (int t = 0; t < NP; ++t) cursor_next(gc, R.u1, RB);
+      s += NP;
+      if (s >= D) {
+        s -= D;
+        eph ^= 1u;
+      }
+    }
+    // every copy this warp issued lands before the CTA may exit
+    for (int s2 = pw; s2 < D && s2 < issued; s2 += NP) {
+      const int klast = issued - 1 - ((issued - 1 - s2) % D);
+      (void)mbar_wait_bounded(full0 + 8u * s2, (uint32_t)((klast / D) & 1), prm.timeout_ns);
+    }
+  }
+  __syncwarp();
+}
+
+// Split-K reduction, run by all nthreads consumer threads of the CTA after
+// a barrier that follows their partial-sum stores.  Every unit's fp32
+// partials [kb][m][row] are in the workspace.  Each CTA counts its arrivals
+// (fence, then release), then reduces the row-blocks it is designated for --
+// row-block rb belongs to the CTA that computed its unit in K-block rb mod KB,
+// so the work is spread evenly whatever the order in which CTAs finish.  The
+// reducer waits (bounded) until all KB partials of rb have arrived, adds them
+// in K-block order (the result does not depend on scheduling), writes y (row
+// m of the launch goes to y row ymap[m], or m without a map) and clears the
+// partials and the counter, so the whole workspace is zero again for the
+// next call, whatever its shape.
+__device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRange& R, int Mrows,
+                                            const int* ymap, int tid, int nthreads,
+                                            volatile int* abort_flag) {
+  const int RB = prm.RB;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
+  const size_t part_stride = (size_t)RB * kRowBlock;
+  const bool live = *abort_flag == 0;
+  for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
+    const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+    const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+    for (int rb = a + tid; rb < b; rb += nthreads) {
+      __threadfence();  // cumulative over the barrier: the CTA's stores
+      red_add_release(prm.cnt + rb, 1u);
+    }
+  }
+  for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
+    const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+    const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+    int first = kb;  // designated row-blocks: kb, kb + KB, ...
+    if (first < a) first += (a - first + prm.KB - 1) / prm.KB * prm.KB;
+    for (int rbx = first + warp * prm.KB; rbx < b; rbx += nwarps * prm.KB) {
+      bool ready = true;
+      if (lane == 0)
+        ready = wait_count(prm.cnt + rbx, (unsigned int)prm.KB, abort_flag, prm.timeout_ns);
+      ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
+      if (!ready) {
+        if (lane == 0 && *abort_flag == 0) {
+          record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        continue;
+      }
+      const int row = rbx * kRowBlock + lane;
+      for (int m = 0; m < Mrows; ++m) {
+        const float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
+        float sum = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < prm.KB; ++k) sum += ldg_cg_f32(pp + (size_t)k * Mrows * part_stride);
+        const int ym = ymap ? ymap[m] : m;
+        if (row < prm.N) prm.y[(size_t)ym * prm.N + row] = f2h_rn(sum);
+      }
+      // the workspace is left zero-filled for any later shape
+      for (int m = 0; m < Mrows; ++m) {
+        float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
+        for (int k = 0; k < prm.KB; ++k) stg_cg_zero(pp + (size_t)k * Mrows * part_stride);
+      }
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
+    }
+  }
+}
+
+}  // namespace bcq

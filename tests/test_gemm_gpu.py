@@ -56,10 +56,18 @@ def _run(prob, w=None, p=None, p_row=None):
 
 # --------------------------------------------------------------- small / ragged
 
+@pytest.fixture(params=["lut", "mma"])
+def path(request, monkeypatch):
+    """Run a test through one of the two kernels: the lookup-table kernel for
+    every batch size, or the tensor-core kernel for every batch size."""
+    monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1000" if request.param == "lut" else "1")
+    return request.param
+
+
 @pytest.mark.parametrize("N,K", [(1, 128), (31, 384), (33, 640), (100, 1024),
                                  (256, 512), (1000, 2048), (64, 128 * 33)])
-@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
-def test_parity_small_and_ragged(N, K, M):
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16, 17])
+def test_parity_small_and_ragged(N, K, M, path):
     prob = synth.make_problem(N, K, M, seed=N + K + M, precisions=(1, 2, 3, 4))
     w = _weights(prob)
     for p in (1, 2, 3, 4):
@@ -96,7 +104,7 @@ def test_parity_mlp_decode_with_outliers_full(N, K):
 
 
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096)])
-def test_parity_batch_sweep(N, K):
+def test_parity_batch_sweep(N, K, path):
     """M in {1, 2, 4, 8, 16}, p = 2, 3, 4, all outputs."""
     prob = synth.make_problem(N, K, 16, seed=3)
     w = _weights(prob)
@@ -108,7 +116,7 @@ def test_parity_batch_sweep(N, K):
 
 
 @pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
-def test_parity_mixed_precision_70b_sampled(N, K):
+def test_parity_mixed_precision_70b_sampled(N, K, path):
     """M = 8 rows with p drawn from {2,3,4}; outputs checked on 1024 sampled
     rows plus the first and last row-blocks."""
     prob = synth.make_problem(N, K, 8, seed=4, mixed=True)
@@ -123,7 +131,7 @@ def test_parity_mixed_precision_70b_sampled(N, K):
 
 # ------------------------------------------------------------------ invariants
 
-def test_p_prefix_poisoned_planes_are_never_read():
+def test_p_prefix_poisoned_planes_are_never_read(path):
     """Planes p..p_H-1 replaced by random bits: bitwise identical output."""
     prob = synth.make_problem(1000, 2048, 3, seed=5, precisions=(1, 2, 3, 4))
     w = _weights(prob)
@@ -137,14 +145,14 @@ def test_p_prefix_poisoned_planes_are_never_read():
         assert torch.equal(y1, y2), f"p={p}"
 
 
-def test_results_are_reproducible():
+def test_results_are_reproducible(path):
     prob = synth.make_problem(14336, 4096, 2, seed=6)
     w = _weights(prob)
     ys = [_run(prob, w, p=3) for _ in range(3)]
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
 
 
-def test_mixed_rows_match_uniform_calls():
+def test_mixed_rows_match_uniform_calls(path):
     prob = synth.make_problem(4096, 4096, 8, seed=7, mixed=True)
     prob.p_row[:] = [4, 2, 3, 3, 2, 4, 2, 3]
     w = _weights(prob)
@@ -239,7 +247,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 # ------------------------------------------------- launch shapes and workspace
 
 @pytest.mark.parametrize("C,D,NP", [(1, 2, 1), (3, 4, 2), (7, 6, 2), (13, 2, 2), (148, 8, 2)])
-def test_forced_launch_shapes(monkeypatch, C, D, NP):
+def test_forced_launch_shapes(monkeypatch, C, D, NP, path):
     """Few CTAs (each spanning several K-blocks, groups cut at K-block
     boundaries), shallow and deep rings, one or two producer warps."""
     monkeypatch.setenv("BCQ_FORCE_C", str(C))
@@ -255,7 +263,7 @@ def test_forced_launch_shapes(monkeypatch, C, D, NP):
                f"C={C} p={p}")
 
 
-def test_workspace_is_left_zero_filled():
+def test_workspace_is_left_zero_filled(path):
     prob = synth.make_problem(4096, 4096, 2, seed=21)
     w = _weights(prob)
     for p in (2, 3):
@@ -266,7 +274,7 @@ def test_workspace_is_left_zero_filled():
 
 
 @pytest.mark.parametrize("mode", [1, 2])
-def test_programmatic_dependent_launch_gives_the_same_bits(mode):
+def test_programmatic_dependent_launch_gives_the_same_bits(mode, path):
     """Back-to-back calls with PDL (and early plane streaming) equal the plain
     stream-ordered results bit for bit."""
     prob = synth.make_problem(14336, 4096, 2, seed=22)
@@ -285,7 +293,7 @@ def test_programmatic_dependent_launch_gives_the_same_bits(mode):
         assert torch.equal(a, b)
 
 
-def test_workspace_shared_across_shapes():
+def test_workspace_shared_across_shapes(path):
     """One workspace serves calls of different shapes in turn: a smaller N
     leaves no partial sums where a larger N keeps its arrival counters."""
     a = synth.make_problem(4096, 4096, 2, seed=23)
@@ -294,3 +302,17 @@ def test_workspace_shared_across_shapes():
     for _ in range(2):
         _check(_run(a, wa, p=3), oracle.gemm(a.x, a.planes, a.alphas, a.z, p=3), "4096")
         _check(_run(b, wb, p=2), oracle.gemm(b.x, b.planes, b.alphas, b.z, p=2), "14336")
+
+
+def test_both_paths_agree_with_each_other(monkeypatch):
+    """The lookup-table and tensor-core kernels compute the same sums (fp32,
+    different order): within the parity bound of each other on a full-size
+    batch of 16 rows of mixed precision."""
+    prob = synth.make_problem(14336, 4096, 16, seed=25, mixed=True)
+    w = _weights(prob)
+    monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1000")
+    y_lut = _run(prob, w, p_row=prob.p_row)
+    monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1")
+    y_mma = _run(prob, w, p_row=prob.p_row)
+    d = (y_lut.float() - y_mma.float()).abs()
+    assert (d <= ATOL + RTOL * y_lut.float().abs()).all()

@@ -47,11 +47,17 @@ def algo_bytes(N, K, M, p):
     return N * K * p // 8 + N * G * p * 2 + N * G * 2 + M * K * 2 + M * N * 2
 
 
+KERNEL_SOURCES = ("bcq_kernels.cu", "bcq_device.cuh", "bcq_pipeline.cuh", "bcq_mma.cuh",
+                  "bcq_layout.h")
+
+
 def csrc_sha256():
+    """Hash of the sources that define the GEMV kernels (recorded DRAM
+    traffic is only reported while they are unchanged)."""
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "bit_gemv_bcq_b200", "csrc")
-    for f in sorted(os.listdir(src)):
+    for f in KERNEL_SOURCES:
         h.update(f.encode())
         with open(os.path.join(src, f), "rb") as fh:
             h.update(fh.read())
@@ -285,9 +291,18 @@ def run_gpu(args, rank, world, local_rank):
     return result
 
 
+MMA_MIN_ROWS = 3   # bcq_gemm's default switch to the tensor-core kernel
+
+
 def launches_per_call(M):
-    """GEMV kernel launches of one bcq_gemm call: one per two activation rows."""
-    return -(-M // 2)
+    """GEMV kernel launches of one single-precision bcq_gemm call: the lookup
+    kernel takes two activation rows per launch, the tensor-core kernel up to
+    sixteen."""
+    return -(-M // 16) if M >= MMA_MIN_ROWS else -(-M // 2)
+
+
+def kernel_of(M):
+    return "gemv_mma_kernel" if M >= MMA_MIN_ROWS else "gemv_lut_kernel"
 
 
 # ------------------------------------------------------------- CPU oracle arm
@@ -397,7 +412,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
                      "peak_kind": peak_kind, "traffic": None,
-                     "kernel": "gemv_lut_kernel (every launch of the step)"},
+                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 2, "
+                               "gemv_mma_kernel for M >= 3)"},
         "per_call": res["per_case"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
@@ -408,6 +424,16 @@ def main():
         line["roofline"]["traffic_per"] = "launch (mean over one step's launches, ncu launch list)"
         line["roofline"]["algorithmic_bytes_per_launch"] = round(tr["algorithmic_bytes_per_launch"])
         line["roofline"]["traffic_source"] = tr["source"]
+    by_kernel = {}
+    for c in res["per_case"]:
+        k = by_kernel.setdefault(kernel_of(c["M"]), {"us": 0.0, "bytes": 0})
+        k["us"] += c["us"]
+        k["bytes"] += c["bytes"]
+    for name, k in by_kernel.items():
+        gbps = k["bytes"] / k["us"] / 1e3
+        by_kernel[name] = {"us_per_step": round(k["us"], 2), "GBps": round(gbps, 1),
+                           "frac": round(gbps / peak, 4)}
+    line["roofline"]["by_kernel"] = by_kernel
     m1 = [c for c in res["per_case"] if c["M"] == 1]
     line["headline_m1"] = {f"p{c['p']}": {"us": c["us"], "GBps": c["GBps"],
                                           "frac": round(c["GBps"] / peak, 4)} for c in m1}

@@ -31,6 +31,8 @@ BCQ_ERR_ALIGN = 4
 BCQ_ERR_CUDA = 5
 BCQ_ERR_TIMEOUT = 6
 BCQ_ERR_UNSUPPORTED = 7
+BCQ_ERR_SCRATCH = 8
+NOALLOC_SCRATCH_BYTES = 16 << 20   # BCQ_NOALLOC_SCRATCH_BYTES
 GROUP = 128
 MAX_M = 64
 
@@ -79,6 +81,8 @@ def lib():
         L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, S, P]
         L.bcq_gemm_host.restype = I
         L.bcq_gemm_host.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, P, P, S, P]
+        L.bcq_gemm_noalloc.restype = I
+        L.bcq_gemm_noalloc.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
         L.bcq_build_lut.restype = I
         L.bcq_build_lut.argtypes = [P, I, I, P, P, P]
         L.bcq_device_error.restype = I
@@ -91,8 +95,9 @@ def lib():
 
 EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
-            "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl", "bcq_gemm_host", "bcq_build_lut",
-            "bcq_device_error", "bcq_debug_wait_timeout")
+            "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl",
+            "bcq_gemm_host", "bcq_gemm_noalloc", "bcq_build_lut", "bcq_device_error",
+            "bcq_debug_wait_timeout")
 
 
 def status_string(status: int) -> str:
@@ -291,6 +296,32 @@ def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
                         _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
                         _stream(stream))
     _check(st, "bcq_gemm")
+    del pr_keep
+    return out
+
+
+def gemm_noalloc(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bcq_gemm_noalloc: as gemm, but the split-K scratch is the library's own
+    static array instead of a workspace, for callers that cannot allocate
+    device memory.  Calls that may overlap on the GPU share that array and
+    race; shapes needing more than NOALLOC_SCRATCH_BYTES raise
+    BcqError(BCQ_ERR_SCRATCH).  `out` should be given by such callers (the
+    binding allocates it otherwise)."""
+    _need_cuda(x, "x", torch.float16)
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M][{w.K}]")
+    M = x.shape[0]
+    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.float16, device=x.device)
+    else:
+        _need_cuda(out, "out", torch.float16)
+    alpha = _alpha_array(w.alphas)
+    st = lib().bcq_gemm_noalloc(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                                _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                                _ptr(out), _stream(stream))
+    _check(st, "bcq_gemm_noalloc")
     del pr_keep
     return out
 

@@ -307,6 +307,13 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
 }
 
 }  // namespace
+bcq_status check_gemm_args(const uint16_t* x, const uint32_t* planes,
+                           const uint16_t* const alpha[4], const uint16_t* z, int p,
+                           const int32_t* p_row, int M, int N, int K, int p_H, int group,
+                           const uint16_t* y, const void* ws, size_t ws_bytes) {
+  return validate_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, group, y, ws, ws_bytes);
+}
+
 }  // namespace bcq
 
 using namespace bcq;
@@ -323,6 +330,7 @@ const char* bcq_status_string(int status) {
     case BCQ_ERR_CUDA: return "BCQ_ERR_CUDA: CUDA runtime or launch failure";
     case BCQ_ERR_TIMEOUT: return "BCQ_ERR_TIMEOUT: a bounded wait in a kernel ran out";
     case BCQ_ERR_UNSUPPORTED: return "BCQ_ERR_UNSUPPORTED: request not handled by this build";
+    case BCQ_ERR_SCRATCH: return "BCQ_ERR_SCRATCH: the call needs more than the built-in scratch";
     default: return "BCQ_ERR_UNKNOWN";
   }
 }

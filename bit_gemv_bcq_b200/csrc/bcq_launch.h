@@ -5,6 +5,7 @@
 
 #include <cstdint>
 
+#include "bcq.h"
 #include "bcq_layout.h"
 
 namespace bcq {
@@ -40,5 +41,11 @@ cudaError_t launch_wait_probe(unsigned long long limit_ns, cudaStream_t st);
 
 // Synchronises st, returns the device error word in *code and clears it.
 cudaError_t read_and_clear_device_error(cudaStream_t st, int* code);
+
+// The argument checks of bcq_gemm (defined in bcq_api.cu).
+bcq_status check_gemm_args(const uint16_t* x, const uint32_t* planes,
+                           const uint16_t* const alpha[4], const uint16_t* z, int p,
+                           const int32_t* p_row, int M, int N, int K, int p_H, int group,
+                           const uint16_t* y, const void* ws, size_t ws_bytes);
 
 }  // namespace bcq

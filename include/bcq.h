@@ -56,12 +56,14 @@ typedef enum bcq_status {
   BCQ_ERR_ALIGN = 4,        /* a device pointer breaks its alignment rule      */
   BCQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed            */
   BCQ_ERR_TIMEOUT = 6,      /* a bounded wait inside a kernel ran out          */
-  BCQ_ERR_UNSUPPORTED = 7   /* valid request this build does not handle (e.g. group != 128) */
+  BCQ_ERR_UNSUPPORTED = 7,  /* valid request this build does not handle (e.g. group != 128) */
+  BCQ_ERR_SCRATCH = 8       /* bcq_gemm_noalloc: the call needs more scratch than it has */
 } bcq_status;
 
 #define BCQ_GROUP 128       /* columns per scale group                          */
 #define BCQ_MAX_PLANES 4    /* p_H <= 4                                         */
 #define BCQ_MAX_M 64        /* rows of x per call                               */
+#define BCQ_NOALLOC_SCRATCH_BYTES (16u << 20)  /* bcq_gemm_noalloc's built-in scratch */
 
 /* Human-readable name of a status code.  Never NULL. */
 const char* bcq_status_string(int status);
@@ -208,6 +210,38 @@ bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
                          int p_H, int group, uint16_t* y_host,
                          uint16_t* x_dev, uint16_t* y_dev, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * bcq_gemm without a caller workspace, for callers that cannot allocate
+ * device memory: code that runs where cudaMalloc is not allowed (inside a
+ * memory pool or allocator that must not recurse into itself, a plug-in whose
+ * host framework owns every allocation, or a real-time loop that must not
+ * block on the driver's allocator) still needs the split-K scratch that
+ * bcq_gemm takes as `workspace`.  This entry point uses a scratch array that
+ * is part of the library itself instead.  The paper has no counterpart: it
+ * is a packaging choice of this library, not part of the method.
+ *
+ * Arguments, results and errors are those of bcq_gemm, without workspace and
+ * workspace_bytes.  In addition:
+ *   - The scratch is one static device array of BCQ_NOALLOC_SCRATCH_BYTES
+ *     (16 MiB), held on every GPU that loads the library until the process
+ *     exits.  A call whose bcq_workspace_bytes(M, N, K) exceeds it returns
+ *     BCQ_ERR_SCRATCH and launches nothing; use bcq_gemm for such shapes.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on that device.
+ *   - Each call clears the part of the scratch it uses (cudaMemsetAsync on
+ *     `stream`) before its kernels.  Nothing is allocated, by this call or
+ *     by any routine it calls.
+ *   - Every call on a device shares the one array.  Calls that may overlap on
+ *     the GPU (different streams, or other threads' streams) race on it and
+ *     their results are undefined; serialise them, or use bcq_gemm with a
+ *     workspace per stream.
+ */
+bcq_status bcq_gemm_noalloc(const uint16_t* x, const uint32_t* planes,
+                            const uint16_t* const alpha[4], const uint16_t* z,
+                            int p, const int32_t* p_row, int M, int N, int K,
+                            int p_H, int group, uint16_t* y, void* stream);
 
 /*
  * The lookup table and group sums exactly as the GEMV kernel builds them in

@@ -24,6 +24,15 @@ constexpr int kDefaultProducers = 2;
 // Calls with at least this many rows take the tensor-core path.
 constexpr int kDefaultMmaMinRows = 3;
 
+// Kernels: the lookup-table kernel (one or two rows), and for batches a
+// tensor-core kernel: mma.sync (default) or tcgen05 (BCQ_MMA_KIND=tcgen05).
+enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2 };
+
+int batch_path() {
+  const char* v = std::getenv("BCQ_MMA_KIND");
+  return (v && std::strcmp(v, "tcgen05") == 0) ? kPathUmma : kPathMmaSync;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int env_int(const char* name, int dflt) {
@@ -89,7 +98,7 @@ bcq_status get_device(DeviceCache** dc) {
 
 struct Plan {
   GemvKernel fn = nullptr;
-  int C = 0, D = 0, NP = 0;
+  int C = 0, D = 0, NP = 0, MW = 0;
   size_t dyn = 0;
   long long units_max = 0;
   int KB = 0;
@@ -101,14 +110,20 @@ struct Plan {
 // of one K-block) fed by NP producer warps, as deep as shared memory allows
 // beside the 64 KiB table; D is even (a stage's team consumed the stage D
 // earlier) and a multiple of NP (a producer refills only its own slots).
-bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, bool mma, Plan* out) {
+bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out) {
   DeviceCache* dc = nullptr;
   bcq_status st = get_device(&dc);
   if (st != BCQ_OK) return st;
   Plan pl;
-  pl.fn = mma ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P) : gemv_kernel_for(M, P, mixed);
+  pl.fn = path == kPathUmma      ? gemv_umma_kernel_for(P)
+          : path == kPathMmaSync ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P)
+                                 : gemv_kernel_for(M, P, mixed);
   if (!pl.fn) return BCQ_ERR_UNSUPPORTED;
-  auto dyn_of = [&](int d) { return mma ? mma_dyn_bytes(d, P) : gemv_dyn_bytes(d, P); };
+  auto dyn_of = [&](int d) {
+    return path == kPathUmma      ? umma_dyn_bytes(d, P)
+           : path == kPathMmaSync ? mma_dyn_bytes(d, P)
+                                  : gemv_dyn_bytes(d, P);
+  };
   const long long RB = (long long)row_blocks(N);
   const long long KB = (long long)k_blocks(K);
   const long long U = RB * KB;
@@ -119,7 +134,8 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, bool mma, Plan* out
   D = std::min(kMaxStages, D) / step * step;
   if (D < step) D = step;
   while (D > step && dyn_of(D) > kMaxDynSmem) D -= step;
-  const int nthreads = 32 * (kConsumerWarps + pl.NP);
+  pl.MW = path == kPathUmma ? kUmmaGroups : 0;
+  const int nthreads = 32 * (kConsumerWarps + pl.MW + pl.NP);
   while (true) {
     pl.dyn = dyn_of(D);
     int per_sm = 0;
@@ -243,6 +259,7 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const ui
   plan_units(RB, KB, pl.C, g.work);
   g.D = pl.D;
   g.NP = pl.NP;
+  g.MW = pl.MW;
   g.early_weights = pdl_mode == 2 ? 1 : 0;
   g.timeout_ns = wait_us > 0 ? (unsigned long long)wait_us * 1000ull : kDefaultWaitNs;
 }
@@ -258,6 +275,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
   const int wait_us = env_int("BCQ_WAIT_LIMIT_US", 0);
   const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
   if (M >= mma_min) {
+    const int path = batch_path();
     for (int q = 1; q <= 4; ++q) {
       int rows[BCQ_MAX_M];
       int n = 0;
@@ -266,7 +284,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
       for (int r0 = 0; r0 < n; r0 += kMmaRows) {
         const int cnt = std::min(kMmaRows, n - r0);
         Plan pl;
-        bcq_status s = plan_gemv(cnt, N, K, q, false, true, &pl);
+        bcq_status s = plan_gemv(cnt, N, K, q, false, path, &pl);
         if (s != BCQ_OK) return s;
         GemvParams g{};
         fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
@@ -289,7 +307,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
     const int P = std::max(q[0], q[1]);
     const bool mixed = q[0] != q[1];
     Plan pl;
-    bcq_status s = plan_gemv(rows, N, K, P, mixed, false, &pl);
+    bcq_status s = plan_gemv(rows, N, K, P, mixed, kPathLut, &pl);
     if (s != BCQ_OK) return s;
     GemvParams g{};
     fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
@@ -380,13 +398,13 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
   if (M < 1 || M > kMmaRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
   if (p_load < 1 || p_load > 4) return BCQ_ERR_PRECISION;
   if (mixed && (M != 2 || p_load < 2)) return BCQ_ERR_PRECISION;
-  const bool mma = M > kMaxMPerLaunch;
+  const int path = M > kMaxMPerLaunch ? batch_path() : kPathLut;
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;
   if (t_virtual) (void)cudaGetLastError();
   Plan pl;
-  bcq_status st = plan_gemv(M, N, K, p_load, mixed != 0, mma, &pl);
+  bcq_status st = plan_gemv(M, N, K, p_load, mixed != 0, path, &pl);
   t_virtual = false;
   if (st != BCQ_OK) return st;
   out[0] = pl.C;

@@ -614,6 +614,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 }  // namespace bcq
 
 #include "bcq_mma.cuh"
+#include "bcq_umma.cuh"
 
 namespace bcq {
 
@@ -749,11 +750,21 @@ GemvKernel gemv_mma_kernel_for(int NT, int P) {
   return nullptr;
 }
 
+GemvKernel gemv_umma_kernel_for(int P) {
+  switch (P) {
+    case 1: return gemv_umma_kernel<1>;
+    case 2: return gemv_umma_kernel<2>;
+    case 3: return gemv_umma_kernel<3>;
+    case 4: return gemv_umma_kernel<4>;
+    default: return nullptr;
+  }
+}
+
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,
                         cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.C, 1, 1);
-  cfg.blockDim = dim3((unsigned)(32 * (kConsumerWarps + p.NP)), 1, 1);
+  cfg.blockDim = dim3((unsigned)(32 * (kConsumerWarps + p.MW + p.NP)), 1, 1);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

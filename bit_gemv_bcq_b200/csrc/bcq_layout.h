@@ -114,6 +114,43 @@ __host__ __device__ constexpr uint32_t mma_dyn_bytes(int D, int P) {
   return mma_off_bar(D, P) + 16u * (uint32_t)D + 16u;
 }
 
+// The tcgen05 GEMV (bcq_umma.cuh).  Shared memory: the activation tiles of
+// two K-blocks in the canonical K-major layout of the MMA's B operand (16
+// rows x 256 columns, 8 KiB each), their group sums, per-warp scale buffers
+// (as above), the ring, then the barriers.  Tensor memory (512 columns,
+// lane = weight row): four MMA groups (team x half of a team's row group) of
+// 128 columns each: two fp32 accumulators of 16 columns (alternate units;
+// column = activation row) and three A-operand buffers of 32 columns (64
+// K-columns of +-alpha).
+constexpr int kUmmaN = 16;                      // activation rows per launch (MMA N)
+constexpr uint32_t kUmmaXTileBytes = 8192;
+constexpr uint32_t kUmmaGsumOff = 2 * kUmmaXTileBytes;                   // 16384
+constexpr uint32_t kUmmaScaleOff = kUmmaGsumOff + 2 * kUmmaN * 2 * 4;    // 16640
+constexpr int kUmmaGroups = 4;                  // = MMA-issuing warps
+constexpr int kUmmaGroupWarps = 4;              // expanding warps of an MMA group
+constexpr int kUmmaAccBufs = 2;
+constexpr int kUmmaABufs = 3;
+constexpr uint32_t kUmmaGroupCols = 128;
+constexpr uint32_t kUmmaACol = 32;              // first A column of a group
+constexpr uint32_t kUmmaABufCols = 32;
+constexpr uint32_t kUmmaTmemCols = 512;
+__host__ __device__ constexpr uint32_t umma_ring_off(int P) {
+  return (kUmmaScaleOff + 16u * 2u * mma_scale_buf_bytes(P) + 1023u) & ~1023u;
+}
+__host__ __device__ constexpr uint32_t umma_off_bar(int D, int P) {
+  return umma_ring_off(P) + (uint32_t)D * gemv_stage_bytes(P);
+}
+// full[D], empty[D], then per MMA group: A full[3], A empty[3], accumulator
+// full[2], accumulator empty[2]; then the tensor-memory address and the
+// abort flag.
+constexpr int kUmmaBarsPerGroup = 2 * kUmmaABufs + 2 * kUmmaAccBufs;
+__host__ __device__ constexpr uint32_t umma_off_misc(int D, int P) {
+  return umma_off_bar(D, P) + 16u * (uint32_t)D + 8u * (kUmmaGroups * kUmmaBarsPerGroup);
+}
+__host__ __device__ constexpr uint32_t umma_dyn_bytes(int D, int P) {
+  return umma_off_misc(D, P) + 16u;
+}
+
 struct GemvParams {
   const uint16_t* x;         // fp16 [M][K] (rows of this launch)
   const uint32_t* planes;    // packed planes
@@ -127,6 +164,7 @@ struct GemvParams {
   int U;                     // units (< 2^31)
   int C;                     // CTAs
   int D, NP;                 // ring stages, producer warps
+  int MW;                    // MMA-issuing warps (tcgen05 kernel), else 0
   int early_weights;         // with PDL: stream weights before the grid wait
   unsigned long long timeout_ns;
   int rows[kMmaRows];        // tensor-core launches: x / y row of launch row m

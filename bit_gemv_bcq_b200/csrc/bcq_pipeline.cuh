@@ -142,17 +142,20 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
 // (fence, then release), then reduces the row-blocks it is designated for --
 // row-block rb belongs to the CTA that computed its unit in K-block rb mod KB,
 // so the work is spread evenly whatever the order in which CTAs finish.  The
-// reducer waits (bounded) until all KB partials of rb have arrived, adds them
-// in K-block order (the result does not depend on scheduling), writes y (row
-// m of the launch goes to y row ymap[m], or m without a map) and clears the
-// partials and the counter, so the whole workspace is zero again for the
-// next call, whatever its shape.
+// (row-block, launch row) pairs of the CTA are dealt to its warps in turn; a
+// warp waits (bounded) until all KB partials of its row-block have arrived,
+// loads them all at once, adds them in K-block order (the result does not
+// depend on scheduling), writes y (row m of the launch goes to y row ymap[m],
+// or m without a map) and clears those partials.  After a barrier the CTA
+// clears its row-blocks' counters, so the whole workspace is zero again for
+// the next call, whatever its shape.
 __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRange& R, int Mrows,
                                             const int* ymap, int tid, int nthreads,
                                             volatile int* abort_flag) {
-  const int RB = prm.RB;
+  const int RB = prm.RB, KB = prm.KB;
   const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
   const size_t part_stride = (size_t)RB * kRowBlock;
+  const size_t kstride = (size_t)Mrows * part_stride;  // one K-block of partials
   const bool live = *abort_flag == 0;
   for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
     const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
@@ -162,40 +165,55 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
       red_add_release(prm.cnt + rb, 1u);
     }
   }
+  int task = 0, mine = warp;  // tasks dealt round-robin: no division
   for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
     const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
     const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
     int first = kb;  // designated row-blocks: kb, kb + KB, ...
-    if (first < a) first += (a - first + prm.KB - 1) / prm.KB * prm.KB;
-    for (int rbx = first + warp * prm.KB; rbx < b; rbx += nwarps * prm.KB) {
-      bool ready = true;
-      if (lane == 0)
-        ready = wait_count(prm.cnt + rbx, (unsigned int)prm.KB, abort_flag, prm.timeout_ns);
-      ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
-      if (!ready) {
-        if (lane == 0 && *abort_flag == 0) {
-          record_error(&g_device_error, BCQ_ERR_TIMEOUT);
-          *abort_flag = 1;
+    if (first < a) first += (a - first + KB - 1) / KB * KB;
+    for (int rbx = first; rbx < b; rbx += KB) {
+      for (int m = 0; m < Mrows; ++m, ++task) {
+        if (task != mine) continue;
+        mine += nwarps;
+        bool ready = true;
+        if (lane == 0)
+          ready = wait_count(prm.cnt + rbx, (unsigned int)KB, abort_flag, prm.timeout_ns);
+        ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
+        if (!ready) {
+          if (lane == 0 && *abort_flag == 0) {
+            record_error(&g_device_error, BCQ_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          continue;
         }
-        continue;
-      }
-      const int row = rbx * kRowBlock + lane;
-      for (int m = 0; m < Mrows; ++m) {
-        const float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
+        const int row = rbx * kRowBlock + lane;
+        float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
         float sum = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < prm.KB; ++k) sum += ldg_cg_f32(pp + (size_t)k * Mrows * part_stride);
+        for (int k0 = 0; k0 < KB; k0 += 16) {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            v[j] = k0 + j < KB ? ldg_cg_f32(pp + (size_t)(k0 + j) * kstride) : 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (k0 + j < KB) sum += v[j];
+        }
         const int ym = ymap ? ymap[m] : m;
         if (row < prm.N) prm.y[(size_t)ym * prm.N + row] = f2h_rn(sum);
+        // the workspace is left zero-filled for any later shape
+        for (int k = 0; k < KB; ++k) stg_cg_zero(pp + (size_t)k * kstride);
       }
-      // the workspace is left zero-filled for any later shape
-      for (int m = 0; m < Mrows; ++m) {
-        float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
-        for (int k = 0; k < prm.KB; ++k) stg_cg_zero(pp + (size_t)k * Mrows * part_stride);
-      }
-      __syncwarp();
-      if (lane == 0) *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
     }
+  }
+  // every task's wait is over: clear the designated counters
+  named_barrier_sync(1, nthreads);
+  for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
+    const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+    const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+    int first = kb;
+    if (first < a) first += (a - first + KB - 1) / KB * KB;
+    for (int rbx = first + tid * KB; rbx < b; rbx += nthreads * KB)
+      *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
   }
 }
 

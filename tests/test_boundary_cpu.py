@@ -92,7 +92,7 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     assert pl["units_max"] == -(-U // pl["C"])
     assert pl["dyn_bytes"] <= 232448
     assert pl["stage_bytes"] == 8192 * p    # the p planes of one row group
-    table = 65536 if M <= 2 else 16 * 264 * 2 * 2   # lookup table, or activation tiles
+    table = 65536 if M <= 2 else 2 * 16 * 256 * 2   # lookup table, or two activation tiles
     assert pl["dyn_bytes"] >= table + pl["D"] * pl["stage_bytes"]
     assert pl["D"] % 2 == 0 and pl["D"] % pl["NP"] == 0 and 2 <= pl["D"] <= 20
     # as deep as the shared memory allows

@@ -56,11 +56,13 @@ def _run(prob, w=None, p=None, p_row=None):
 
 # --------------------------------------------------------------- small / ragged
 
-@pytest.fixture(params=["lut", "mma"])
+@pytest.fixture(params=["lut", "sync", "tcgen05"])
 def path(request, monkeypatch):
-    """Run a test through one of the two kernels: the lookup-table kernel for
-    every batch size, or the tensor-core kernel for every batch size."""
+    """Run a test through one of the kernels for every batch size: the
+    lookup-table kernel, the mma.sync tensor-core kernel or the tcgen05 one."""
     monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1000" if request.param == "lut" else "1")
+    if request.param != "lut":
+        monkeypatch.setenv("BCQ_MMA_KIND", request.param)
     return request.param
 
 
@@ -313,6 +315,8 @@ def test_both_paths_agree_with_each_other(monkeypatch):
     monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1000")
     y_lut = _run(prob, w, p_row=prob.p_row)
     monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "1")
-    y_mma = _run(prob, w, p_row=prob.p_row)
-    d = (y_lut.float() - y_mma.float()).abs()
-    assert (d <= ATOL + RTOL * y_lut.float().abs()).all()
+    for kind in ("sync", "tcgen05"):
+        monkeypatch.setenv("BCQ_MMA_KIND", kind)
+        y_mma = _run(prob, w, p_row=prob.p_row)
+        d = (y_lut.float() - y_mma.float()).abs()
+        assert (d <= ATOL + RTOL * y_lut.float().abs()).all(), kind

@@ -349,6 +349,15 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     if (ok && active && *abort_flag == 0) {
       // offsets: z[row][group] * S[m][group]; then the unit's partial sums
       const uint32_t gsl = sbase + kMmaGsumOff + (uint32_t)(gc.kb & 1) * kMmaRows * 8u;
+      float sg[NT][2][2];  // S[m][group] of this thread's activation rows m
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int m = nt * 8 + 2 * q + c;
+          sg[nt][c][0] = lds_f32_dyn(gsl + (uint32_t)(m * 2) * 4u);
+          sg[nt][c][1] = lds_f32_dyn(gsl + (uint32_t)(m * 2 + 1) * 4u);
+        }
 #pragma unroll
       for (int f = 0; f < 2; ++f) {
 #pragma unroll
@@ -367,9 +376,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
             for (int c = 0; c < 2; ++c) {
               const int m = nt * 8 + 2 * q + c;
               float v = acc[0][f][nt][2 * hr + c] + acc[1][f][nt][2 * hr + c];
-              const float sA = lds_f32_dyn(gsl + (uint32_t)(m * 2) * 4u);
-              const float sB = lds_f32_dyn(gsl + (uint32_t)(m * 2 + 1) * 4u);
-              v = fmaf(zz[0], sA, fmaf(zz[1], sB, v));
+              v = fmaf(zz[0], sg[nt][c][0], fmaf(zz[1], sg[nt][c][1], v));
               if (m < prm.M) {
                 if (prm.KB > 1)
                   prm.part[((size_t)gc.kb * prm.M + m) * part_stride + (size_t)row] = v;

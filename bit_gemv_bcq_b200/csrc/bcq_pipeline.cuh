@@ -142,9 +142,9 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
 // (fence, then release), then reduces the row-blocks it is designated for --
 // row-block rb belongs to the CTA that computed its unit in K-block rb mod KB,
 // so the work is spread evenly whatever the order in which CTAs finish.  The
-// (row-block, launch row) pairs of the CTA are dealt to its warps in turn; a
-// warp waits (bounded) until all KB partials of its row-block have arrived,
-// loads them all at once, adds them in K-block order (the result does not
+// (row-block, two launch rows) tasks of the CTA are dealt to its warps in
+// turn; a warp waits (bounded) until all KB partials of its row-block have
+// arrived, loads them all at once, adds them in K-block order (the result does not
 // depend on scheduling), writes y (row m of the launch goes to y row ymap[m],
 // or m without a map) and clears those partials.  After a barrier the CTA
 // clears its row-blocks' counters, so the whole workspace is zero again for
@@ -157,12 +157,15 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
   const size_t part_stride = (size_t)RB * kRowBlock;
   const size_t kstride = (size_t)Mrows * part_stride;  // one K-block of partials
   const bool live = *abort_flag == 0;
-  for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
-    const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
-    const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
-    for (int rb = a + tid; rb < b; rb += nthreads) {
-      __threadfence();  // cumulative over the barrier: the CTA's stores
-      red_add_release(prm.cnt + rb, 1u);
+  if (warp == 0 && live) {
+    // one warp: a release fence in each lane, cumulative over the barrier
+    // before this call (every partial of the CTA), then that lane's arrivals
+    // as relaxed atomics
+    fence_acq_rel_gpu();
+    for (int kb = R.kb0; kb <= R.kb_last; ++kb) {
+      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
+      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
+      for (int rb = a + lane; rb < b; rb += 32) red_add_relaxed(prm.cnt + rb, 1u);
     }
   }
   int task = 0, mine = warp;  // tasks dealt round-robin: no division
@@ -172,7 +175,7 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
     int first = kb;  // designated row-blocks: kb, kb + KB, ...
     if (first < a) first += (a - first + KB - 1) / KB * KB;
     for (int rbx = first; rbx < b; rbx += KB) {
-      for (int m = 0; m < Mrows; ++m, ++task) {
+      for (int m0 = 0; m0 < Mrows; m0 += 2, ++task) {  // two launch rows per task
         if (task != mine) continue;
         mine += nwarps;
         bool ready = true;
@@ -187,21 +190,31 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
           continue;
         }
         const int row = rbx * kRowBlock + lane;
-        float* pp = prm.part + (size_t)m * part_stride + (size_t)row;
-        float sum = 0.f;
+        const int nm = Mrows - m0 < 2 ? Mrows - m0 : 2;
+        float* pp = prm.part + (size_t)m0 * part_stride + (size_t)row;
+        float sum[2] = {0.f, 0.f};
         for (int k0 = 0; k0 < KB; k0 += 16) {
-          float v[16];
+          float v[2][16];  // every load of the task in flight at once
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] = k0 + j < KB ? ldg_cg_f32(pp + (size_t)(k0 + j) * kstride) : 0.f;
+          for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (k0 + j < KB) sum += v[j];
+            for (int j = 0; j < 16; ++j)
+              v[mm][j] = mm < nm && k0 + j < KB
+                             ? ldg_cg_f32(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride)
+                             : 0.f;
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (k0 + j < KB) sum[mm] += v[mm][j];
         }
-        const int ym = ymap ? ymap[m] : m;
-        if (row < prm.N) prm.y[(size_t)ym * prm.N + row] = f2h_rn(sum);
-        // the workspace is left zero-filled for any later shape
-        for (int k = 0; k < KB; ++k) stg_cg_zero(pp + (size_t)k * kstride);
+        for (int mm = 0; mm < nm; ++mm) {
+          const int ym = ymap ? ymap[m0 + mm] : m0 + mm;
+          if (row < prm.N) prm.y[(size_t)ym * prm.N + row] = f2h_rn(sum[mm]);
+          // the workspace is left zero-filled for any later shape
+          for (int k = 0; k < KB; ++k)
+            stg_cg_zero(pp + (size_t)mm * part_stride + (size_t)k * kstride);
+        }
       }
     }
   }

@@ -255,9 +255,57 @@ def run_gpu(args, rank, world, local_rank):
         per_case.append({"p": p, "M": M, "us": round(us, 3), "bytes": by,
                          "GBps": round(by / us / 1e3, 1)})
 
+    # an MLP's gate and up projections (same x) stacked into one weight: one
+    # call for both (M = 1, 2), against two calls on the separate weights
+    stacked = None
+    if not args.cases:
+        prob_b = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed + 1)
+        sbase = api.BcqWeights.stack([(prob.planes, prob.alphas, prob.z),
+                                      (prob_b.planes, prob_b.alphas, prob_b.z)], device=dev)
+        s_copy = sbase.packed.numel() * 4 + sum(a.numel() * 2 for a in sbase.alphas.values()) \
+            + sbase.z.numel() * 2
+        RS = max(2, math.ceil(2 * L2_BYTES / s_copy) + 1)
+        scopies = [sbase] + [api.BcqWeights(packed=sbase.packed.clone(),
+                                            alphas={q: a.clone() for q, a in sbase.alphas.items()},
+                                            z=sbase.z.clone(), N=sbase.N, K=sbase.K, p_H=sbase.p_H,
+                                            row_splits=sbase.row_splits)
+                             for _ in range(RS - 1)]
+        ys2 = {M: torch.empty((M, sbase.N), dtype=torch.float16, device=dev) for M in (1, 2)}
+        with torch.cuda.stream(stream):
+            for M in (1, 2):
+                for p in PRECISIONS:
+                    sbase.gemm(x[:M], p=p, out=ys2[M], stream=stream)
+        stream.synchronize()
+        stacked = {"weights": f"2 x {N_OUT} rows (gate and up) x {K_IN}, stacked along N",
+                   "l2": f"{RS} rotating copies of {s_copy / 2**20:.1f} MiB"}
+        single = {(c["p"], c["M"]): c["us"] for c in per_case}
+        for M in (1, 2):
+            for p in PRECISIONS:
+                def sone(p=p, M=M):
+                    for w in scopies:
+                        w.gemm(x[:M], p=p, out=ys2[M], stream=stream)
+                g = capture(sone)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    b.record(stream)
+                b.synchronize()
+                us = a.elapsed_time(b) * 1000.0 / (reps * RS)
+                by = algo_bytes(2 * N_OUT, K_IN, M, p)
+                two = 2 * single[(p, M)] if (p, M) in single else None
+                stacked[f"M{M}p{p}"] = {"us": round(us, 3), "GBps": round(by / us / 1e3, 1),
+                                        "us_two_calls": None if two is None else round(two, 3)}
+                del g
+        del scopies, sbase
+        assert api.device_error(stream) == api.BCQ_OK
+
     result = {"ms_total": ms_total, "bytes_step": bytes_step, "R": R,
               "per_copy_bytes": per_copy, "launches_per_step": launches_per_step,
-              "per_case": per_case, "clocks": clocks}
+              "per_case": per_case, "clocks": clocks, "stacked": stacked}
 
     # end to end through bcq_gemm_host: pinned host x and y, copies inside
     if not args.profile:
@@ -434,6 +482,8 @@ def main():
         by_kernel[name] = {"us_per_step": round(k["us"], 2), "GBps": round(gbps, 1),
                            "frac": round(gbps / peak, 4)}
     line["roofline"]["by_kernel"] = by_kernel
+    if res.get("stacked"):
+        line["stacked_gate_up"] = res["stacked"]
     m1 = [c for c in res["per_case"] if c["M"] == 1]
     line["headline_m1"] = {f"p{c['p']}": {"us": c["us"], "GBps": c["GBps"],
                                           "frac": round(c["GBps"] / peak, 4)} for c in m1}

@@ -241,6 +241,7 @@ class BcqWeights:
     N: int
     K: int
     p_H: int
+    row_splits: tuple = ()      # rows of each stacked matrix (see stack), else ()
 
     @classmethod
     def from_canonical(cls, planes, alphas: dict, z=None, device="cuda", stream=None):
@@ -261,6 +262,52 @@ class BcqWeights:
             zz = (torch.as_tensor(z) if isinstance(z, np.ndarray) else z)
             zz = pack_scales(zz.to(device=device, dtype=torch.float16).contiguous(), 1, stream)
         return cls(packed=packed, alphas=al, z=zz, N=N, K=KW * 32, p_H=p_H)
+
+    @classmethod
+    def stack(cls, parts, device="cuda", stream=None):
+        """Matrices that multiply the same x -- an MLP's gate and up
+        projections -- as one weight: their canonical planes, scales and
+        offsets stacked along N and packed together.  One call then reads x,
+        builds each K-block's lookup table and reduces the split-K partial sums
+        once for all of them: the table of cached +-x partial sums depends on x
+        only (AnyBCQ Paper-Notes page, 关键设计 / 直接bit-plane运算的CUDA内核),
+        and its build is the cost the FluxBin page's "Lookup Table Building
+        Approach with Scale Fusion" sets out to keep small.
+        parts: sequence of (planes uint32 [p_H][N_i][K/32], {q: alpha fp16
+        [N_i][G][q]}, z fp16 [N_i][G] or None); every part has the same p_H,
+        K and precisions, and all or none have z.  gemm() returns y
+        [M][sum N_i]; split_rows() gives the per-matrix views."""
+        parts = list(parts)
+        if not parts:
+            raise ValueError("nothing to stack")
+
+        def cat(arrays, axis):
+            if all(isinstance(a, np.ndarray) for a in arrays):
+                return np.concatenate(arrays, axis=axis)
+            return torch.cat([torch.as_tensor(a) for a in arrays], dim=axis)
+
+        planes = cat([pl for pl, _, _ in parts], 1)
+        qs = set(parts[0][1])
+        if any(set(al) != qs for _, al, _ in parts):
+            raise ValueError("every stacked matrix needs the same precisions")
+        alphas = {q: cat([al[q] for _, al, _ in parts], 0) for q in sorted(qs)}
+        zs = [z for _, _, z in parts]
+        if any((z is None) != (zs[0] is None) for z in zs):
+            raise ValueError("give z for every stacked matrix or for none")
+        z = None if zs[0] is None else cat(zs, 0)
+        w = cls.from_canonical(planes, alphas, z, device=device, stream=stream)
+        w.row_splits = tuple(int(pl.shape[1]) for pl, _, _ in parts)
+        return w
+
+    def split_rows(self, y):
+        """Per-matrix views [M][N_i] of the output of a stacked weight."""
+        if not self.row_splits:
+            return [y]
+        out, r0 = [], 0
+        for n in self.row_splits:
+            out.append(y[:, r0:r0 + n])
+            r0 += n
+        return out
 
     def gemm(self, x, p=None, p_row=None, out=None, stream=None):
         return gemm(x, self, p=p, p_row=p_row, out=out, stream=stream)

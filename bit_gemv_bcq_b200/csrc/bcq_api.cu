@@ -50,12 +50,12 @@ size_t k_blocks(int K) { return ((size_t)K + kKBlock - 1) / kKBlock; }
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace: arrival counters [RB] (256-byte aligned), then fp32 partial
-// sums [KB][min(M, 16)][RB * 32] (the rows of the largest launch).
+// sums [KB][min(M, 64)][RB * 32] (the rows of the largest launch).
 size_t counter_bytes(int N) { return align256(row_blocks(N) * sizeof(unsigned int)); }
 size_t workspace_bytes(int M, int N, int K) {
   const size_t KB = k_blocks(K);
   if (M < 1 || KB <= 1) return 0;
-  const size_t ml = (size_t)std::min(M, kMmaRows);
+  const size_t ml = (size_t)std::min(M, kMaxLaunchRows);
   return counter_bytes(N) + KB * ml * row_blocks(N) * kRowBlock * sizeof(float);
 }
 
@@ -115,12 +115,14 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   bcq_status st = get_device(&dc);
   if (st != BCQ_OK) return st;
   Plan pl;
-  pl.fn = path == kPathUmma      ? gemv_umma_kernel_for(P)
+  const int NN = M > kMmaRows ? kMaxLaunchRows : kMmaRows;  // tcgen05: 16 or 64 rows
+  pl.fn = path == kPathUmma      ? gemv_umma_kernel_for(P, NN)
           : path == kPathMmaSync ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P)
                                  : gemv_kernel_for(M, P, mixed);
   if (!pl.fn) return BCQ_ERR_UNSUPPORTED;
   auto dyn_of = [&](int d) {
-    return path == kPathUmma      ? umma_dyn_bytes(d, P)
+    return path == kPathUmma      ? (NN == kMmaRows ? umma_dyn_bytes<16>(d, P)
+                                                     : umma_dyn_bytes<64>(d, P))
            : path == kPathMmaSync ? mma_dyn_bytes(d, P)
                                   : gemv_dyn_bytes(d, P);
   };
@@ -266,8 +268,12 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const ui
 
 // Small batches: lookup-table launches of at most two rows, in order; two
 // rows with different precisions share one launch (planes streamed up to
-// the larger one).  Larger batches: tensor-core launches of up to 16 rows of
-// one precision each (rows grouped by precision, in order).
+// the larger one).  Larger batches, per precision (rows grouped by
+// precision, in order): tcgen05 launches of up to 64 rows while at least 32
+// rows are left (measured: 64 rows in one launch cost 0.6 of four 16-row
+// launches), then tensor-core launches of 16 rows, then one for a
+// remainder of at least BCQ_MMA_MIN_ROWS rows, else a lookup launch per
+// remaining row.
 bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
                     const uint16_t* z, int p, const int32_t* p_row, int M, int N, int K,
                     int p_H, uint16_t* y, void* ws, cudaStream_t st) {
@@ -281,20 +287,37 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
       int n = 0;
       for (int m = 0; m < M; ++m)
         if ((p > 0 ? p : p_row[m]) == q) rows[n++] = m;
-      for (int r0 = 0; r0 < n; r0 += kMmaRows) {
-        const int cnt = std::min(kMmaRows, n - r0);
+      for (int r0 = 0; r0 < n;) {
+        const int left = n - r0;
+        int cnt, qpath;
+        if (left >= 2 * kMmaRows) {
+          cnt = std::min(kMaxLaunchRows, left);
+          qpath = kPathUmma;
+        } else if (left >= mma_min) {
+          cnt = std::min(kMmaRows, left);
+          qpath = path;
+        } else {
+          cnt = 1;
+          qpath = kPathLut;
+        }
         Plan pl;
-        bcq_status s = plan_gemv(cnt, N, K, q, false, path, &pl);
+        bcq_status s = plan_gemv(cnt, N, K, q, false, qpath, &pl);
         if (s != BCQ_OK) return s;
         GemvParams g{};
         fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
-        g.x = x;
-        g.y = y;
         g.alpha[0] = g.alpha[1] = alpha[q - 1];
         g.M = cnt;
         g.q[0] = g.q[1] = q;
-        for (int j = 0; j < cnt; ++j) g.rows[j] = rows[r0 + j];
+        if (qpath == kPathLut) {  // one row, addressed directly
+          g.x = x + (size_t)rows[r0] * K;
+          g.y = y + (size_t)rows[r0] * N;
+        } else {
+          g.x = x;
+          g.y = y;
+          for (int j = 0; j < cnt; ++j) g.rows[j] = rows[r0 + j];
+        }
         if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st) != cudaSuccess) return BCQ_ERR_CUDA;
+        r0 += cnt;
       }
     }
     return BCQ_OK;
@@ -395,10 +418,10 @@ size_t bcq_workspace_bytes(int M, int N, int K) {
 
 int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, int* out) {
   if (!out) return BCQ_ERR_NULL;
-  if (M < 1 || M > kMmaRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
+  if (M < 1 || M > kMaxLaunchRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
   if (p_load < 1 || p_load > 4) return BCQ_ERR_PRECISION;
   if (mixed && (M != 2 || p_load < 2)) return BCQ_ERR_PRECISION;
-  const int path = M > kMaxMPerLaunch ? batch_path() : kPathLut;
+  const int path = M > kMmaRows ? kPathUmma : M > kMaxMPerLaunch ? batch_path() : kPathLut;
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;

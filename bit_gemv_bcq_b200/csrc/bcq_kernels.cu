@@ -750,14 +750,26 @@ GemvKernel gemv_mma_kernel_for(int NT, int P) {
   return nullptr;
 }
 
-GemvKernel gemv_umma_kernel_for(int P) {
-  switch (P) {
-    case 1: return gemv_umma_kernel<1>;
-    case 2: return gemv_umma_kernel<2>;
-    case 3: return gemv_umma_kernel<3>;
-    case 4: return gemv_umma_kernel<4>;
-    default: return nullptr;
+GemvKernel gemv_umma_kernel_for(int P, int NN) {
+  if (NN == 16) {
+    switch (P) {
+      case 1: return gemv_umma_kernel<1, 16>;
+      case 2: return gemv_umma_kernel<2, 16>;
+      case 3: return gemv_umma_kernel<3, 16>;
+      case 4: return gemv_umma_kernel<4, 16>;
+      default: return nullptr;
+    }
   }
+  if (NN == 64) {
+    switch (P) {
+      case 1: return gemv_umma_kernel<1, 64>;
+      case 2: return gemv_umma_kernel<2, 64>;
+      case 3: return gemv_umma_kernel<3, 64>;
+      case 4: return gemv_umma_kernel<4, 64>;
+      default: return nullptr;
+    }
+  }
+  return nullptr;
 }
 
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,

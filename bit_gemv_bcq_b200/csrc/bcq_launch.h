@@ -26,9 +26,9 @@ GemvKernel gemv_kernel_for(int M, int P, bool mixed);
 // streaming P planes (one precision); nullptr if there is none.
 GemvKernel gemv_mma_kernel_for(int NT, int P);
 
-// The tcgen05 GEMV kernel for up to 16 activation rows streaming P planes
-// (one precision); nullptr if there is none.
-GemvKernel gemv_umma_kernel_for(int P);
+// The tcgen05 GEMV kernel for up to NN (16 or 64) activation rows streaming
+// P planes (one precision); nullptr if there is none.
+GemvKernel gemv_umma_kernel_for(int P, int NN);
 
 // p.C CTAs of 32 * (16 + p.MW + p.NP) threads.
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,

@@ -114,41 +114,54 @@ __host__ __device__ constexpr uint32_t mma_dyn_bytes(int D, int P) {
   return mma_off_bar(D, P) + 16u * (uint32_t)D + 16u;
 }
 
-// The tcgen05 GEMV (bcq_umma.cuh).  Shared memory: the activation tiles of
-// two K-blocks in the canonical K-major layout of the MMA's B operand (16
-// rows x 256 columns, 8 KiB each), their group sums, per-warp scale buffers
-// (as above), the ring, then the barriers.  Tensor memory (512 columns,
-// lane = weight row): four MMA groups (team x half of a team's row group) of
-// 128 columns each: two fp32 accumulators of 16 columns (alternate units;
-// column = activation row) and three A-operand buffers of 32 columns (64
-// K-columns of +-alpha).
-constexpr int kUmmaN = 16;                      // activation rows per launch (MMA N)
-constexpr uint32_t kUmmaXTileBytes = 8192;
-constexpr uint32_t kUmmaGsumOff = 2 * kUmmaXTileBytes;                   // 16384
-constexpr uint32_t kUmmaScaleOff = kUmmaGsumOff + 2 * kUmmaN * 2 * 4;    // 16640
+// The tcgen05 GEMV (bcq_umma.cuh), for NN = 16 or 64 activation rows per
+// launch (the MMA's N).  Shared memory: the activation tiles of two K-blocks
+// in the canonical K-major layout of the MMA's B operand (NN rows x 256
+// columns), their group sums, per-warp scale buffers (as above), the ring,
+// then the barriers.  Tensor memory (512 columns, lane = weight row): four
+// MMA groups (team x half of a team's row group) of 128 columns each: fp32
+// accumulators of NN columns (column = activation row; two, alternating by
+// unit, for NN = 16, one for NN = 64) and 32-column A-operand buffers (64
+// K-columns of +-alpha; three for NN = 16, two for NN = 64).
 constexpr int kUmmaGroups = 4;                  // = MMA-issuing warps
 constexpr int kUmmaGroupWarps = 4;              // expanding warps of an MMA group
-constexpr int kUmmaAccBufs = 2;
-constexpr int kUmmaABufs = 3;
 constexpr uint32_t kUmmaGroupCols = 128;
-constexpr uint32_t kUmmaACol = 32;              // first A column of a group
 constexpr uint32_t kUmmaABufCols = 32;
 constexpr uint32_t kUmmaTmemCols = 512;
+constexpr int kMaxLaunchRows = 64;              // activation rows of one launch (any kernel)
+
+template <int NN>
+struct UmmaShape {
+  static_assert(NN == 16 || NN == 64, "16 or 64 activation rows");
+  static constexpr int kN = NN;
+  static constexpr uint32_t kXTileBytes = (uint32_t)NN * 512u;  // NN rows x 256 fp16
+  static constexpr uint32_t kGsumOff = 2u * kXTileBytes;
+  static constexpr uint32_t kScaleOff = kGsumOff + 2u * NN * 2u * 4u;
+  static constexpr int kAccBufs = NN == 16 ? 2 : 1;
+  static constexpr int kABufs = NN == 16 ? 3 : 2;
+  static constexpr uint32_t kACol = (uint32_t)kAccBufs * NN;  // first A column of a group
+  static constexpr int kBarsPerGroup = 2 * kABufs + 2 * kAccBufs;
+  static_assert(kACol + kABufs * kUmmaABufCols <= kUmmaGroupCols, "tensor memory budget");
+};
+template <int NN>
 __host__ __device__ constexpr uint32_t umma_ring_off(int P) {
-  return (kUmmaScaleOff + 16u * 2u * mma_scale_buf_bytes(P) + 1023u) & ~1023u;
+  return (UmmaShape<NN>::kScaleOff + 16u * 2u * mma_scale_buf_bytes(P) + 1023u) & ~1023u;
 }
+template <int NN>
 __host__ __device__ constexpr uint32_t umma_off_bar(int D, int P) {
-  return umma_ring_off(P) + (uint32_t)D * gemv_stage_bytes(P);
+  return umma_ring_off<NN>(P) + (uint32_t)D * gemv_stage_bytes(P);
 }
-// full[D], empty[D], then per MMA group: A full[3], A empty[3], accumulator
-// full[2], accumulator empty[2]; then the tensor-memory address and the
-// abort flag.
-constexpr int kUmmaBarsPerGroup = 2 * kUmmaABufs + 2 * kUmmaAccBufs;
+// full[D], empty[D], then per MMA group: A full[kABufs], A empty[kABufs],
+// accumulator full[kAccBufs], accumulator empty[kAccBufs]; then the
+// tensor-memory address and the abort flag.
+template <int NN>
 __host__ __device__ constexpr uint32_t umma_off_misc(int D, int P) {
-  return umma_off_bar(D, P) + 16u * (uint32_t)D + 8u * (kUmmaGroups * kUmmaBarsPerGroup);
+  return umma_off_bar<NN>(D, P) + 16u * (uint32_t)D +
+         8u * (kUmmaGroups * UmmaShape<NN>::kBarsPerGroup);
 }
+template <int NN>
 __host__ __device__ constexpr uint32_t umma_dyn_bytes(int D, int P) {
-  return umma_off_misc(D, P) + 16u;
+  return umma_off_misc<NN>(D, P) + 16u;
 }
 
 struct GemvParams {
@@ -167,7 +180,7 @@ struct GemvParams {
   int MW;                    // MMA-issuing warps (tcgen05 kernel), else 0
   int early_weights;         // with PDL: stream weights before the grid wait
   unsigned long long timeout_ns;
-  int rows[kMmaRows];        // tensor-core launches: x / y row of launch row m
+  int rows[kMaxLaunchRows];  // tensor-core launches: x / y row of launch row m
   CtaWork work[kMaxCtas];    // per CTA (C entries)
 };
 

@@ -117,32 +117,37 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Instruction descriptor of kind::f16: fp16 A and B, fp32 D, both K-major,
-// M = 128, N = kUmmaN (bits 4-5 D format, 7-9 / 10-12 A / B format, 15 / 16
+// M = 128, N = NN (bits 4-5 D format, 7-9 / 10-12 A / B format, 15 / 16
 // A / B major, 17-22 N / 8, 24-28 M / 16).
-constexpr uint32_t kUmmaIdesc =
-    (1u << 4) | ((uint32_t)(kUmmaN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+template <int NN>
+__host__ __device__ constexpr uint32_t umma_idesc() {
+  return (1u << 4) | ((uint32_t)(NN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
 
-// Shared-memory descriptor of a 16-row B operand slice in the canonical
+// Shared-memory descriptor of an NN-row B operand slice in the canonical
 // K-major layout without swizzle: 8-row x 16-byte core matrices, K-adjacent
-// ones 256 bytes apart (leading byte offset), row-adjacent ones 128 bytes
+// ones NN * 16 bytes apart (leading byte offset), row-adjacent ones 128 bytes
 // apart (stride byte offset); bits 46-47 = 1 (descriptor version).
+template <int NN>
 __device__ __forceinline__ uint64_t umma_bdesc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(256u >> 4) << 16) |
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((NN * 16u) >> 4) << 16) |
          ((uint64_t)(128u >> 4) << 32) | (1ull << 46);
 }
 
 // ------------------------------------------------------- activation tile
 
-// Row `warp` (launch row) of K-block kb's activation tile into slot kb & 1:
-// lane l holds columns 8l .. 8l + 7 (v, from load_x_tile), stored at their
-// permuted K positions (see above) of the canonical layout: row n, position
-// j at (j / 8) * 256 + (n / 8) * 128 + (n % 8) * 16 + (j % 8) * 2.  Also
-// the row's group sums, and the fence that shows the tile to the MMAs.
-__device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int warp, int lane,
+// Launch row n of K-block kb's activation tile into slot kb & 1: lane l
+// holds columns 8l .. 8l + 7 (v, from load_x_tile), stored at their permuted
+// K positions (see above) of the canonical layout: row n, position j at
+// (j / 8) * NN * 16 + (n / 8) * 128 + (n % 8) * 16 + (j % 8) * 2.  Also the
+// row's group sums, and the fence that shows the tile to the MMAs.
+template <int NN>
+__device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int n, int lane,
                                                   const uint4& v) {
+  using S = UmmaShape<NN>;
   const uint32_t slot = (uint32_t)(kb & 1);
-  const uint32_t tile = sbase + slot * kUmmaXTileBytes +
-                        (uint32_t)((warp >> 3) * 128 + (warp & 7) * 16);
+  const uint32_t tile = sbase + slot * S::kXTileBytes +
+                        (uint32_t)((n >> 3) * 128 + (n & 7) * 16);
   const int h = lane >> 4, U = (lane >> 2) & 3, t0 = 8 * (lane & 3);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -152,7 +157,7 @@ __device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int wa
     const int s = (e ? 31 : 15) - t;         // the shift that brings bit t to a sign
     const int j = 2 * (64 * h + 16 * U + s) + e;
     const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(tile + (uint32_t)((j >> 3) * 256 + (j & 7) * 2)),
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(tile + (uint32_t)((j >> 3) * (NN * 16) + (j & 7) * 2)),
                  "h"((unsigned short)half)
                  : "memory");
   }
@@ -162,7 +167,7 @@ __device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int wa
 #pragma unroll
   for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
   if ((lane & 15) == 0)  // lane 0: group A, lane 16: group B
-    sts_f32(sbase + kUmmaGsumOff + ((slot * kUmmaN + warp) * 2 + (lane >> 4)) * 4u, sum);
+    sts_f32(sbase + S::kGsumOff + ((slot * NN + n) * 2 + (lane >> 4)) * 4u, sum);
   fence_proxy_async_smem();
 }
 
@@ -180,11 +185,13 @@ __device__ __forceinline__ void expand_word(uint32_t wd, uint32_t alpha2, uint32
 
 // Barriers of MMA group G (each an 8-byte mbarrier), after the ring's.
 struct UmmaBars {
-  uint32_t afull, aempty, accfull, accempty;  // first of kUmmaABufs / kUmmaAccBufs each
+  uint32_t afull, aempty, accfull, accempty;  // first of kABufs / kAccBufs each
 };
+template <int NN>
 __device__ __forceinline__ UmmaBars umma_bars(uint32_t bar0, int G) {
-  const uint32_t b = bar0 + 8u * (uint32_t)(G * kUmmaBarsPerGroup);
-  return {b, b + 8u * kUmmaABufs, b + 16u * kUmmaABufs, b + 16u * kUmmaABufs + 8u * kUmmaAccBufs};
+  using S = UmmaShape<NN>;
+  const uint32_t b = bar0 + 8u * (uint32_t)(G * S::kBarsPerGroup);
+  return {b, b + 8u * S::kABufs, b + 16u * S::kABufs, b + 16u * S::kABufs + 8u * S::kAccBufs};
 }
 
 // Warp-specialised, one CTA per SM, with the units, groups, ring, producer
@@ -204,7 +211,7 @@ __device__ __forceinline__ UmmaBars umma_bars(uint32_t bar0, int G) {
 //                 accumulator's full barrier.
 //   warps 20..    produce: bulk copies of the planes into the ring.
 //   P  planes streamed (one precision for every row of the launch)
-template <int P>
+template <int P, int NN>
 __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     gemv_umma_kernel(const __grid_constant__ GemvParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -216,24 +223,27 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
   constexpr uint32_t kStage = gemv_stage_bytes(P);
   constexpr int kMmaWarp0 = kConsumerWarps;
   constexpr int kProducerWarp0 = kConsumerWarps + kUmmaGroups;
-  const uint32_t ring = sbase + umma_ring_off(P);
-  const uint32_t full0 = sbase + umma_off_bar(D, P);
+  using S = UmmaShape<NN>;
+  constexpr int XR = NN / 16;  // activation tile rows per expanding warp
+  const uint32_t ring = sbase + umma_ring_off<NN>(P);
+  const uint32_t full0 = sbase + umma_off_bar<NN>(D, P);
   const uint32_t empty0 = full0 + 8u * (uint32_t)D;
   const uint32_t gbar0 = empty0 + 8u * (uint32_t)D;
-  const uint32_t misc = umma_off_misc(D, P);
+  const uint32_t misc = umma_off_misc<NN>(D, P);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + misc + 4u);
   constexpr int kConsumers = kConsumerWarps * 32;
 
   const bool cfg_ok = D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 && (D & 1) == 0 &&
-                      prm.M >= 1 && prm.M <= kUmmaN && prm.MW == kUmmaGroups &&
+                      prm.M >= 1 && prm.M <= NN && prm.MW == kUmmaGroups &&
                       (int)blockDim.x == 32 * (kConsumerWarps + kUmmaGroups + NP);
   CtaRange R;
   make_range(prm, R);
-  uint4 xv;  // expanding warps: the first activation tile's row, first of all
+  uint4 xv[XR];  // expanding warps: the first activation tile's rows, first of all
   if (warp < kConsumerWarps) {
     grid_dependency_wait();
-    load_x_tile(prm, R.kb0, warp, lane, xv);
+#pragma unroll
+    for (int r = 0; r < XR; ++r) load_x_tile(prm, R.kb0, warp + 16 * r, lane, xv[r]);
   }
   if (warp == 0) {
     if (cfg_ok && lane < D) {
@@ -241,9 +251,9 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
       mbar_init(empty0 + 8u * lane, kTeamWarps);
     }
     if (cfg_ok) {
-      for (int b = lane; b < kUmmaGroups * kUmmaBarsPerGroup; b += 32) {
-        const int k = b % kUmmaBarsPerGroup;  // A full, A empty, acc full, acc empty
-        const bool by_warps = k < kUmmaABufs || k >= 2 * kUmmaABufs + kUmmaAccBufs;
+      for (int b = lane; b < kUmmaGroups * S::kBarsPerGroup; b += 32) {
+        const int k = b % S::kBarsPerGroup;  // A full, A empty, acc full, acc empty
+        const bool by_warps = k < S::kABufs || k >= 2 * S::kABufs + S::kAccBufs;
         mbar_init(gbar0 + 8u * b, by_warps ? kUmmaGroupWarps : 1);
       }
     }
@@ -279,7 +289,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     const int G = warp - kMmaWarp0;
     const int team = G >> 1, hf = G & 1;
     const uint32_t tg = tmem + (uint32_t)G * kUmmaGroupCols;
-    const UmmaBars bars = umma_bars(gbar0, G);
+    const UmmaBars bars = umma_bars<NN>(gbar0, G);
     GroupCursor gc;
     cursor_init(gc, R.u0, R.u1, R.kb0, RB);
     if (team) cursor_next(gc, R.u1, RB);
@@ -287,8 +297,8 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     uint32_t a_round = 0, acc_round = 0;
     for (int gg = team; gg < R.NG; gg += 2) {
       if (hf * 4 < gc.n) {  // the same test as the group's expanding warps
-        const uint32_t xt = sbase + (uint32_t)(gc.kb & 1) * kUmmaXTileBytes;
-        const uint32_t tacc = tg + (uint32_t)accb * 16u;
+        const uint32_t xt = sbase + (uint32_t)(gc.kb & 1) * S::kXTileBytes;
+        const uint32_t tacc = tg + (uint32_t)accb * (uint32_t)NN;
         // the accumulator's previous unit has been read
         if (acc_round > 0 &&
             !mbar_wait_bounded(bars.accempty + 8u * accb, (acc_round - 1u) & 1u, prm.timeout_ns))
@@ -302,23 +312,24 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
             umma_fence_after();
             if (lane == 0) {
               if (*abort_flag == 0) {
-                const uint32_t acol = tg + kUmmaACol + (uint32_t)ab * kUmmaABufCols;
+                const uint32_t acol = tg + S::kACol + (uint32_t)ab * kUmmaABufCols;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                   umma_f16_ts(tacc, acol + 8u * (uint32_t)j,
-                              umma_bdesc(xt + (uint32_t)(4 * c + j) * 512u), kUmmaIdesc,
+                              umma_bdesc<NN>(xt + (uint32_t)(4 * c + j) * (NN * 32u)),
+                              umma_idesc<NN>(),
                               (i | c | j) != 0 ? 1u : 0u);
               }
               umma_commit(bars.aempty + 8u * ab);
             }
-            if (++ab == kUmmaABufs) {
+            if (++ab == S::kABufs) {
               ab = 0;
               ++a_round;
             }
           }
         }
         if (lane == 0) umma_commit(bars.accfull + 8u * accb);
-        if (++accb == kUmmaAccBufs) {
+        if (++accb == S::kAccBufs) {
           accb = 0;
           ++acc_round;
         }
@@ -338,17 +349,15 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
   const int G = team * 2 + hf;          // MMA group
   const uint32_t tg = tmem + (uint32_t)G * kUmmaGroupCols;
   const uint32_t tl = tg + ((uint32_t)(qd * 32) << 16);  // this warp's lanes
-  const UmmaBars bars = umma_bars(gbar0, G);
+  const UmmaBars bars = umma_bars<NN>(gbar0, G);
   // rotation of this lane's row (bcq_layout.h): natural word v of a pass is
   // the funnel shift of rotated words (v - ra) mod 4 and (v - ra + 1) mod 4
   const int rho = lane & 15;
   const uint32_t ra = (uint32_t)(((rho + 3) >> 2) & 3);
   const uint32_t dsh = (uint32_t)((-rho) & 3) * 8u;
-  const uint32_t sbuf0 = sbase + kUmmaScaleOff + (uint32_t)warp * 2u * mma_scale_buf_bytes(P);
+  const uint32_t sbuf0 = sbase + S::kScaleOff + (uint32_t)warp * 2u * mma_scale_buf_bytes(P);
   const size_t part_stride = (size_t)RB * kRowBlock;
   int cur_kb = -1;
-  uint4 xn = make_uint4(0u, 0u, 0u, 0u);
-  int xn_kb = -1;
 
   // The unit whose accumulator is still to be read (deferred epilogue).
   bool pending = false, p_store = false;
@@ -359,11 +368,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     if (!mbar_wait_bounded(bars.accfull + 8u * p_accb, p_use & 1u, prm.timeout_ns)) give_up();
     __syncwarp();
     umma_fence_after();
-    const uint32_t gsl = sbase + kUmmaGsumOff + (uint32_t)(p_kb & 1) * kUmmaN * 8u;
+    const uint32_t gsl = sbase + S::kGsumOff + (uint32_t)(p_kb & 1) * NN * 8u;
 #pragma unroll 1
-    for (int m0 = 0; m0 < kUmmaN; m0 += 8) {
+    for (int m0 = 0; m0 < NN; m0 += 8) {
       uint32_t d[8];
-      tmem_ld8(tl + (uint32_t)p_accb * 16u + (uint32_t)m0, d);
+      tmem_ld8(tl + (uint32_t)p_accb * (uint32_t)NN + (uint32_t)m0, d);
       tmem_wait_ld();
       if (p_store && *abort_flag == 0) {
 #pragma unroll
@@ -396,15 +405,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     if (pending) epilogue();
     while (cur_kb < kbt) {
       const int kbn = cur_kb < 0 ? R.kb0 : cur_kb + 1;
-      if (cur_kb >= 0) {
-        if (xn_kb == kbn) xv = xn;
-        else load_x_tile(prm, kbn, warp, lane, xv);
+#pragma unroll
+      for (int r = 0; r < XR; ++r) {  // rows warp, warp + 16, ... of the tile
+        if (cur_kb >= 0) load_x_tile(prm, kbn, warp + 16 * r, lane, xv[r]);
+        umma_store_x_tile<NN>(sbase, kbn, warp + 16 * r, lane, xv[r]);
       }
-      if (kbn < R.kb_last) {
-        load_x_tile(prm, kbn + 1, warp, lane, xn);
-        xn_kb = kbn + 1;
-      }
-      umma_store_x_tile(sbase, kbn, warp, lane, xv);
       named_barrier_sync(1, kConsumers);
       cur_kb = kbn;
     }
@@ -469,7 +474,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
               give_up();
             __syncwarp();
             umma_fence_after();
-            const uint32_t acol = kUmmaACol + (uint32_t)ab * kUmmaABufCols;
+            const uint32_t acol = S::kACol + (uint32_t)ab * kUmmaABufCols;
             if (work) {
 #pragma unroll
               for (int t = 0; t < 2; ++t) {
@@ -482,7 +487,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
             umma_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cta(bars.afull + 8u * ab);
-            if (++ab == kUmmaABufs) {
+            if (++ab == S::kABufs) {
               ab = 0;
               ++a_round;
             }
@@ -507,7 +512,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
         p_z0 = h2f((uint16_t)lds_u16(sbuf + 128u * P + (uint32_t)(lane * 2 + (lane >> 4)) * 2u));
         p_z1 = h2f((uint16_t)lds_u16(sbuf + 128u * P + (uint32_t)(lane * 2 + ((lane >> 4) ^ 1)) * 2u));
       }
-      if (++accb == kUmmaAccBufs) {
+      if (++accb == S::kAccBufs) {
         accb = 0;
         ++acc_round;
       }

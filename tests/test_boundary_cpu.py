@@ -59,10 +59,11 @@ def test_workspace_bytes_formula(L):
     # one K-block: no split over K, no workspace
     assert api.workspace_bytes(1, 4096, 256) == 0
     assert api.workspace_bytes(4, 4096, 128) == 0
-    # counters (row-blocks x 4 B, rounded to 256 B) + KB x min(M, 16) x rows x 4 B
+    # counters (row-blocks x 4 B, rounded to 256 B) + KB x min(M, 64) x rows x 4 B
     assert api.workspace_bytes(1, 14336, 4096) == 1792 + 16 * 1 * 14336 * 4
     assert api.workspace_bytes(8, 14336, 4096) == 1792 + 16 * 8 * 14336 * 4
-    assert api.workspace_bytes(64, 14336, 4096) == 1792 + 16 * 16 * 14336 * 4
+    assert api.workspace_bytes(64, 14336, 4096) == 1792 + 16 * 64 * 14336 * 4
+    assert api.workspace_bytes(17, 14336, 4096) == 1792 + 16 * 17 * 14336 * 4
     assert api.workspace_bytes(2, 33, 640) == 256 + 3 * 2 * 64 * 4
     assert api.workspace_bytes(0, 64, 512) == 0
     assert api.workspace_bytes(1, 64, 100) == 0
@@ -72,7 +73,8 @@ def test_workspace_bytes_formula(L):
                                            (1, 14336, 4096, 2, False), (1, 14336, 4096, 4, False),
                                            (1, 4096, 14336, 3, False), (2, 4096, 4096, 2, False),
                                            (2, 28672, 8192, 4, True), (1, 256, 512, 4, False),
-                                           (1, 1, 128, 1, False), (2, 33, 640, 2, False)])
+                                           (1, 1, 128, 1, False), (2, 33, 640, 2, False),
+                                           (64, 14336, 4096, 4, False), (33, 4096, 4096, 2, False)])
 def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     """Plans for a nominal 148-SM B200 (no GPU needed): one CTA per SM at
     most (never more CTAs than units), whole K-blocks per CTA when the CTAs
@@ -92,7 +94,8 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     assert pl["units_max"] == -(-U // pl["C"])
     assert pl["dyn_bytes"] <= 232448
     assert pl["stage_bytes"] == 8192 * p    # the p planes of one row group
-    table = 65536 if M <= 2 else 2 * 16 * 256 * 2   # lookup table, or two activation tiles
+    tiles = 2 * (16 if M <= 16 else 64) * 256 * 2        # two activation tiles
+    table = 65536 if M <= 2 else tiles                    # or the lookup table
     assert pl["dyn_bytes"] >= table + pl["D"] * pl["stage_bytes"]
     assert pl["D"] % 2 == 0 and pl["D"] % pl["NP"] == 0 and 2 <= pl["D"] <= 20
     # as deep as the shared memory allows
@@ -102,7 +105,7 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
 
 def test_plan_query_rejects_bad_arguments(L):
     with pytest.raises(api.BcqError):
-        api.plan_query(17, 64, 256, 2)            # at most 16 rows per launch
+        api.plan_query(65, 64, 256, 2)            # at most 64 rows per launch
     with pytest.raises(api.BcqError):
         api.plan_query(4, 64, 256, 3, mixed=True)  # tensor-core launches: one precision
     with pytest.raises(api.BcqError):

@@ -117,6 +117,23 @@ def test_parity_batch_sweep(N, K, path):
             _check(y, oracle.gemm(sub.x, prob.planes, prob.alphas, prob.z, p=p), f"M={M} p={p}")
 
 
+@pytest.mark.parametrize("N,K", [(4096, 4096), (1000, 2048), (14336, 4096)])
+def test_parity_wide_batches(N, K, path):
+    """17 to 64 rows of one precision: one tcgen05 launch of up to 64 rows (the
+    lookup kernel in pairs), and mixed precisions that split into groups of
+    more and of fewer than 16 rows."""
+    prob = synth.make_problem(N, K, 64, seed=4)
+    w = _weights(prob)
+    for M in (17, 33, 64):
+        sub = synth.Problem(x=prob.x[:M], planes=prob.planes, alphas=prob.alphas, z=prob.z)
+        for p in (2, 4):
+            y = _run(sub, w, p=p)
+            _check(y, oracle.gemm(sub.x, prob.planes, prob.alphas, prob.z, p=p), f"M={M} p={p}")
+    p_row = np.array([2] * 40 + [3] * 5 + [4] * 19, dtype=np.int32)
+    y = _run(prob, w, p_row=p_row)
+    _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=p_row), "mixed 64")
+
+
 @pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
 def test_parity_mixed_precision_70b_sampled(N, K, path):
     """M = 8 rows with p drawn from {2,3,4}; outputs checked on 1024 sampled

@@ -89,6 +89,8 @@ def lib():
         L.bcq_device_error.argtypes = [P]
         L.bcq_debug_wait_timeout.restype = I
         L.bcq_debug_wait_timeout.argtypes = [I, P]
+        L.bcq_quantize.restype = I
+        L.bcq_quantize.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -97,7 +99,7 @@ EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
             "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl",
             "bcq_gemm_host", "bcq_gemm_noalloc", "bcq_build_lut", "bcq_device_error",
-            "bcq_debug_wait_timeout")
+            "bcq_debug_wait_timeout", "bcq_quantize")
 
 
 def status_string(status: int) -> str:
@@ -181,6 +183,30 @@ def pack_scales(src: torch.Tensor, q: int, stream=None) -> torch.Tensor:
     return out
 
 
+def quantize(w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
+             with_sse: bool = False, stream=None):
+    """Offline quantiser (bcq_quantize): fp16 CUDA weights [N][K] ->
+    (planes int32 [p_H][N][K/32] holding the uint32 words, {p: alpha^(p) fp16
+    [N][K/128][p]} for p = p_L..p_H, z fp16 [N][K/128], and with_sse: fp64
+    [p_H - p_L + 1][N][K/128] squared error per group, else None)."""
+    _need_cuda(w, "w", torch.float16)
+    if w.dim() != 2:
+        raise ValueError("w must be [N][K]")
+    N, K = w.shape
+    G = K // GROUP
+    dev = w.device
+    planes = torch.empty((p_H, N, K // 32), dtype=torch.int32, device=dev)
+    alphas = {p: torch.empty((N, G, p), dtype=torch.float16, device=dev)
+              for p in range(p_L, p_H + 1)} if 1 <= p_L <= p_H <= 4 else {}
+    z = torch.empty((N, G), dtype=torch.float16, device=dev)
+    sse = (torch.empty((max(p_H - p_L + 1, 0), N, G), dtype=torch.float64, device=dev)
+           if with_sse else None)
+    _check(lib().bcq_quantize(_ptr(w), N, K, int(p_L), int(p_H), int(rounds), _ptr(planes),
+                              _alpha_array(alphas), _ptr(z), _ptr(sse), _stream(stream)),
+           "bcq_quantize")
+    return planes, alphas, z, sse
+
+
 PLAN_FIELDS = ("C", "consumer_warps", "NP", "D", "dyn_bytes", "stage_bytes", "units_max",
                "KB")
 
@@ -262,6 +288,14 @@ class BcqWeights:
             zz = (torch.as_tensor(z) if isinstance(z, np.ndarray) else z)
             zz = pack_scales(zz.to(device=device, dtype=torch.float16).contiguous(), 1, stream)
         return cls(packed=packed, alphas=al, z=zz, N=N, K=KW * 32, p_H=p_H)
+
+    @classmethod
+    def quantize(cls, w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
+                 stream=None):
+        """Quantise fp16 CUDA weights [N][K] on the device (bcq_quantize) and
+        pack the result for bcq_gemm."""
+        planes, alphas, z, _ = quantize(w, p_L, p_H, rounds, stream=stream)
+        return cls.from_canonical(planes, alphas, z, device=w.device, stream=stream)
 
     @classmethod
     def stack(cls, parts, device="cuda", stream=None):

@@ -1,0 +1,471 @@
+// bcq_quantize.cu -- the offline multi-precision BCQ quantiser (bcq_quantize).
+//
+// "AnyBCQ ..." (Paper-Notes page), "关键设计 / 渐进式精度扩展": at the base
+// precision p_L the codes start greedy and are refined by alternating a
+// least-squares fit of the scales with a nearest-code update; each expansion
+// p -> p + 1 keeps B_1..B_p, appends B_{p+1} = sign(R_p) and refits every
+// scale of alpha^(p+1) by least squares.  "训练策略": asymmetric, group 128,
+// 20 refinement rounds.
+//
+// One warp quantises one 128-weight group; lane l holds columns l + 32 s,
+// s = 0..3, so a ballot over the lanes of plane bit i in slot s is word s of
+// the group's canonical plane i.  Everything is fp64 (the weights are fp16,
+// widened exactly).  Per step:
+//   * the Gram matrix of the +-1 planes (and the all-ones column of z) is
+//     integer-valued and comes exactly from popcounts of the ballot words;
+//   * right-hand sides are warp sums (xor butterfly: every lane ends with the
+//     same bits, since a + b == b + a), so every lane solves the same system
+//     and holds the same scales without a broadcast;
+//   * columns exactly dependent on the columns before them (a plane equal to
+//     another, to its negation or to the all-ones column, or any exact linear
+//     dependence) get scale 0: fraction-free integer elimination decides it,
+//     then an LDL^T solve in fp64 on the kept columns gives the scales;
+//   * the code update gives every weight the code whose value
+//     z + (((alpha_1 b_1) + alpha_2 b_2) + ...) is nearest, first code in
+//     enumeration order on ties (code c: b_i = +1 where bit i of c is set).
+// The greedy start peels b = sign(r), alpha = <b, r> / 128 off r = w - mean(w);
+// sign(0) = +1.  z is fitted jointly with the base precision's scales and
+// kept for the expansions.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "bcq.h"
+
+namespace bcq {
+namespace {
+
+constexpr int kQuantGroup = 128;
+constexpr int kQuantWarps = 8;  // groups per CTA
+
+struct QuantParams {
+  const __half* w;       // fp16 [N][K]
+  uint32_t* planes;      // uint32 [p_H][N][K/32]
+  __half* alpha[4];      // alpha[q-1]: fp16 [N][G][q] (q = p_L..p_H)
+  __half* z;             // fp16 [N][G]
+  double* sse;           // fp64 [p_H - p_L + 1][N][G], or nullptr
+  long long groups;      // N * G
+  int N, K, G, rounds;
+};
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Two warp sums at once (lanes 0-15 reduce a, lanes 16-31 reduce b, then
+// both are broadcast).  Only for sums that are exact in any order: sums of
+// +-fp16 weights, whose partial sums are multiples of 2^-24 below 2^23.
+__device__ __forceinline__ void warp_sum2_exact(double a, double b, double& sa, double& sb) {
+  const bool hi = (threadIdx.x & 16) != 0;
+  double keep = hi ? b : a;
+  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 16);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  sa = __shfl_sync(0xffffffffu, keep, 0);
+  sb = __shfl_sync(0xffffffffu, keep, 16);
+}
+
+__device__ __forceinline__ double signed_val(bool plus, double a) { return plus ? a : -a; }
+
+// x_a = (adj[a][0] r_0 + adj[a][1] r_1 + ...) / det: products and sums
+// rounded one at a time, left to right (no contraction into fma).
+template <int K>
+__device__ __forceinline__ double cramer_row(const long long (&adj)[K], const double (&r)[K],
+                                             long long det) {
+  double acc = __dmul_rn((double)adj[0], r[0]);
+#pragma unroll
+  for (int b = 1; b < K; ++b) acc = __dadd_rn(acc, __dmul_rn((double)adj[b], r[b]));
+  return __ddiv_rn(acc, (double)det);
+}
+
+// Any M <= 5, any dependent columns: the kept columns (each independent of
+// the kept columns before it) by symmetric fraction-free elimination on
+// G / 2 -- a zero pivot of the positive semidefinite Schur complement means
+// its whole row and column are zero, so skipping it keeps the elimination
+// exact -- then the exact adjugate and determinant of the kept columns' Gram
+// matrix by fraction-free Gauss-Jordan elimination of [G/2 | I] (left block
+// det I, right block the adjugate; every division is exact; products in
+// 128 bits), scaled back to G: adj(G) = 2^(k-1) adj(G/2), det(G) = 2^k det(G/2).
+__device__ __forceinline__ void solve_general(int M, const int* G, const double* r, double* x) {
+  long long S[5][5];
+  for (int i = 0; i < M; ++i)
+    for (int j = 0; j < M; ++j) S[i][j] = G[i * M + j] / 2;
+  int idx[5];
+  int k = 0;
+  long long prev = 1;
+  for (int c = 0; c < M; ++c) {
+    if (S[c][c] == 0) continue;
+    idx[k++] = c;
+    for (int i = c + 1; i < M; ++i)
+      for (int j = c + 1; j < M; ++j) S[i][j] = (S[c][c] * S[i][j] - S[i][c] * S[c][j]) / prev;
+    prev = S[c][c];
+  }
+  long long A[5][10];
+  for (int a = 0; a < k; ++a)
+    for (int b = 0; b < k; ++b) {
+      A[a][b] = G[idx[a] * M + idx[b]] / 2;
+      A[a][k + b] = a == b ? 1 : 0;
+    }
+  prev = 1;
+  for (int c = 0; c < k; ++c) {
+    const long long p = A[c][c];
+    for (int i = 0; i < k; ++i) {
+      if (i == c) continue;
+      const long long f = A[i][c];
+      for (int j = 0; j < 2 * k; ++j)
+        A[i][j] = (long long)(((__int128)p * A[i][j] - (__int128)f * A[c][j]) / prev);
+    }
+    prev = p;
+  }
+  const long long det = prev * (1ll << k);
+  for (int j = 0; j < M; ++j) x[j] = 0.0;
+  for (int a = 0; a < k; ++a) {
+    const long long sc = 1ll << (k - 1);  // adj(G) = 2^(k-1) adj(G / 2)
+    double acc = __dmul_rn((double)(A[a][k] * sc), r[idx[0]]);
+    for (int b = 1; b < k; ++b)
+      acc = __dadd_rn(acc, __dmul_rn((double)(A[a][k + b] * sc), r[idx[b]]));
+    x[idx[a]] = __ddiv_rn(acc, (double)det);
+  }
+}
+
+// Least squares on M columns with integer Gram matrix G and right-hand
+// sides r, by Cramer's rule with the exact adjugate; columns dependent on
+// earlier ones get 0.  Full-rank systems of 1 to 4 columns (every leading
+// principal minor non-zero) take closed forms; the rest solve_general.
+template <int M>
+__device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (&r)[M],
+                                            double (&x)[M]) {
+  if constexpr (M == 1) {
+    x[0] = __ddiv_rn(r[0], (double)G[0][0]);  // adj = [1]; G[0][0] = 128
+    return;
+  } else if constexpr (M == 2) {
+    const long long det = (long long)G[0][0] * G[1][1] - (long long)G[0][1] * G[1][0];
+    if (det != 0) {
+      const long long a0[2] = {G[1][1], -G[0][1]}, a1[2] = {-G[1][0], G[0][0]};
+      x[0] = cramer_row<2>(a0, r, det);
+      x[1] = cramer_row<2>(a1, r, det);
+      return;
+    }
+  } else if constexpr (M == 3) {
+    const int g00 = G[0][0], g01 = G[0][1], g02 = G[0][2], g11 = G[1][1], g12 = G[1][2],
+              g22 = G[2][2];
+    const long long c00 = g11 * g22 - g12 * g12, c01 = g02 * g12 - g01 * g22,
+                    c02 = g01 * g12 - g02 * g11, c11 = g00 * g22 - g02 * g02,
+                    c12 = g01 * g02 - g00 * g12, c22 = g00 * g11 - g01 * g01;
+    const long long det = g00 * c00 + g01 * c01 + g02 * c02;
+    if (c22 != 0 && det != 0) {  // leading minors: g00 = 128, c22, det
+      const long long a0[3] = {c00, c01, c02}, a1[3] = {c01, c11, c12}, a2[3] = {c02, c12, c22};
+      x[0] = cramer_row<3>(a0, r, det);
+      x[1] = cramer_row<3>(a1, r, det);
+      x[2] = cramer_row<3>(a2, r, det);
+      return;
+    }
+  } else if constexpr (M == 4) {
+    // Laplace expansion by the 2x2 minors of rows 0-1 (s) and rows 2-3 (c)
+    const long long a00 = G[0][0], a01 = G[0][1], a02 = G[0][2], a03 = G[0][3];
+    const long long a11 = G[1][1], a12 = G[1][2], a13 = G[1][3];
+    const long long a22 = G[2][2], a23 = G[2][3], a33 = G[3][3];
+    const long long a10 = a01, a20 = a02, a21 = a12, a30 = a03, a31 = a13, a32 = a23;
+    const long long s0 = a00 * a11 - a10 * a01, s1 = a00 * a12 - a10 * a02,
+                    s2 = a00 * a13 - a10 * a03, s3 = a01 * a12 - a11 * a02,
+                    s4 = a01 * a13 - a11 * a03, s5 = a02 * a13 - a12 * a03;
+    const long long c5 = a22 * a33 - a32 * a23, c4 = a21 * a33 - a31 * a23,
+                    c3 = a21 * a32 - a31 * a22, c2 = a20 * a33 - a30 * a23,
+                    c1 = a20 * a32 - a30 * a22, c0 = a20 * a31 - a30 * a21;
+    const long long det = s0 * c5 - s1 * c4 + s2 * c3 + s3 * c2 - s4 * c1 + s5 * c0;
+    const long long b00 = a11 * c5 - a12 * c4 + a13 * c3, b01 = -a01 * c5 + a02 * c4 - a03 * c3,
+                    b02 = a31 * s5 - a32 * s4 + a33 * s3, b03 = -a21 * s5 + a22 * s4 - a23 * s3,
+                    b11 = a00 * c5 - a02 * c2 + a03 * c1, b12 = -a30 * s5 + a32 * s2 - a33 * s1,
+                    b13 = a20 * s5 - a22 * s2 + a23 * s1, b22 = a30 * s4 - a31 * s2 + a33 * s0,
+                    b23 = -a20 * s4 + a21 * s2 - a23 * s0, b33 = a20 * s3 - a21 * s1 + a22 * s0;
+    if (s0 != 0 && b33 != 0 && det != 0) {  // leading minors: a00, s0, b33 (= 3x3), det
+      const long long r0[4] = {b00, b01, b02, b03}, r1[4] = {b01, b11, b12, b13},
+                      r2[4] = {b02, b12, b22, b23}, r3[4] = {b03, b13, b23, b33};
+      x[0] = cramer_row<4>(r0, r, det);
+      x[1] = cramer_row<4>(r1, r, det);
+      x[2] = cramer_row<4>(r2, r, det);
+      x[3] = cramer_row<4>(r3, r, det);
+      return;
+    }
+  }
+  if constexpr (M >= 2) solve_general(M, &G[0][0], r, x);
+}
+
+// Ballot words of the first P planes: P[i][s] = plane i, columns 32 s..32 s + 31.
+template <int P>
+__device__ __forceinline__ void plane_words(const unsigned (&code)[4], uint32_t (&pw)[P][4]) {
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) pw[i][s] = __ballot_sync(0xffffffffu, (code[s] >> i) & 1u);
+}
+
+__device__ __forceinline__ int dot_pm1(const uint32_t (&a)[4], const uint32_t (&b)[4]) {
+  return kQuantGroup - 2 * (__popc(a[0] ^ b[0]) + __popc(a[1] ^ b[1]) +
+                            __popc(a[2] ^ b[2]) + __popc(a[3] ^ b[3]));
+}
+__device__ __forceinline__ int sum_pm1(const uint32_t (&a)[4]) {
+  return 2 * (__popc(a[0]) + __popc(a[1]) + __popc(a[2]) + __popc(a[3])) - kQuantGroup;
+}
+
+// Exact sums sum(b_i w) of the first P planes, i = 0..P-1.
+template <int P>
+__device__ __forceinline__ void signed_sums(const double (&w)[4], const unsigned (&code)[4],
+                                            double (&S)[P]) {
+  double t[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    t[i] = 0.0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) t[i] += signed_val((code[s] >> i) & 1u, w[s]);
+  }
+#pragma unroll
+  for (int i = 0; i + 1 < P; i += 2) warp_sum2_exact(t[i], t[i + 1], S[i], S[i + 1]);
+  if constexpr (P % 2 == 1) S[P - 1] = warp_sum(t[P - 1]);
+}
+
+// Joint least squares for (z, alpha_1..alpha_P): columns [ones, b_1..b_P],
+// right-hand sides sum(w) and sum(b_i w).
+template <int P>
+__device__ __forceinline__ void lsq_with_offset(const double (&w)[4], double sumw,
+                                                const unsigned (&code)[4], double (&alpha)[P],
+                                                double& z) {
+  uint32_t pw[P][4];
+  plane_words<P>(code, pw);
+  int G[P + 1][P + 1];
+  double r[P + 1], x[P + 1], S[P];
+  signed_sums<P>(w, code, S);
+  G[0][0] = kQuantGroup;
+  r[0] = sumw;
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    G[0][i + 1] = G[i + 1][0] = sum_pm1(pw[i]);
+#pragma unroll
+    for (int j = 0; j <= i; ++j) G[i + 1][j + 1] = G[j + 1][i + 1] = dot_pm1(pw[i], pw[j]);
+    r[i + 1] = S[i];
+  }
+  solve_exact<P + 1>(G, r, x);
+  z = x[0];
+#pragma unroll
+  for (int i = 0; i < P; ++i) alpha[i] = x[i + 1];
+}
+
+// Least squares for alpha_1..alpha_P with z fixed: columns [b_1..b_P],
+// right-hand sides sum(b_i (w - z)) = sum(b_i w) - z sum(b_i).
+template <int P>
+__device__ __forceinline__ void lsq_fixed_offset(const double (&w)[4], double z,
+                                                 const unsigned (&code)[4], double (&alpha)[P]) {
+  uint32_t pw[P][4];
+  plane_words<P>(code, pw);
+  int G[P][P];
+  double r[P], S[P];
+  signed_sums<P>(w, code, S);
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+#pragma unroll
+    for (int j = 0; j <= i; ++j) G[i][j] = G[j][i] = dot_pm1(pw[i], pw[j]);
+    r[i] = __dsub_rn(S[i], __dmul_rn(z, (double)sum_pm1(pw[i])));
+  }
+  solve_exact<P>(G, r, alpha);
+}
+
+// z + (((alpha_1 b_1) + alpha_2 b_2) + ...) for code c.
+template <int P>
+__device__ __forceinline__ double code_value(const double (&alpha)[P], double z, unsigned c) {
+  double acc = signed_val(c & 1u, alpha[0]);
+#pragma unroll
+  for (int i = 1; i < P; ++i) acc += signed_val((c >> i) & 1u, alpha[i]);
+  return z + acc;
+}
+
+template <int P>
+__device__ __forceinline__ void nearest_codes(const double (&w)[4], const double (&alpha)[P],
+                                              double z, unsigned (&code)[4]) {
+  constexpr int C = 1 << P;
+  double v[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) v[c] = code_value<P>(alpha, z, (unsigned)c);
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    unsigned best = 0;
+    double be = fabs(w[s] - v[0]);
+#pragma unroll
+    for (int c = 1; c < C; ++c) {
+      const double e = fabs(w[s] - v[c]);
+      if (e < be) {
+        be = e;
+        best = (unsigned)c;
+      }
+    }
+    code[s] = best;
+  }
+}
+
+template <int P>
+__device__ __forceinline__ double group_sse(const double (&w)[4], const double (&alpha)[P],
+                                            double z, const unsigned (&code)[4]) {
+  double t = 0.0;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const double e = w[s] - code_value<P>(alpha, z, code[s]);
+    t += e * e;
+  }
+  return warp_sum(t);
+}
+
+// alpha^(P) of the group rounded to fp16 (nearest even), and its error.
+template <int P>
+__device__ __forceinline__ void store_scales(const QuantParams& q, long long gid, int lane,
+                                             const double (&alpha)[P], double sse, int p_L) {
+  __half* a = q.alpha[P - 1] + gid * P;
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (lane == i) a[i] = __double2half(alpha[i]);
+  if (q.sse && lane == 0) q.sse[(long long)(P - p_L) * q.groups + gid] = sse;
+}
+
+// Base precision PL: greedy start, refinement rounds, final refit.
+template <int PL>
+__device__ __forceinline__ void base_precision(const QuantParams& q, const double (&w)[4],
+                                               double sumw, unsigned (&code)[4],
+                                               double (&alpha)[PL], double& z) {
+  z = sumw / kQuantGroup;  // exact: the sum is exact, 128 a power of two
+  double r[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    r[s] = w[s] - z;
+    code[s] = 0;
+  }
+  uint32_t pw[PL][4];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) code[s] |= (r[s] >= 0.0 ? 1u : 0u) << i;  // b_i = sign(r)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) pw[i][s] = __ballot_sync(0xffffffffu, (code[s] >> i) & 1u);
+    // <b_i, r> = sum(b_i w) - z sum(b_i) - sum_j alpha_j <b_i, b_j>, left to right
+    double t = 0.0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) t += signed_val((code[s] >> i) & 1u, w[s]);
+    t = warp_sum(t);
+    t = __dsub_rn(t, __dmul_rn(z, (double)sum_pm1(pw[i])));
+#pragma unroll
+    for (int j = 0; j < i; ++j) t = __dsub_rn(t, __dmul_rn(alpha[j], (double)dot_pm1(pw[i], pw[j])));
+    const double a = t / kQuantGroup;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) r[s] = ((code[s] >> i) & 1u) ? r[s] - a : r[s] + a;
+    alpha[i] = a;
+  }
+  for (int it = 0; it < q.rounds; ++it) {
+    lsq_with_offset<PL>(w, sumw, code, alpha, z);
+    nearest_codes<PL>(w, alpha, z, code);
+  }
+  lsq_with_offset<PL>(w, sumw, code, alpha, z);
+}
+
+template <int P, int PH>
+__device__ __forceinline__ void expand(const QuantParams& q, long long gid, int lane, int p_L,
+                                       const double (&w)[4], double z, unsigned (&code)[4],
+                                       const double (&alpha)[P]) {
+  if constexpr (P < PH) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const double res = w[s] - code_value<P>(alpha, z, code[s]);
+      code[s] |= (res >= 0.0 ? 1u : 0u) << P;
+    }
+    double next[P + 1];
+    lsq_fixed_offset<P + 1>(w, z, code, next);
+    const double e = q.sse ? group_sse<P + 1>(w, next, z, code) : 0.0;
+    store_scales<P + 1>(q, gid, lane, next, e, p_L);
+    expand<P + 1, PH>(q, gid, lane, p_L, w, z, code, next);
+  }
+}
+
+template <int PL, int PH>
+__global__ void __launch_bounds__(32 * kQuantWarps) quantize_kernel(QuantParams q) {
+  const int lane = threadIdx.x & 31;
+  const long long gid = (long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (gid >= q.groups) return;  // uniform per warp
+  const long long n = gid / q.G;
+  const int g = (int)(gid - n * q.G);
+  const __half* src = q.w + n * q.K + (long long)g * kQuantGroup;
+  double w[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) w[s] = (double)__half2float(src[lane + 32 * s]);
+  const double sumw = warp_sum(((w[0] + w[1]) + w[2]) + w[3]);
+
+  unsigned code[4];
+  double alpha[PL], z;
+  base_precision<PL>(q, w, sumw, code, alpha, z);
+  const double e = q.sse ? group_sse<PL>(w, alpha, z, code) : 0.0;
+  store_scales<PL>(q, gid, lane, alpha, e, PL);
+  if (lane == 0) q.z[gid] = __double2half(z);
+  expand<PL, PH>(q, gid, lane, PL, w, z, code, alpha);
+
+  // planes: lane 4 i + s writes word s of plane i
+  uint32_t pw[PH][4];
+  plane_words<PH>(code, pw);
+  const int KW = q.K / 32;
+#pragma unroll
+  for (int i = 0; i < PH; ++i)
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (lane == 4 * i + s) q.planes[((long long)i * q.N + n) * KW + 4 * g + s] = pw[i][s];
+}
+
+using QuantKernel = void (*)(QuantParams);
+
+QuantKernel quantize_kernel_for(int p_L, int p_H) {
+#define BCQ_Q(a, b) \
+  if (p_L == a && p_H == b) return quantize_kernel<a, b>;
+  BCQ_Q(1, 1) BCQ_Q(1, 2) BCQ_Q(1, 3) BCQ_Q(1, 4)
+  BCQ_Q(2, 2) BCQ_Q(2, 3) BCQ_Q(2, 4)
+  BCQ_Q(3, 3) BCQ_Q(3, 4)
+  BCQ_Q(4, 4)
+#undef BCQ_Q
+  return nullptr;
+}
+
+bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+}  // namespace bcq
+
+extern "C" bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int p_H,
+                                   int rounds, uint32_t* planes, uint16_t* const alpha[4],
+                                   uint16_t* z, double* sse, void* stream) {
+  using namespace bcq;
+  if (!alpha) return BCQ_ERR_NULL;
+  if (p_H < 1 || p_H > BCQ_MAX_PLANES || p_L < 1 || p_L > p_H) return BCQ_ERR_PRECISION;
+  if (N < 0 || K < 0 || K % BCQ_GROUP != 0 || rounds < 0 || rounds > 1000) return BCQ_ERR_SHAPE;
+  if ((long long)N * (K / BCQ_GROUP) > (1ll << 33)) return BCQ_ERR_SHAPE;
+  if (N == 0 || K == 0) return BCQ_OK;
+  if (!w || !planes || !z) return BCQ_ERR_NULL;
+  for (int p = p_L; p <= p_H; ++p)
+    if (!alpha[p - 1]) return BCQ_ERR_PRECISION;
+  if (!aligned_to(w, 2) || !aligned_to(planes, 4) || !aligned_to(z, 2) ||
+      (sse && !aligned_to(sse, 8)))
+    return BCQ_ERR_ALIGN;
+  for (int p = p_L; p <= p_H; ++p)
+    if (!aligned_to(alpha[p - 1], 2)) return BCQ_ERR_ALIGN;
+  QuantParams q{};
+  q.w = reinterpret_cast<const __half*>(w);
+  q.planes = planes;
+  for (int p = 1; p <= 4; ++p)
+    q.alpha[p - 1] = (p >= p_L && p <= p_H) ? reinterpret_cast<__half*>(alpha[p - 1]) : nullptr;
+  q.z = reinterpret_cast<__half*>(z);
+  q.sse = sse;
+  q.N = N;
+  q.K = K;
+  q.G = K / BCQ_GROUP;
+  q.groups = (long long)N * q.G;
+  q.rounds = rounds;
+  const QuantKernel fn = quantize_kernel_for(p_L, p_H);
+  if (!fn) return BCQ_ERR_UNSUPPORTED;
+  const long long blocks = (q.groups + kQuantWarps - 1) / kQuantWarps;
+  fn<<<(unsigned)blocks, 32 * kQuantWarps, 0, (cudaStream_t)stream>>>(q);
+  return cudaGetLastError() == cudaSuccess ? BCQ_OK : BCQ_ERR_CUDA;
+}

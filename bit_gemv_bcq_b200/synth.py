@@ -87,3 +87,20 @@ def make_x(M: int, K: int, *, seed: int) -> np.ndarray:
     """Extra activations ~ N(0,1), fp16, from their own seeded generator."""
     rng = np.random.default_rng(seed)
     return rng.normal(0.0, 1.0, size=(M, K)).astype(np.float16)
+
+
+def make_weights(N: int, K: int, *, seed: int, outliers: bool = True) -> np.ndarray:
+    """fp16 weights [N][K] for the offline quantiser, shaped like a trained
+    projection matrix.  Recipe (``np.random.default_rng(seed)``, draws in this
+    order): row scales s_n = 0.02 * U(0.5, 1.5); w = s_n * N(0, 1); when
+    ``outliers``, round(0.001 N K) entries (positions without replacement)
+    multiplied by 8; then rounded to fp16."""
+    rng = np.random.default_rng(seed)
+    s = 0.02 * rng.uniform(0.5, 1.5, size=(N, 1))
+    w = s * rng.normal(0.0, 1.0, size=(N, K))
+    if outliers and N * K > 0:
+        n_out = int(round(0.001 * N * K))
+        if n_out:
+            idx = rng.choice(N * K, size=n_out, replace=False)
+            w.reshape(-1)[idx] *= 8.0
+    return w.astype(np.float16)

@@ -245,6 +245,51 @@ bcq_status bcq_gemm_noalloc(const uint16_t* x, const uint32_t* planes,
                             int p_H, int group, uint16_t* y, void* stream);
 
 /*
+ * Offline quantiser: fp16 weights -> shared bit-planes, per-precision scales
+ * alpha^(p) for p = p_L..p_H and one offset per group, in the canonical
+ * layouts that bcq_pack_planes / bcq_pack_scales take.
+ *
+ * Source: AnyBCQ (Paper-Notes page), "关键设计 / 渐进式精度扩展" (greedy start
+ * and alternating refinement -- least squares for the scales, nearest code
+ * for every weight -- at the base precision p_L; each expansion p -> p + 1
+ * keeps B_1..B_p, appends B_{p+1} = sign(R_p), the sign of the residual, and
+ * refits all p + 1 scales by least squares) and "训练策略" (asymmetric,
+ * group size 128, 20 refinement rounds).  Each 128-column group of each row
+ * is an independent problem, computed in fp64:
+ *   - greedy start: z = mean(w); for i = 1..p_L: b_i = sign(r) (sign(0) = +1),
+ *     alpha_i = <b_i, r> / 128, r -= alpha_i b_i, from r = w - z;
+ *   - `rounds` times: (z, alpha) = joint least squares for the current codes;
+ *     then every weight takes the code whose value
+ *     z + (((alpha_1 b_1) + alpha_2 b_2) + ...) is nearest (ties: the code with
+ *     the smallest index c, b_i = +1 where bit i of c is set); then a final
+ *     least-squares refit.  z is kept from here on;
+ *   - in a least-squares fit, a column (the all-ones column of z first, then
+ *     planes 1..p) that is an exact linear combination of the columns before
+ *     it gets scale 0;
+ *   - scales and offsets are rounded to fp16 (nearest even) when stored.
+ *
+ *   w       device, fp16 [N][K] row-major, 2-byte aligned, read only.
+ *   N, K    N >= 0, K >= 0, K % 128 == 0 (N == 0 or K == 0: nothing to do).
+ *   p_L, p_H  1 <= p_L <= p_H <= 4.
+ *   rounds  refinement rounds at p_L, 0..1000 (the page uses 20).
+ *   planes  device, uint32 [p_H][N][K/32], 4-byte aligned, overwritten
+ *           (bit j of word w of row n = column 32w + j, 1 = +1).
+ *   alpha   HOST array of 4 device pointers; alpha[p-1] for p = p_L..p_H
+ *           receives fp16 [N][K/128][p] (2-byte aligned); the others are
+ *           ignored and may be NULL.
+ *   z       device, fp16 [N][K/128], 2-byte aligned, overwritten.
+ *   sse     device, fp64 [p_H - p_L + 1][N][K/128], 8-byte aligned, or NULL:
+ *           the squared error of every group at precision p_L + j with the
+ *           unrounded scales.
+ * Errors: NULL pointers -> BCQ_ERR_NULL; p_L / p_H out of range or a needed
+ * alpha NULL -> BCQ_ERR_PRECISION; bad N, K or rounds -> BCQ_ERR_SHAPE;
+ * misaligned pointers -> BCQ_ERR_ALIGN; launch failure -> BCQ_ERR_CUDA.
+ */
+bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int p_H, int rounds,
+                        uint32_t* planes, uint16_t* const alpha[4], uint16_t* z,
+                        double* sse, void* stream);
+
+/*
  * The lookup table and group sums exactly as the GEMV kernel builds them in
  * shared memory (AnyBCQ page, "直接bit-plane运算的CUDA内核": cached signed
  * partial sums of x).  For test and inspection.

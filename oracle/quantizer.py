@@ -27,7 +27,9 @@ Readings (the pages leave them open):
     group mean, and is frozen afterwards, so that, like the codes, it is
     shared and the error can only fall as planes are added;
   * greedy initialisation: b_i = sign(r), alpha_i = <b_i, r> / n, r -= alpha_i b_i,
-    starting from r = w - mean(w);
+    starting from r = w - mean(w); <b_i, r> is evaluated as
+    sum(b_i w) - z sum(b_i) - sum_j alpha_j <b_i, b_j> (exact sums and
+    integers, left to right);
   * "BS" (the code update) is read as its result: every weight takes the
     code in {-1,+1}^p whose value z + sum_i alpha_i b_i is nearest to the
     weight; ties go to the candidate enumerated first (candidate c has
@@ -41,8 +43,10 @@ Readings (the pages leave them open):
     other exact dependence) is solved on the columns that are independent
     of the columns before them, in column order (the all-ones column of z
     first, then planes 1..p); the others get scale 0.  A constant group is
-    thus all offset (z = its value, alpha = 0).  The Gram matrix of +-1 and all-ones columns is integer-valued, so the
-    dependence is decided exactly (rational elimination);
+    thus all offset (z = its value, alpha = 0).  The Gram matrix of +-1 and
+    all-ones columns is integer-valued, so the dependence is decided exactly
+    (integer determinants), and the normal equations are solved by Cramer's
+    rule with the exact integer adjugate and determinant;
   * candidate values and residuals are formed in fp64 as
     z + (((alpha_1 b_1) + alpha_2 b_2) + ...), left to right;
   * sign(0) = +1; inputs are fp16 weights widened to fp64; scales and offsets
@@ -50,61 +54,87 @@ Readings (the pages leave them open):
 """
 from __future__ import annotations
 
-from fractions import Fraction
-
 import numpy as np
 
 from .quant import sign_pm1
 
 
+def det_int(M) -> int:
+    """Exact determinant of a small integer matrix (Python integers, Laplace
+    expansion along the first row)."""
+    M = [[int(v) for v in row] for row in M]
+    if not M:
+        return 1
+    if len(M) == 2:
+        return M[0][0] * M[1][1] - M[0][1] * M[1][0]
+    if len(M) == 1:
+        return M[0][0]
+    return sum((-1) ** j * M[0][j] * det_int([r[:j] + r[j + 1:] for r in M[1:]])
+               for j in range(len(M)))
+
+
+def adjugate_int(M) -> list:
+    """Exact adjugate: adj[i][j] = (-1)^(i+j) det(M without row j and column i)."""
+    M = [[int(v) for v in row] for row in M]
+    n = len(M)
+    return [[(-1) ** (i + j) * det_int([r[:i] + r[i + 1:] for k, r in enumerate(M) if k != j])
+             for j in range(n)] for i in range(n)]
+
+
 def independent_columns(gram) -> list:
     """Columns of an integer Gram matrix that are linearly independent of
-    the columns before them, decided in exact rational arithmetic.
-
-    Column j is kept when the Gram matrix of the kept columns plus j is
-    non-singular, i.e. when Gaussian elimination (over the rationals) of
-    that matrix finds a non-zero pivot in every column."""
-    G = [[Fraction(int(round(v))) for v in row] for row in np.asarray(gram)]
+    the kept columns before them: column j is kept when the Gram matrix of
+    the kept columns plus j has a non-zero determinant (exact integers)."""
+    G = [[int(round(float(v))) for v in row] for row in gram]
     kept = []
     for j in range(len(G)):
         trial = kept + [j]
-        A = [[G[r][c] for c in trial] for r in trial]
-        n = len(trial)
-        full = True
-        for col in range(n):
-            piv = next((r for r in range(col, n) if A[r][col] != 0), None)
-            if piv is None:
-                full = False
-                break
-            A[col], A[piv] = A[piv], A[col]
-            for r in range(col + 1, n):
-                f = A[r][col] / A[col][col]
-                if f:
-                    A[r] = [a - f * b for a, b in zip(A[r], A[col])]
-        if full:
+        if det_int([[G[a][b] for b in trial] for a in trial]) != 0:
             kept.append(j)
     return kept
+
+
+def solve_normal_equations(gram, rhs):
+    """x with gram x = rhs on the kept columns (0 elsewhere), by Cramer's rule
+    with the exact integer adjugate and determinant of the kept columns' Gram
+    matrix: x_a = (adj[a][0] r_0 + adj[a][1] r_1 + ...) / det, the products
+    and sums in fp64 from left to right."""
+    kept = independent_columns(gram)
+    G = [[int(round(float(v))) for v in row] for row in gram]
+    Gk = [[G[a][b] for b in kept] for a in kept]
+    r = [float(v) for v in rhs]
+    adj = adjugate_int(Gk)
+    det = float(det_int(Gk))
+    x = np.zeros(len(r))
+    for a, ka in enumerate(kept):
+        acc = float(adj[a][0]) * r[kept[0]]
+        for b in range(1, len(kept)):
+            acc = acc + float(adj[a][b]) * r[kept[b]]
+        x[ka] = acc / det
+    return x
 
 
 def lsq(W, B, z=None):
     """Least squares per problem.  W [P][n]; B [P][p][n] in {-1,+1}.
     With z None the unknowns are (z, alpha_1..alpha_p) (an all-ones column
     first); otherwise z [P] is fixed and only alpha is solved.
-    Returns (alpha [P][p], z [P])."""
+    Returns (alpha [P][p], z [P]).
+
+    Right-hand sides: with z free, sum(w) and sum(b_i w); with z fixed,
+    sum(b_i (w - z)) evaluated as sum(b_i w) - z sum(b_i).  For fp16 weights
+    sum(b_i w) is exact in fp64 in any order (every partial sum is a multiple
+    of 2^-24 below 2^23) and sum(b_i) is an integer, so every right-hand
+    side is exact or one rounding from exact."""
     W = np.asarray(W, dtype=np.float64)
     P, p, n = B.shape
     if z is None:
         A = np.concatenate([np.ones((P, 1, n)), B], axis=1)
-        target = W
+        rhs = np.einsum("qin,qn->qi", A, W)
     else:
         A = B
-        target = W - z[:, None]
+        rhs = np.einsum("qin,qn->qi", B, W) - z[:, None] * B.sum(axis=2)
     gram = np.einsum("qin,qjn->qij", A, A)        # integers, exact in fp64
-    rhs = np.einsum("qin,qn->qi", A, target)
-    sol = np.zeros_like(rhs)
-    for q in range(P):
-        kept = independent_columns(gram[q])
-        sol[q, kept] = np.linalg.solve(gram[q][np.ix_(kept, kept)], rhs[q, kept])
+    sol = np.stack([solve_normal_equations(gram[q], rhs[q]) for q in range(P)])
     if z is None:
         return sol[:, 1:], sol[:, 0]
     return sol, np.array(z, dtype=np.float64, copy=True)
@@ -170,7 +200,11 @@ def quantize_groups(W, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None)
     Bs, alphas = [], []
     for _ in range(p_L):
         b = sign_pm1(r)
-        a = np.sum(b * r, axis=1) / n
+        # <b, r> = sum(b w) - z sum(b) - sum_j alpha_j <b, b_j>, left to right
+        t = np.sum(b * W, axis=1) - z * np.sum(b, axis=1)
+        for bj, aj in zip(Bs, alphas):
+            t = t - aj * np.sum(b * bj, axis=1)
+        a = t / n
         r = r - a[:, None] * b
         Bs.append(b)
         alphas.append(a)
@@ -195,19 +229,19 @@ def quantize_groups(W, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None)
     return B, out_alpha, z
 
 
-def quantize(W, group: int = 128, p_L: int = 2, p_H: int = 4, rounds: int = 20):
+def quantize(W, group: int = 128, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None):
     """Quantise a weight W [N][K] (K a multiple of the group size and of 32)
     into the canonical format the GEMV reads.
 
     Returns (planes uint32 [p_H][N][K/32], bit j of word w = column 32w + j,
     bit 1 = +1; {p: alpha^(p) fp64 [N][K/group][p]} for p = p_L..p_H;
-    z fp64 [N][K/group])."""
+    z fp64 [N][K/group]).  trace: as for quantize_groups (groups row-major)."""
     W = np.asarray(W, dtype=np.float64)
     N, K = W.shape
     if K % group or K % 32:
         raise ValueError("K must be a multiple of the group size and of 32")
     G = K // group
-    B, alphas, z = quantize_groups(W.reshape(N * G, group), p_L, p_H, rounds)
+    B, alphas, z = quantize_groups(W.reshape(N * G, group), p_L, p_H, rounds, trace)
     bits = (B > 0).reshape(N, G, p_H, group).transpose(2, 0, 1, 3).reshape(p_H, N, K)
     words = bits.reshape(p_H, N, K // 32, 32).astype(np.uint64)
     planes = np.sum(words << np.arange(32, dtype=np.uint64), axis=3).astype(np.uint32)

@@ -36,7 +36,7 @@ MUTANTS = {
         "np.where((c >> np.arange(p)[None, :]) & 1, 1.0, -1.0)",
         "np.where((c >> np.arange(p)[::-1][None, :]) & 1, 1.0, -1.0)"),
     "greedy_scale_over_n_minus_1": (
-        "a = np.sum(b * r, axis=1) / n", "a = np.sum(b * r, axis=1) / (n - 1)"),
+        "        a = t / n\n", "        a = t / (n - 1)\n"),
     "greedy_from_raw_weights": ("    r = W - z[:, None]\n", "    r = W.copy()\n"),
     "one_round_short": ("    for _ in range(rounds):", "    for _ in range(rounds - 1):"),
     "no_final_refit": (
@@ -45,8 +45,19 @@ MUTANTS = {
         "        alpha, z = lsq(W, B)\n        record(\"lsq\"",
         "        alpha, _ = lsq(W, B, z)\n        record(\"lsq\""),
     "dependent_columns_min_norm": (
-        "        sol[q, kept] = np.linalg.solve(gram[q][np.ix_(kept, kept)], rhs[q, kept])",
-        "        sol[q] = np.linalg.lstsq(gram[q], rhs[q], rcond=None)[0]"),
+        "    sol = np.stack([solve_normal_equations(gram[q], rhs[q]) for q in range(P)])",
+        "    sol = np.stack([np.linalg.lstsq(gram[q], rhs[q], rcond=None)[0] for q in range(P)])"),
+    "adjugate_transposed_cofactor": (
+        "[r[:i] + r[i + 1:] for k, r in enumerate(M) if k != j]",
+        "[r[:j] + r[j + 1:] for k, r in enumerate(M) if k != i]"),
+    "adjugate_sign_pattern": ("(-1) ** (i + j) * det_int", "(-1) ** i * det_int"),
+    "cramer_drops_last_term": (
+        "        for b in range(1, len(kept)):", "        for b in range(1, len(kept) - 1):"),
+    "greedy_ignores_earlier_planes": (
+        "            t = t - aj * np.sum(b * bj, axis=1)", "            t = t - 0.0 * aj"),
+    "fixed_offset_rhs_sign": (
+        "np.einsum(\"qin,qn->qi\", B, W) - z[:, None] * B.sum(axis=2)",
+        "np.einsum(\"qin,qn->qi\", B, W) + z[:, None] * B.sum(axis=2)"),
     "offset_column_last": (
         "A = np.concatenate([np.ones((P, 1, n)), B], axis=1)",
         "A = np.concatenate([B, np.ones((P, 1, n))], axis=1)"),
@@ -56,9 +67,8 @@ MUTANTS = {
     "packing_groups_transposed": (
         "bits = (B > 0).reshape(N, G, p_H, group).transpose(2, 0, 1, 3).reshape(p_H, N, K)",
         "bits = (B > 0).reshape(G, N, p_H, group).transpose(2, 1, 0, 3).reshape(p_H, N, K)"),
-    "rank_test_skips_last_pivot": (
-        "        for col in range(n):\n            piv",
-        "        for col in range(n - 1):\n            piv"),
+    "dependence_test_skips_last_column": (
+        "    for j in range(len(G)):", "    for j in range(len(G) - 1):"),
 }
 
 

@@ -115,6 +115,30 @@ def test_independent_columns_random_against_rank():
 
 # --------------------------------------------------------------- least squares
 
+def test_adjugate_and_determinant_identities():
+    # M adj(M) = adj(M) M = det(M) I on random integer matrices (not symmetric),
+    # and det against numpy's floating-point determinant
+    rng = np.random.default_rng(4)
+    for k in range(1, 6):
+        for _ in range(20):
+            M = rng.integers(-9, 10, (k, k))
+            adj = np.array(Q.adjugate_int(M), dtype=np.int64)
+            d = Q.det_int(M)
+            assert np.array_equal(M @ adj, d * np.eye(k, dtype=np.int64))
+            assert np.array_equal(adj @ M, d * np.eye(k, dtype=np.int64))
+            assert abs(d - np.linalg.det(M)) < 1e-6 * max(1.0, abs(d))
+    assert Q.det_int(np.zeros((0, 0))) == 1
+
+
+def test_solve_normal_equations_closed_forms():
+    # 1x1: x = r / g; 2x2 [[2, 1], [1, 2]] x = (3, 3) -> (1, 1); a dependent
+    # middle column gets 0 and the others solve the reduced system
+    assert np.array_equal(Q.solve_normal_equations(np.array([[128.0]]), np.array([64.0])), [0.5])
+    assert np.array_equal(Q.solve_normal_equations(np.array([[2.0, 1], [1, 2]]), np.array([3.0, 3])),
+                          [1.0, 1.0])
+    G = np.array([[4.0, 4, 0], [4, 4, 0], [0, 0, 4]])
+    assert np.array_equal(Q.solve_normal_equations(G, np.array([8.0, 8, 2])), [2.0, 0.0, 0.5])
+
 def test_lsq_reproduces_biloco_joint_refit():
     g = _read_golden("biloco_greedy_3x2.txt")
     W = g["W"].reshape(1, -1)                                   # 3x2 flattened

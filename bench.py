@@ -77,6 +77,23 @@ def recorded_traffic():
         return None
 
 
+def recorded_quantizer_insts():
+    """Warp instructions per group of the quantiser kernel from the committed
+    ncu capture, or None when bcq_quantize.cu changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "quantize_issue.json")) as f:
+            t = json.load(f)
+        with open(os.path.join(ROOT, "bit_gemv_bcq_b200", "csrc", "bcq_quantize.cu"), "rb") as f:
+            h = hashlib.sha256(b"bcq_quantize.cu" + f.read()).hexdigest()
+        return t if t.get("source_sha256") == h else None
+    except Exception:
+        return None
+
+
+SM_COUNT, SM_SUBPARTITIONS, SM_MAX_MHZ = 148, 4, 1965.0
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -339,6 +356,81 @@ def run_gpu(args, rank, world, local_rank):
     return result
 
 
+def run_quantizer(args, dev, rows=N_OUT):
+    """The offline quantiser (bcq_quantize) on one fp16 weight of `rows` x
+    K_IN: p_L = 2 -> p_H = 4, 20 refinement rounds.  Each timed call is
+    preceded by an L2 flush (a write of 2x L2) outside its events."""
+    import torch
+    from bit_gemv_bcq_b200 import api, synth
+    w16 = synth.make_weights(rows, K_IN, seed=args.seed + 7)
+    w = torch.from_numpy(w16.view(np.int16)).view(torch.float16).to(dev)
+    G = K_IN // GROUP
+    planes = torch.empty((P_H, rows, K_IN // 32), dtype=torch.int32, device=dev)
+    alphas = {p: torch.empty((rows, G, p), dtype=torch.float16, device=dev) for p in PRECISIONS}
+    z = torch.empty((rows, G), dtype=torch.float16, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    arr = api._alpha_array(alphas)
+
+    def call():
+        st = api.lib().bcq_quantize(api._ptr(w), rows, K_IN, 2, P_H, 20, api._ptr(planes), arr,
+                                    api._ptr(z), None, api._stream(stream))
+        if st != api.BCQ_OK:
+            raise api.BcqError(st, "bcq_quantize")
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    stream.synchronize()
+    reps = 10
+    ms = 0.0
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+        b.synchronize()
+        ms += a.elapsed_time(b)
+    ms /= reps
+    assert api.device_error(stream) == api.BCQ_OK
+    groups = rows * G
+    out = {"workload": f"bcq_quantize fp16 {rows}x{K_IN}, g=128, p_L=2 -> p_H=4, 20 rounds "
+                       f"({groups} groups, one warp each)",
+           "ms": round(ms, 4), "groups_per_s": round(groups / (ms * 1e-3), 1),
+           "weights_GBps": round(rows * K_IN * 2 / (ms * 1e-3) / 1e9, 2),
+           "launches_per_call": 1, "reps": reps, "l2": "flushed before every call"}
+    # issue-bound fp64/integer code: achieved warp instructions per second
+    # (ncu's count per group x groups / event time) against the issue peak
+    # of 148 SMs x 4 schedulers x one warp instruction per cycle at 1965 MHz
+    rec = recorded_quantizer_insts()
+    peak = SM_COUNT * SM_SUBPARTITIONS * SM_MAX_MHZ * 1e6
+    if rec is not None:
+        ach = rec["warp_insts_per_group"] * groups / (ms * 1e-3)
+        out["roofline"] = {"bound": "alu", "achieved": round(ach / 1e9, 1), "peak": round(peak / 1e9, 1),
+                           "unit": "G warp-instructions/s", "frac": round(ach / peak, 4),
+                           "insts_per_group": rec["warp_insts_per_group"], "source": rec["source"]}
+    return out
+
+
+def run_quantizer_oracle(seed, n_groups=1024):
+    """The fp64 quantiser oracle on a sample of groups of the same weight."""
+    from oracle import quantizer as Q
+    from bit_gemv_bcq_b200 import synth
+    w16 = synth.make_weights(N_OUT, K_IN, seed=seed + 7)
+    rng = np.random.default_rng(seed + 8)
+    G = K_IN // GROUP
+    picks = rng.choice(N_OUT * G, n_groups, replace=False)
+    sub = np.stack([w16[q // G, (q % G) * GROUP:(q % G + 1) * GROUP] for q in picks])
+    t0 = time.perf_counter()
+    Q.quantize_groups(sub.astype(np.float64), 2, P_H, 20)
+    dt = time.perf_counter() - t0
+    return {"groups_per_s": round(n_groups / dt, 2), "cores": 1, "kind": "oracle",
+            "sample": f"{n_groups} random groups of the same weight ({dt:.1f} s)"}
+
+
 MMA_MIN_ROWS = 3   # bcq_gemm's default switch to the tensor-core kernel
 
 
@@ -395,6 +487,8 @@ def main():
                          "while the previous kernel drains; no kernel of the step writes them)")
     ap.add_argument("--profile", action="store_true",
                     help="GPU timing only (no e2e or CPU legs), for profiler runs")
+    ap.add_argument("--quantizer-only", type=int, default=0, metavar="ROWS",
+                    help="only time the offline quantiser on ROWS x 4096 weights (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -439,7 +533,14 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.quantizer_only:
+        torch.cuda.set_device(local_rank)
+        q = run_quantizer(args, torch.device("cuda", local_rank), rows=args.quantizer_only)
+        if rank == 0:
+            print(json.dumps({"quantizer": q}), flush=True)
+        return 0
     res = run_gpu(args, rank, world, local_rank)
+    quant = run_quantizer(args, torch.device("cuda", local_rank)) if not args.cases else None
 
     peak, peak_kind = measured_peaks()
     ms_step = res["ms_total"] / args.steps
@@ -493,7 +594,11 @@ def main():
                        "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": round(e["ms"] / e["steps"], 4),
                        "path": "bcq_gemm_host (pinned host x/y, copies on the stream)"}
+    if quant is not None:
+        line["quantizer"] = quant
     if rank == 0 and world == 1 and not args.profile:
+        if quant is not None:
+            quant["cpu_oracle"] = run_quantizer_oracle(args.seed)
         secs, by, thr = 0.0, 0.0, 1
         for k in range(max(1, args.cpu_reps)):
             s_k, b_k, thr = run_oracle_sample(args.seed + k, args.cpu_rows)

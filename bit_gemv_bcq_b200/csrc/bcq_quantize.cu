@@ -38,6 +38,11 @@ namespace {
 
 constexpr int kQuantGroup = 128;
 constexpr int kQuantWarps = 8;  // groups per CTA
+// Four CTAs (32 warps) per SM: 64 registers a thread.  The code is a chain
+// of dependent fp64 steps per group, so resident warps, not registers, set
+// the speed (measured: 3.8 ms against 4.4 ms at two CTAs per SM for a
+// 14336 x 4096 weight); the spills sit on the rare general-solve path.
+constexpr int kQuantMinBlocks = 4;
 
 struct QuantParams {
   const __half* w;       // fp16 [N][K]
@@ -72,8 +77,8 @@ __device__ __forceinline__ double signed_val(bool plus, double a) { return plus 
 
 // x_a = (adj[a][0] r_0 + adj[a][1] r_1 + ...) / det: products and sums
 // rounded one at a time, left to right (no contraction into fma).
-template <int K>
-__device__ __forceinline__ double cramer_row(const long long (&adj)[K], const double (&r)[K],
+template <int K, typename T>
+__device__ __forceinline__ double cramer_row(const T (&adj)[K], const double (&r)[K],
                                              long long det) {
   double acc = __dmul_rn((double)adj[0], r[0]);
 #pragma unroll
@@ -89,24 +94,42 @@ __device__ __forceinline__ double cramer_row(const long long (&adj)[K], const do
 // matrix by fraction-free Gauss-Jordan elimination of [G/2 | I] (left block
 // det I, right block the adjugate; every division is exact; products in
 // 128 bits), scaled back to G: adj(G) = 2^(k-1) adj(G/2), det(G) = 2^k det(G/2).
-__device__ __forceinline__ void solve_general(int M, const int* G, const double* r, double* x) {
-  long long S[5][5];
-  for (int i = 0; i < M; ++i)
-    for (int j = 0; j < M; ++j) S[i][j] = G[i * M + j] / 2;
-  int idx[5];
+template <int M>
+__device__ __forceinline__ void solve_general(const int (&G)[M][M], const double (&r)[M],
+                                              double (&x)[M]) {
+  // Local copies (static indexes only on the caller's arrays, so that they
+  // stay in registers on the fast paths); dynamic indexes below touch only
+  // these.
+  long long S[M][M];
+  int Gc[M][M];
+  double rc[M], xs[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    rc[i] = r[i];
+    xs[i] = 0.0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      Gc[i][j] = G[i][j];
+      S[i][j] = G[i][j] / 2;
+    }
+  }
+  int idx[M];
   int k = 0;
   long long prev = 1;
+#pragma unroll
   for (int c = 0; c < M; ++c) {
     if (S[c][c] == 0) continue;
     idx[k++] = c;
+#pragma unroll
     for (int i = c + 1; i < M; ++i)
+#pragma unroll
       for (int j = c + 1; j < M; ++j) S[i][j] = (S[c][c] * S[i][j] - S[i][c] * S[c][j]) / prev;
     prev = S[c][c];
   }
-  long long A[5][10];
+  long long A[M][2 * M];
   for (int a = 0; a < k; ++a)
     for (int b = 0; b < k; ++b) {
-      A[a][b] = G[idx[a] * M + idx[b]] / 2;
+      A[a][b] = Gc[idx[a]][idx[b]] / 2;
       A[a][k + b] = a == b ? 1 : 0;
     }
   prev = 1;
@@ -121,14 +144,14 @@ __device__ __forceinline__ void solve_general(int M, const int* G, const double*
     prev = p;
   }
   const long long det = prev * (1ll << k);
-  for (int j = 0; j < M; ++j) x[j] = 0.0;
+  const long long sc = 1ll << (k - 1);  // adj(G) = 2^(k-1) adj(G / 2)
   for (int a = 0; a < k; ++a) {
-    const long long sc = 1ll << (k - 1);  // adj(G) = 2^(k-1) adj(G / 2)
-    double acc = __dmul_rn((double)(A[a][k] * sc), r[idx[0]]);
-    for (int b = 1; b < k; ++b)
-      acc = __dadd_rn(acc, __dmul_rn((double)(A[a][k + b] * sc), r[idx[b]]));
-    x[idx[a]] = __ddiv_rn(acc, (double)det);
+    double acc = __dmul_rn((double)(A[a][k] * sc), rc[idx[0]]);
+    for (int b = 1; b < k; ++b) acc = __dadd_rn(acc, __dmul_rn((double)(A[a][k + b] * sc), rc[idx[b]]));
+    xs[idx[a]] = __ddiv_rn(acc, (double)det);
   }
+#pragma unroll
+  for (int j = 0; j < M; ++j) x[j] = xs[j];
 }
 
 // Least squares on M columns with integer Gram matrix G and right-hand
@@ -142,9 +165,9 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
     x[0] = __ddiv_rn(r[0], (double)G[0][0]);  // adj = [1]; G[0][0] = 128
     return;
   } else if constexpr (M == 2) {
-    const long long det = (long long)G[0][0] * G[1][1] - (long long)G[0][1] * G[1][0];
+    const int det = G[0][0] * G[1][1] - G[0][1] * G[1][0];
     if (det != 0) {
-      const long long a0[2] = {G[1][1], -G[0][1]}, a1[2] = {-G[1][0], G[0][0]};
+      const int a0[2] = {G[1][1], -G[0][1]}, a1[2] = {-G[1][0], G[0][0]};
       x[0] = cramer_row<2>(a0, r, det);
       x[1] = cramer_row<2>(a1, r, det);
       return;
@@ -152,12 +175,13 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
   } else if constexpr (M == 3) {
     const int g00 = G[0][0], g01 = G[0][1], g02 = G[0][2], g11 = G[1][1], g12 = G[1][2],
               g22 = G[2][2];
-    const long long c00 = g11 * g22 - g12 * g12, c01 = g02 * g12 - g01 * g22,
-                    c02 = g01 * g12 - g02 * g11, c11 = g00 * g22 - g02 * g02,
-                    c12 = g01 * g02 - g00 * g12, c22 = g00 * g11 - g01 * g01;
-    const long long det = g00 * c00 + g01 * c01 + g02 * c02;
+    // |G| <= 128: cofactors below 2^15, the determinant below 2^24
+    const int c00 = g11 * g22 - g12 * g12, c01 = g02 * g12 - g01 * g22,
+              c02 = g01 * g12 - g02 * g11, c11 = g00 * g22 - g02 * g02,
+              c12 = g01 * g02 - g00 * g12, c22 = g00 * g11 - g01 * g01;
+    const int det = g00 * c00 + g01 * c01 + g02 * c02;
     if (c22 != 0 && det != 0) {  // leading minors: g00 = 128, c22, det
-      const long long a0[3] = {c00, c01, c02}, a1[3] = {c01, c11, c12}, a2[3] = {c02, c12, c22};
+      const int a0[3] = {c00, c01, c02}, a1[3] = {c01, c11, c12}, a2[3] = {c02, c12, c22};
       x[0] = cramer_row<3>(a0, r, det);
       x[1] = cramer_row<3>(a1, r, det);
       x[2] = cramer_row<3>(a2, r, det);
@@ -165,25 +189,28 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
     }
   } else if constexpr (M == 4) {
     // Laplace expansion by the 2x2 minors of rows 0-1 (s) and rows 2-3 (c)
-    const long long a00 = G[0][0], a01 = G[0][1], a02 = G[0][2], a03 = G[0][3];
-    const long long a11 = G[1][1], a12 = G[1][2], a13 = G[1][3];
-    const long long a22 = G[2][2], a23 = G[2][3], a33 = G[3][3];
-    const long long a10 = a01, a20 = a02, a21 = a12, a30 = a03, a31 = a13, a32 = a23;
-    const long long s0 = a00 * a11 - a10 * a01, s1 = a00 * a12 - a10 * a02,
-                    s2 = a00 * a13 - a10 * a03, s3 = a01 * a12 - a11 * a02,
-                    s4 = a01 * a13 - a11 * a03, s5 = a02 * a13 - a12 * a03;
-    const long long c5 = a22 * a33 - a32 * a23, c4 = a21 * a33 - a31 * a23,
-                    c3 = a21 * a32 - a31 * a22, c2 = a20 * a33 - a30 * a23,
-                    c1 = a20 * a32 - a30 * a22, c0 = a20 * a31 - a30 * a21;
-    const long long det = s0 * c5 - s1 * c4 + s2 * c3 + s3 * c2 - s4 * c1 + s5 * c0;
-    const long long b00 = a11 * c5 - a12 * c4 + a13 * c3, b01 = -a01 * c5 + a02 * c4 - a03 * c3,
-                    b02 = a31 * s5 - a32 * s4 + a33 * s3, b03 = -a21 * s5 + a22 * s4 - a23 * s3,
-                    b11 = a00 * c5 - a02 * c2 + a03 * c1, b12 = -a30 * s5 + a32 * s2 - a33 * s1,
-                    b13 = a20 * s5 - a22 * s2 + a23 * s1, b22 = a30 * s4 - a31 * s2 + a33 * s0,
-                    b23 = -a20 * s4 + a21 * s2 - a23 * s0, b33 = a20 * s3 - a21 * s1 + a22 * s0;
+    // |G| <= 128: 2x2 minors below 2^15, adjugate entries (3x3 minors)
+    // below 2^24, the determinant below 2^33 (64-bit)
+    const int a00 = G[0][0], a01 = G[0][1], a02 = G[0][2], a03 = G[0][3];
+    const int a11 = G[1][1], a12 = G[1][2], a13 = G[1][3];
+    const int a22 = G[2][2], a23 = G[2][3], a33 = G[3][3];
+    const int a10 = a01, a20 = a02, a21 = a12, a30 = a03, a31 = a13, a32 = a23;
+    const int s0 = a00 * a11 - a10 * a01, s1 = a00 * a12 - a10 * a02,
+              s2 = a00 * a13 - a10 * a03, s3 = a01 * a12 - a11 * a02,
+              s4 = a01 * a13 - a11 * a03, s5 = a02 * a13 - a12 * a03;
+    const int c5 = a22 * a33 - a32 * a23, c4 = a21 * a33 - a31 * a23,
+              c3 = a21 * a32 - a31 * a22, c2 = a20 * a33 - a30 * a23,
+              c1 = a20 * a32 - a30 * a22, c0 = a20 * a31 - a30 * a21;
+    const long long det = (long long)s0 * c5 - (long long)s1 * c4 + (long long)s2 * c3 +
+                          (long long)s3 * c2 - (long long)s4 * c1 + (long long)s5 * c0;
+    const int b00 = a11 * c5 - a12 * c4 + a13 * c3, b01 = -a01 * c5 + a02 * c4 - a03 * c3,
+              b02 = a31 * s5 - a32 * s4 + a33 * s3, b03 = -a21 * s5 + a22 * s4 - a23 * s3,
+              b11 = a00 * c5 - a02 * c2 + a03 * c1, b12 = -a30 * s5 + a32 * s2 - a33 * s1,
+              b13 = a20 * s5 - a22 * s2 + a23 * s1, b22 = a30 * s4 - a31 * s2 + a33 * s0,
+              b23 = -a20 * s4 + a21 * s2 - a23 * s0, b33 = a20 * s3 - a21 * s1 + a22 * s0;
     if (s0 != 0 && b33 != 0 && det != 0) {  // leading minors: a00, s0, b33 (= 3x3), det
-      const long long r0[4] = {b00, b01, b02, b03}, r1[4] = {b01, b11, b12, b13},
-                      r2[4] = {b02, b12, b22, b23}, r3[4] = {b03, b13, b23, b33};
+      const int r0[4] = {b00, b01, b02, b03}, r1[4] = {b01, b11, b12, b13},
+                r2[4] = {b02, b12, b22, b23}, r3[4] = {b03, b13, b23, b33};
       x[0] = cramer_row<4>(r0, r, det);
       x[1] = cramer_row<4>(r1, r, det);
       x[2] = cramer_row<4>(r2, r, det);
@@ -191,7 +218,7 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
       return;
     }
   }
-  if constexpr (M >= 2) solve_general(M, &G[0][0], r, x);
+  if constexpr (M >= 2) solve_general<M>(G, r, x);
 }
 
 // Ballot words of the first P planes: P[i][s] = plane i, columns 32 s..32 s + 31.
@@ -385,7 +412,7 @@ __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int 
 }
 
 template <int PL, int PH>
-__global__ void __launch_bounds__(32 * kQuantWarps) quantize_kernel(QuantParams q) {
+__global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinBlocks) quantize_kernel(QuantParams q) {
   const int lane = threadIdx.x & 31;
   const long long gid = (long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
   if (gid >= q.groups) return;  // uniform per warp

@@ -123,7 +123,7 @@ bcq_status bcq_pack_scales(const uint16_t* src, int q, int N, int K,
  * Bytes of workspace bcq_gemm needs for M rows of x and an N x K weight: 0
  * when K <= 256 (no split over K), else room for the arrival counters of the
  * row-blocks and the fp32 partial sums of every (256-column K-block, row) for
- * the rows of one launch (min(M, 16)).  0 for invalid shapes as well.
+ * the rows of the largest launch (min(M, 64)).  0 for invalid shapes as well.
  */
 size_t bcq_workspace_bytes(int M, int N, int K);
 
@@ -170,10 +170,11 @@ bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes,
                     void* stream);
 
 /*
- * The launch plan bcq_gemm would use for one launch of M (1..16) activation
+ * The launch plan bcq_gemm would use for one launch of M (1..64) activation
  * rows streaming p_load planes (mixed = 1: two rows of different
- * precisions).  M <= 2 plans the lookup-table kernel, M >= 3 the tensor-core
- * kernel that bcq_gemm would use for a batch (BCQ_MMA_KIND).  use_device = 1
+ * precisions).  M <= 2 plans the lookup-table kernel, 3 <= M <= 16 the
+ * tensor-core kernel that bcq_gemm would use for a batch (BCQ_MMA_KIND), and
+ * M >= 17 the 64-row tcgen05 launch.  use_device = 1
  * plans for the current device; 0 (or no usable device) plans for a nominal
  * 148-SM B200 without touching CUDA.  out[8] receives: CTAs, consumer warps,
  * producer warps, ring stages, dynamic shared memory bytes, bytes per ring

@@ -47,16 +47,14 @@ bool shape_ok(int N, int K) {
 
 size_t row_blocks(int N) { return ((size_t)N + kRowBlock - 1) / kRowBlock; }
 size_t k_blocks(int K) { return ((size_t)K + kKBlock - 1) / kKBlock; }
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Workspace: arrival counters [RB] (256-byte aligned), then fp32 partial
-// sums [KB][min(M, 64)][RB * 32] (the rows of the largest launch).
-size_t counter_bytes(int N) { return align256(row_blocks(N) * sizeof(unsigned int)); }
+// Workspace: the tagged fp32 partial sums [KB][min(M, 64)][RB * 32] (the
+// rows of the largest launch); zero = not written yet.
 size_t workspace_bytes(int M, int N, int K) {
   const size_t KB = k_blocks(K);
   if (M < 1 || KB <= 1) return 0;
   const size_t ml = (size_t)std::min(M, kMaxLaunchRows);
-  return counter_bytes(N) + KB * ml * row_blocks(N) * kRowBlock * sizeof(float);
+  return KB * ml * row_blocks(N) * kRowBlock * sizeof(float);
 }
 
 // Per-device facts, cached after the first query (callers hold g_mu).
@@ -247,9 +245,7 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const ui
   const int KB = (int)k_blocks(K);
   g.planes = planes;
   g.z = z;
-  g.cnt = KB > 1 ? static_cast<unsigned int*>(ws) : nullptr;
-  g.part = KB > 1 ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + counter_bytes(N))
-                  : nullptr;
+  g.part = KB > 1 ? static_cast<float*>(ws) : nullptr;
   g.N = N;
   g.K = K;
   g.KB = KB;

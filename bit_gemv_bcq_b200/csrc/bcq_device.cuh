@@ -103,45 +103,26 @@ __device__ __forceinline__ uint16_t ldg_nc_u16(const void* p) {
   return v;
 }
 
-// Global load cached in L2 only: data other CTAs wrote during this launch.
-__device__ __forceinline__ float ldg_cg_f32(const float* p) {
-  float v;
-  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ void stg_cg_zero(float* p) {
   asm volatile("st.global.cg.f32 [%0], %1;" ::"l"(p), "f"(0.f) : "memory");
 }
 
-// Arrival counter increment, release at GPU scope (no value returned).
-__device__ __forceinline__ void red_add_release(unsigned int* p, unsigned int v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Split-K partial sums travel as the complement of their fp32 bits, so a
+// zero word means "not written yet": the complement of a value is zero only
+// for the bit pattern 0xFFFFFFFF, a NaN that fp32 arithmetic never returns
+// (its NaN results are the canonical 0x7FFFFFFF).  Relaxed GPU-scope stores
+// and loads: each partial is one single-copy-atomic 32-bit word, read by
+// another CTA while the kernel runs.
+__device__ __forceinline__ void st_partial(float* p, float v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(~__float_as_uint(v))
+               : "memory");
 }
-
-__device__ __forceinline__ void red_add_relaxed(unsigned int* p, unsigned int v) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Release fence at GPU scope: with a CTA barrier before it, orders every
-// thread's earlier writes before this thread's later relaxed atomics.
-__device__ __forceinline__ void fence_acq_rel_gpu() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
-
-__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint32_t ld_partial_tag(const float* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-
-// Arrival counter increment with acquire-release semantics at GPU scope.
-__device__ __forceinline__ unsigned int atom_add_acq_rel(unsigned int* p, unsigned int v) {
-  unsigned int old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
+__device__ __forceinline__ float partial_value(uint32_t tag) { return __uint_as_float(~tag); }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -190,23 +171,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
-}
-
-// Waits until *cnt >= target (acquire), for at most limit_ns of
-// %globaltimer, giving up early when the CTA aborts.  Returns false if it
-// gave up.
-__device__ __forceinline__ bool wait_count(const unsigned int* cnt, unsigned int target,
-                                           volatile int* abort_flag,
-                                           unsigned long long limit_ns) {
-  if (ld_acquire_u32(cnt) >= target) return true;
-  const unsigned long long t0 = globaltimer_ns();
-#pragma unroll 1
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire_u32(cnt) >= target) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
 }
 
 // Non-blocking test: has phase `parity` of the barrier completed?

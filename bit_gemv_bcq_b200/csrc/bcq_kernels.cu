@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     if (prm.KB > 1) {
 #pragma unroll
       for (int m = 0; m < M; ++m)
-        prm.part[((size_t)pend_kb[J] * M + m) * part_stride + (size_t)row] = r[m];
+        st_partial(prm.part + ((size_t)pend_kb[J] * M + m) * part_stride + (size_t)row, r[m]);
     } else if (row < prm.N) {
 #pragma unroll
       for (int m = 0; m < M; ++m) prm.y[(size_t)m * prm.N + row] = f2h_rn(r[m]);
@@ -605,9 +605,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   advance_tables(R.kb_last);  // the same barriers in both teams
 
   // split-K reduction (a no-op when the launch has one K-block)
+  // (no barrier: a warp starts its reduction tasks as soon as it is done;
+  // the partials it waits for are polled, not counted)
   if (prm.KB > 1) {
-    named_barrier_sync(1, kConsumers);  // every partial of the CTA is stored
-    splitk_tail(prm, R, M, nullptr, tid, kConsumers, abort_flag);
+    splitk_tail<M == 1 ? 16 : 8>(prm, R, M, nullptr, tid, kConsumers, abort_flag);
   }
 }
 

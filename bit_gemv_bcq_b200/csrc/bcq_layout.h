@@ -170,8 +170,7 @@ struct GemvParams {
   const uint16_t* alpha[2];  // packed scales of row 0 and row 1 (q[m] per entry)
   const uint16_t* z;         // packed offsets, or nullptr
   uint16_t* y;               // fp16 [M][N] (rows of this launch)
-  float* part;               // fp32 partial sums [KB][M][RB * 32] (KB > 1)
-  unsigned int* cnt;         // arrival counters [RB] (KB > 1), zero between calls
+  float* part;               // tagged fp32 partial sums [KB][M][RB * 32] (KB > 1), zero between calls
   int M, N, K, KB, RB, RG, p_H;
   int q[2];                  // precision of each row (<= planes streamed)
   int U;                     // units (< 2^31)

@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
               v = fmaf(zz[0], sg[nt][c][0], fmaf(zz[1], sg[nt][c][1], v));
               if (m < prm.M) {
                 if (prm.KB > 1)
-                  prm.part[((size_t)gc.kb * prm.M + m) * part_stride + (size_t)row] = v;
+                  st_partial(prm.part + ((size_t)gc.kb * prm.M + m) * part_stride + (size_t)row, v);
                 else if (row < prm.N)
                   prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(v);
               }
@@ -403,9 +403,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   cp_async_wait<0>();
   advance_tiles(R.kb_last);  // the same barriers in both teams
 
+  // (no barrier: a warp starts its reduction tasks as soon as it is done;
+  // the partials it waits for are polled, not counted)
   if (prm.KB > 1) {
-    named_barrier_sync(1, kConsumers);  // every partial of the CTA is stored
-    splitk_tail(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
+    splitk_tail<8>(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
   }
 }
 

@@ -136,19 +136,21 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
   __syncwarp();
 }
 
-// Split-K reduction, run by all nthreads consumer threads of the CTA after
-// a barrier that follows their partial-sum stores.  Every unit's fp32
-// partials [kb][m][row] are in the workspace.  Each CTA counts its arrivals
-// (fence, then release), then reduces the row-blocks it is designated for --
-// row-block rb belongs to the CTA that computed its unit in K-block rb mod KB,
-// so the work is spread evenly whatever the order in which CTAs finish.  The
-// (row-block, two launch rows) tasks of the CTA are dealt to its warps in
-// turn; a warp waits (bounded) until all KB partials of its row-block have
-// arrived, loads them all at once, adds them in K-block order (the result does not
-// depend on scheduling), writes y (row m of the launch goes to y row ymap[m],
-// or m without a map) and clears those partials.  After a barrier the CTA
-// clears its row-blocks' counters, so the whole workspace is zero again for
-// the next call, whatever its shape.
+// Split-K reduction, run by each of the CTA's nthreads consumer threads once
+// its warp has stored its own partial sums (no barrier).  Every unit's fp32
+// partials [kb][m][row] go to the workspace as tagged words (st_partial: zero
+// = not written yet), so no fence or arrival counter is needed: a reducer
+// polls the partials themselves.  Row-block rb is reduced by the CTA that
+// computed its unit in K-block rb mod KB, so the work is spread evenly
+// whatever the order in which CTAs finish.  The (row-block, two launch rows)
+// tasks of the CTA are dealt to its warps in turn; a warp loads all KB
+// partials of its task at once, re-loads (bounded) those still zero, adds
+// them in K-block order (the result does not depend on scheduling), writes y
+// (row m of the launch goes to y row ymap[m], or m without a map) and zeroes
+// those partials, so the workspace is zero again for the next call.  kC
+// K-blocks of partials are loaded at once (one round trip each): 16 where
+// registers allow (the lookup kernel), 8 in the tensor-core kernels.
+template <int kC>
 __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRange& R, int Mrows,
                                             const int* ymap, int tid, int nthreads,
                                             volatile int* abort_flag) {
@@ -157,17 +159,6 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
   const size_t part_stride = (size_t)RB * kRowBlock;
   const size_t kstride = (size_t)Mrows * part_stride;  // one K-block of partials
   const bool live = *abort_flag == 0;
-  if (warp == 0 && live) {
-    // one warp: a release fence in each lane, cumulative over the barrier
-    // before this call (every partial of the CTA), then that lane's arrivals
-    // as relaxed atomics
-    fence_acq_rel_gpu();
-    for (int kb = R.kb0; kb <= R.kb_last; ++kb) {
-      const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
-      const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
-      for (int rb = a + lane; rb < b; rb += 32) red_add_relaxed(prm.cnt + rb, 1u);
-    }
-  }
   int task = 0, mine = warp;  // tasks dealt round-robin: no division
   for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
     const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
@@ -178,35 +169,60 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
       for (int m0 = 0; m0 < Mrows; m0 += 2, ++task) {  // two launch rows per task
         if (task != mine) continue;
         mine += nwarps;
-        bool ready = true;
-        if (lane == 0)
-          ready = wait_count(prm.cnt + rbx, (unsigned int)KB, abort_flag, prm.timeout_ns);
-        ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
-        if (!ready) {
+        const int row = rbx * kRowBlock + lane;
+        const int nm = Mrows - m0 < 2 ? Mrows - m0 : 2;
+        float* pp = prm.part + (size_t)m0 * part_stride + (size_t)row;
+        float sum[2] = {0.f, 0.f};
+        bool ok = true;
+        for (int k0 = 0; k0 < KB && ok; k0 += kC) {
+          uint32_t v[2][kC];  // every load of the chunk in flight at once
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int j = 0; j < kC; ++j)
+              v[mm][j] = mm < nm && k0 + j < KB
+                             ? ld_partial_tag(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride)
+                             : 1u;
+          bool have = true;
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int j = 0; j < kC; ++j) have = have && v[mm][j] != 0u;
+          if (!__all_sync(0xFFFFFFFFu, have)) {
+            // some partials are still on their way: re-load the missing ones
+            const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+            while (true) {
+              __nanosleep(32);
+              have = true;
+#pragma unroll
+              for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+                for (int j = 0; j < kC; ++j) {
+                  if (v[mm][j] == 0u)
+                    v[mm][j] = ld_partial_tag(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride);
+                  have = have && v[mm][j] != 0u;
+                }
+              if (__all_sync(0xFFFFFFFFu, have)) break;
+              if (*abort_flag || globaltimer_ns() - t0 > prm.timeout_ns) {
+                ok = false;
+                break;
+              }
+            }
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int j = 0; j < kC; ++j)
+              if (k0 + j < KB) sum[mm] += partial_value(v[mm][j]);
+        }
+        if (!ok) {
           if (lane == 0 && *abort_flag == 0) {
             record_error(&g_device_error, BCQ_ERR_TIMEOUT);
             *abort_flag = 1;
           }
           continue;
-        }
-        const int row = rbx * kRowBlock + lane;
-        const int nm = Mrows - m0 < 2 ? Mrows - m0 : 2;
-        float* pp = prm.part + (size_t)m0 * part_stride + (size_t)row;
-        float sum[2] = {0.f, 0.f};
-        for (int k0 = 0; k0 < KB; k0 += 16) {
-          float v[2][16];  // every load of the task in flight at once
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              v[mm][j] = mm < nm && k0 + j < KB
-                             ? ldg_cg_f32(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride)
-                             : 0.f;
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (k0 + j < KB) sum[mm] += v[mm][j];
         }
         for (int mm = 0; mm < nm; ++mm) {
           const int ym = ymap ? ymap[m0 + mm] : m0 + mm;
@@ -217,16 +233,6 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
         }
       }
     }
-  }
-  // every task's wait is over: clear the designated counters
-  named_barrier_sync(1, nthreads);
-  for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
-    const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
-    const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
-    int first = kb;
-    if (first < a) first += (a - first + KB - 1) / KB * KB;
-    for (int rbx = first + tid * KB; rbx < b; rbx += nthreads * KB)
-      *reinterpret_cast<volatile unsigned int*>(prm.cnt + rbx) = 0u;
   }
 }
 

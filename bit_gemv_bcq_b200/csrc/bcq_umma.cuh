@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
             const float sB = lds_f32_dyn(gsl + (uint32_t)(m * 2 + 1) * 4u);
             const float v = fmaf(p_z0, sA, fmaf(p_z1, sB, __uint_as_float(d[e])));
             if (prm.KB > 1)
-              prm.part[((size_t)p_kb * prm.M + m) * part_stride + (size_t)p_row] = v;
+              st_partial(prm.part + ((size_t)p_kb * prm.M + m) * part_stride + (size_t)p_row, v);
             else if (p_row < prm.N)
               prm.y[(size_t)prm.rows[m] * prm.N + p_row] = f2h_rn(v);
           }
@@ -541,9 +541,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     umma_fence_after();
     tmem_dealloc(tmem, kUmmaTmemCols);
   }
+  // (no barrier: a warp starts its reduction tasks as soon as it is done;
+  // the partials it waits for are polled, not counted)
   if (prm.KB > 1) {
-    named_barrier_sync(1, kConsumers);
-    splitk_tail(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
+    splitk_tail<4>(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
   }
 }
 

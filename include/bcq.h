@@ -121,9 +121,11 @@ bcq_status bcq_pack_scales(const uint16_t* src, int q, int N, int K,
 
 /*
  * Bytes of workspace bcq_gemm needs for M rows of x and an N x K weight: 0
- * when K <= 256 (no split over K), else room for the arrival counters of the
- * row-blocks and the fp32 partial sums of every (256-column K-block, row) for
- * the rows of the largest launch (min(M, 64)).  0 for invalid shapes as well.
+ * when K <= 256 (no split over K), else room for the fp32 partial sums of
+ * every (256-column K-block, row) for the rows of the largest launch
+ * (min(M, 64)), rows padded to a multiple of 32:
+ * ceil(K / 256) * min(M, 64) * ceil(N / 32) * 32 * 4 bytes.  0 for invalid
+ * shapes as well.
  */
 size_t bcq_workspace_bytes(int M, int N, int K);
 

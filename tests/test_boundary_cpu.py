@@ -59,12 +59,12 @@ def test_workspace_bytes_formula(L):
     # one K-block: no split over K, no workspace
     assert api.workspace_bytes(1, 4096, 256) == 0
     assert api.workspace_bytes(4, 4096, 128) == 0
-    # counters (row-blocks x 4 B, rounded to 256 B) + KB x min(M, 64) x rows x 4 B
-    assert api.workspace_bytes(1, 14336, 4096) == 1792 + 16 * 1 * 14336 * 4
-    assert api.workspace_bytes(8, 14336, 4096) == 1792 + 16 * 8 * 14336 * 4
-    assert api.workspace_bytes(64, 14336, 4096) == 1792 + 16 * 64 * 14336 * 4
-    assert api.workspace_bytes(17, 14336, 4096) == 1792 + 16 * 17 * 14336 * 4
-    assert api.workspace_bytes(2, 33, 640) == 256 + 3 * 2 * 64 * 4
+    # KB x min(M, 64) x rows (padded to 32) x 4 B of tagged partial sums
+    assert api.workspace_bytes(1, 14336, 4096) == 16 * 1 * 14336 * 4
+    assert api.workspace_bytes(8, 14336, 4096) == 16 * 8 * 14336 * 4
+    assert api.workspace_bytes(64, 14336, 4096) == 16 * 64 * 14336 * 4
+    assert api.workspace_bytes(17, 14336, 4096) == 16 * 17 * 14336 * 4
+    assert api.workspace_bytes(2, 33, 640) == 3 * 2 * 64 * 4
     assert api.workspace_bytes(0, 64, 512) == 0
     assert api.workspace_bytes(1, 64, 100) == 0
 

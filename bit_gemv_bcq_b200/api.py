@@ -81,6 +81,8 @@ def lib():
         L.bcq_gemm.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, S, P]
         L.bcq_gemm_host.restype = I
         L.bcq_gemm_host.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, P, P, S, P]
+        L.bcq_gemm_zp.restype = I
+        L.bcq_gemm_zp.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P, S, P]
         L.bcq_gemm_noalloc.restype = I
         L.bcq_gemm_noalloc.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
         L.bcq_build_lut.restype = I
@@ -99,7 +101,7 @@ EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
             "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl",
             "bcq_gemm_host", "bcq_gemm_noalloc", "bcq_build_lut", "bcq_device_error",
-            "bcq_debug_wait_timeout", "bcq_quantize")
+            "bcq_debug_wait_timeout", "bcq_quantize", "bcq_gemm_zp")
 
 
 def status_string(status: int) -> str:
@@ -129,12 +131,12 @@ def _need_cuda(t: torch.Tensor, name: str, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
-def _alpha_array(alphas: dict):
+def _alpha_array(alphas: dict, what: str = "alpha"):
     arr = (ctypes.c_void_p * 4)()
     for q in range(1, 5):
         a = alphas.get(q) if alphas else None
         if a is not None:
-            _need_cuda(a, f"alpha[{q}]", torch.float16)
+            _need_cuda(a, f"{what}[{q}]", torch.float16)
             arr[q - 1] = a.data_ptr()
         else:
             arr[q - 1] = None
@@ -268,11 +270,13 @@ class BcqWeights:
     K: int
     p_H: int
     row_splits: tuple = ()      # rows of each stacked matrix (see stack), else ()
+    zq: dict | None = None      # {q: packed offsets z^(q)} when every precision has its own
 
     @classmethod
     def from_canonical(cls, planes, alphas: dict, z=None, device="cuda", stream=None):
         """planes: uint32 [p_H][N][K/32] (numpy or tensor); alphas {q: fp16
-        [N][G][q]}; z fp16 [N][G] or None."""
+        [N][G][q]}; z fp16 [N][G], or {q: fp16 [N][G]} (offsets per precision,
+        used through bcq_gemm_zp), or None."""
         if isinstance(planes, np.ndarray):
             planes = torch.from_numpy(np.ascontiguousarray(planes).view(np.int32))
         planes = planes.to(device).contiguous()
@@ -283,10 +287,14 @@ class BcqWeights:
             a = torch.as_tensor(a) if isinstance(a, np.ndarray) else a
             al[int(q)] = pack_scales(a.to(device=device, dtype=torch.float16).contiguous(),
                                      int(q), stream)
-        zz = None
-        if z is not None:
-            zz = (torch.as_tensor(z) if isinstance(z, np.ndarray) else z)
-            zz = pack_scales(zz.to(device=device, dtype=torch.float16).contiguous(), 1, stream)
+        def pack_z(zv):
+            zv = torch.as_tensor(zv) if isinstance(zv, np.ndarray) else zv
+            return pack_scales(zv.to(device=device, dtype=torch.float16).contiguous(), 1, stream)
+
+        if isinstance(z, dict):
+            zq = {int(q): pack_z(zv) for q, zv in z.items() if zv is not None}
+            return cls(packed=packed, alphas=al, z=None, N=N, K=KW * 32, p_H=p_H, zq=zq)
+        zz = None if z is None else pack_z(z)
         return cls(packed=packed, alphas=al, z=zz, N=N, K=KW * 32, p_H=p_H)
 
     @classmethod
@@ -372,11 +380,19 @@ def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
         _need_cuda(out, "out", torch.float16)
     alpha = _alpha_array(w.alphas)
     ws = workspace(M, w.N, w.K, x.device, stream)
-    st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                        _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                        _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
-                        _stream(stream))
-    _check(st, "bcq_gemm")
+    if w.zq is not None:
+        zarr = _alpha_array(w.zq, "z")   # 4 device pointers or NULL
+        st = lib().bcq_gemm_zp(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                               ctypes.cast(zarr, ctypes.c_void_p), pv, pr_ptr, M, w.N, w.K,
+                               w.p_H, GROUP, _ptr(out), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream))
+        _check(st, "bcq_gemm_zp")
+    else:
+        st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                            _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                            _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                            _stream(stream))
+        _check(st, "bcq_gemm")
     del pr_keep
     return out
 
@@ -389,6 +405,8 @@ def gemm_noalloc(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=Non
     race; shapes needing more than NOALLOC_SCRATCH_BYTES raise
     BcqError(BCQ_ERR_SCRATCH).  `out` should be given by such callers (the
     binding allocates it otherwise)."""
+    if w.zq is not None:
+        raise ValueError("per-precision offsets: use gemm (bcq_gemm_zp)")
     _need_cuda(x, "x", torch.float16)
     if x.dim() != 2 or x.shape[1] != w.K:
         raise ValueError(f"x must be [M][{w.K}]")
@@ -412,6 +430,8 @@ def gemm_host(x_host: torch.Tensor, w: BcqWeights, y_host: torch.Tensor,
               p_row=None, stream=None) -> None:
     """bcq_gemm_host: x and y in (pinned) host memory, copies on the stream.
     The caller synchronises the stream before reading y_host."""
+    if w.zq is not None:
+        raise ValueError("per-precision offsets: use gemm (bcq_gemm_zp)")
     if x_host.is_cuda or y_host.is_cuda:
         raise ValueError("x_host and y_host must be host tensors")
     M = x_host.shape[0]

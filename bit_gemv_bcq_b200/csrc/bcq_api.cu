@@ -169,7 +169,7 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
 }
 
 bcq_status validate_gemm(const uint16_t* x, const uint32_t* planes,
-                         const uint16_t* const alpha[4], const uint16_t* z, int p,
+                         const uint16_t* const alpha[4], const uint16_t* const zq[4], int p,
                          const int32_t* p_row, int M, int N, int K, int p_H, int group,
                          const uint16_t* y, const void* ws, size_t ws_bytes) {
   if (!alpha) return BCQ_ERR_NULL;
@@ -193,7 +193,8 @@ bcq_status validate_gemm(const uint16_t* x, const uint32_t* planes,
   }
   if (M > 0) {
     if (!aligned(x, 16) || !aligned(planes, 16) || !aligned(y, 2)) return BCQ_ERR_ALIGN;
-    if (z && !aligned(z, 16)) return BCQ_ERR_ALIGN;
+    for (int q = 1; q <= 4; ++q)
+      if (used[q] && zq[q - 1] && !aligned(zq[q - 1], 16)) return BCQ_ERR_ALIGN;
     const size_t need = workspace_bytes(M, N, K);
     if (need > 0) {
       if (!ws || ws_bytes < need) return BCQ_ERR_NULL;
@@ -239,12 +240,11 @@ void plan_units(int RB, int KB, int C, CtaWork* work) {
 }
 
 // Fills the fields every launch shares.
-void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const uint16_t* z,
+void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes,
                  int N, int K, int p_H, void* ws, int pdl_mode, int wait_us) {
   const int RB = (int)row_blocks(N);
   const int KB = (int)k_blocks(K);
   g.planes = planes;
-  g.z = z;
   g.part = KB > 1 ? static_cast<float*>(ws) : nullptr;
   g.N = N;
   g.K = K;
@@ -271,7 +271,7 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, const ui
 // remainder of at least BCQ_MMA_MIN_ROWS rows, else a lookup launch per
 // remaining row.
 bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
-                    const uint16_t* z, int p, const int32_t* p_row, int M, int N, int K,
+                    const uint16_t* const zq[4], int p, const int32_t* p_row, int M, int N, int K,
                     int p_H, uint16_t* y, void* ws, cudaStream_t st) {
   const int pdl_mode = g_pdl_mode.load();
   const int wait_us = env_int("BCQ_WAIT_LIMIT_US", 0);
@@ -300,8 +300,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
         bcq_status s = plan_gemv(cnt, N, K, q, false, qpath, &pl);
         if (s != BCQ_OK) return s;
         GemvParams g{};
-        fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
+        fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);
         g.alpha[0] = g.alpha[1] = alpha[q - 1];
+        g.z = g.z1 = zq[q - 1];
         g.M = cnt;
         g.q[0] = g.q[1] = q;
         if (qpath == kPathLut) {  // one row, addressed directly
@@ -329,7 +330,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
     bcq_status s = plan_gemv(rows, N, K, P, mixed, kPathLut, &pl);
     if (s != BCQ_OK) return s;
     GemvParams g{};
-    fill_common(g, pl, planes, z, N, K, p_H, ws, pdl_mode, wait_us);
+    fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);
+    g.z = zq[q[0] - 1];
+    g.z1 = zq[q[1] - 1];
     g.x = x + (size_t)m0 * K;
     g.y = y + (size_t)m0 * N;
     g.alpha[0] = alpha[q[0] - 1];
@@ -348,7 +351,8 @@ bcq_status check_gemm_args(const uint16_t* x, const uint32_t* planes,
                            const uint16_t* const alpha[4], const uint16_t* z, int p,
                            const int32_t* p_row, int M, int N, int K, int p_H, int group,
                            const uint16_t* y, const void* ws, size_t ws_bytes) {
-  return validate_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, group, y, ws, ws_bytes);
+  const uint16_t* const zq[4] = {z, z, z, z};
+  return validate_gemm(x, planes, alpha, zq, p, p_row, M, N, K, p_H, group, y, ws, ws_bytes);
 }
 
 }  // namespace bcq
@@ -447,11 +451,22 @@ bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
                     const uint16_t* z, int p, const int32_t* p_row, int M, int N, int K,
                     int p_H, int group, uint16_t* y, void* workspace, size_t workspace_bytes,
                     void* stream) {
-  bcq_status s = validate_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, group, y, workspace,
+  const uint16_t* const zq[4] = {z, z, z, z};
+  return bcq_gemm_zp(x, planes, alpha, zq, p, p_row, M, N, K, p_H, group, y, workspace,
+                     workspace_bytes, stream);
+}
+
+bcq_status bcq_gemm_zp(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
+                       const uint16_t* const z[4], int p, const int32_t* p_row, int M, int N,
+                       int K, int p_H, int group, uint16_t* y, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  static const uint16_t* const kNoOffsets[4] = {nullptr, nullptr, nullptr, nullptr};
+  const uint16_t* const* zq = z ? z : kNoOffsets;
+  bcq_status s = validate_gemm(x, planes, alpha, zq, p, p_row, M, N, K, p_H, group, y, workspace,
                                workspace_bytes);
   if (s != BCQ_OK || M == 0) return s;
   std::lock_guard<std::mutex> lock(g_mu);
-  return run_gemm(x, planes, alpha, z, p, p_row, M, N, K, p_H, y, workspace,
+  return run_gemm(x, planes, alpha, zq, p, p_row, M, N, K, p_H, y, workspace,
                   (cudaStream_t)stream);
 }
 
@@ -461,7 +476,8 @@ bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
                          uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev, void* workspace,
                          size_t workspace_bytes, void* stream) {
   if (M > 0 && (!x_host || !y_host)) return BCQ_ERR_NULL;
-  bcq_status s = validate_gemm(x_dev, planes, alpha, z, p, p_row, M, N, K, p_H, group, y_dev,
+  const uint16_t* const zq[4] = {z, z, z, z};
+  bcq_status s = validate_gemm(x_dev, planes, alpha, zq, p, p_row, M, N, K, p_H, group, y_dev,
                                workspace, workspace_bytes);
   if (s != BCQ_OK || M == 0) return s;
   cudaStream_t st = (cudaStream_t)stream;
@@ -469,7 +485,7 @@ bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
     return BCQ_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    s = run_gemm(x_dev, planes, alpha, z, p, p_row, M, N, K, p_H, y_dev, workspace, st);
+    s = run_gemm(x_dev, planes, alpha, zq, p, p_row, M, N, K, p_H, y_dev, workspace, st);
   }
   if (s != BCQ_OK) return s;
   if (cudaMemcpyAsync(y_host, y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess)

@@ -277,11 +277,12 @@ __device__ __forceinline__ void plane_sum2(const uint4& w, const uint32_t (&cr)[
 
 // Scales and offsets of one unit for this lane: a[m][r] holds halves
 // 2r, 2r + 1 of the lane's 2P values (pass 0: planes 0..P-1, then pass 1);
-// z holds the offsets of the pass-0 and pass-1 groups.
+// z holds the offsets of the pass-0 and pass-1 groups (z1: those of row 1
+// when the two rows of a mixed launch take their own offsets).
 template <int M, int P>
 struct ScaleSet {
   uint32_t a[M][P];
-  uint32_t z;
+  uint32_t z, z1;
 };
 
 template <int M, int P, bool MIXED>
@@ -330,6 +331,7 @@ __device__ __forceinline__ void load_scales(const GemvParams& prm, int kb, int r
     }
   }
   s.z = prm.z ? ldg_nc_u32(prm.z + e * 2) : 0u;
+  if (MIXED && M == 2) s.z1 = prm.z1 == prm.z ? s.z : (prm.z1 ? ldg_nc_u32(prm.z1 + e * 2) : 0u);
 }
 
 template <int M, int P>
@@ -338,7 +340,7 @@ __device__ __forceinline__ void zero_scales(ScaleSet<M, P>& s) {
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int r = 0; r < P; ++r) s.a[m][r] = 0u;
-  s.z = 0u;
+  s.z = s.z1 = 0u;
 }
 
 __device__ __forceinline__ float half_at(uint32_t r, int hi) {
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   float acc[PF][M];
   bool pend[PF];
   int pend_row[PF] = {0, 0}, pend_kb[PF] = {0, 0};
-  uint32_t pend_z[PF] = {0u, 0u};
+  uint32_t pend_z[PF] = {0u, 0u}, pend_z1[PF] = {0u, 0u};
 #pragma unroll
   for (int j = 0; j < PF; ++j) pend[j] = false;
 
@@ -459,10 +461,12 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     if (!pend[J]) return;
     pend[J] = false;
     if (*abort_flag) return;
-    const float z0 = half_at(pend_z[J], 0), z1 = half_at(pend_z[J], 1);
     float r[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) r[m] = fmaf(z0, gs[m][0], fmaf(z1, gs[m][1], acc[J][m]));
+    for (int m = 0; m < M; ++m) {
+      const uint32_t zr = (MIXED && m == 1) ? pend_z1[J] : pend_z[J];
+      r[m] = fmaf(half_at(zr, 0), gs[m][0], fmaf(half_at(zr, 1), gs[m][1], acc[J][m]));
+    }
     const int row = pend_row[J];
     if (prm.KB > 1) {
 #pragma unroll
@@ -579,6 +583,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     pend_row[J] = (gc.rb0 + tw) * kRowBlock + lane;
     pend_kb[J] = gc.kb;
     pend_z[J] = sc.z;
+    if (MIXED) pend_z1[J] = sc.z1;
     // this slot's scales now take the team's group PF ahead
     zero_scales(pf[J]);
     if (gp < R.NG && tw < pc.n) load_scales<M, P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, pf[J]);

@@ -168,7 +168,8 @@ struct GemvParams {
   const uint16_t* x;         // fp16 [M][K] (rows of this launch)
   const uint32_t* planes;    // packed planes
   const uint16_t* alpha[2];  // packed scales of row 0 and row 1 (q[m] per entry)
-  const uint16_t* z;         // packed offsets, or nullptr
+  const uint16_t* z;         // packed offsets of the launch (of row 0 in a mixed lookup launch), or nullptr
+  const uint16_t* z1;        // packed offsets of row 1 in a mixed lookup launch (per-precision offsets)
   uint16_t* y;               // fp16 [M][N] (rows of this launch)
   float* part;               // tagged fp32 partial sums [KB][M][RB * 32] (KB > 1), zero between calls
   int M, N, K, KB, RB, RG, p_H;

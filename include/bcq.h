@@ -172,6 +172,27 @@ bcq_status bcq_gemm(const uint16_t* x, const uint32_t* planes,
                     void* stream);
 
 /*
+ * bcq_gemm with offsets per precision: row m uses z^(p_m) with its scales
+ * alpha^(p_m), i.e. W_hat^(p)[n][k] = sum_{i<p} alpha^(p)[n][g][i] B_i[n][k]
+ * + z^(p)[n][g].  The pages write the offset without a precision index
+ * (AnyBCQ page, "训练策略": asymmetric quantisation); this entry point is the
+ * variant in which every precision keeps its own offsets, as the expansion
+ * in "渐进式精度扩展" keeps its own scales.
+ *
+ *   z   HOST array of 4 device pointers, or NULL (no offsets); z[q-1] -> the
+ *       offsets of precision q (canonically fp16 [N][K/128]) packed by
+ *       bcq_pack_scales(.., 1, ..), or NULL (= 0 for that precision).  Only
+ *       the precisions used by the call are read; 16-byte aligned.
+ * Every other argument, the result and the errors are those of bcq_gemm;
+ * bcq_gemm(.., z, ..) is bcq_gemm_zp with z[0..3] all equal to z.
+ */
+bcq_status bcq_gemm_zp(const uint16_t* x, const uint32_t* planes,
+                       const uint16_t* const alpha[4], const uint16_t* const z[4],
+                       int p, const int32_t* p_row, int M, int N, int K, int p_H,
+                       int group, uint16_t* y, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
  * The launch plan bcq_gemm would use for one launch of M (1..64) activation
  * rows streaming p_load planes (mixed = 1: two rows of different
  * precisions).  M <= 2 plans the lookup-table kernel, 3 <= M <= 16 the

@@ -132,10 +132,27 @@ def gemm(x, planes, alphas: dict, z=None, p: int | None = None,
     """y = x @ W_hat^T in fp64 (see bcq_oracle.c for the definition).
 
     x: fp16 [M][K]; planes: uint32 [p_H][N][K/32]; alphas: {q: fp16 [N][G][q]};
-    z: fp16 [N][G] or None; exactly one of ``p`` (uniform precision) and
-    ``p_row`` (int per row of x) is given; ``rows`` optionally selects output
-    rows n (returns [M][len(rows)]).
+    z: fp16 [N][G], or {q: fp16 [N][G]} (offsets per precision: row m uses
+    z^(p_m), the variant in which each precision keeps its own offsets, as it
+    keeps its own scales -- AnyBCQ page, 渐进式精度扩展), or None; exactly one
+    of ``p`` (uniform precision) and ``p_row`` (int per row of x) is given;
+    ``rows`` optionally selects output rows n (returns [M][len(rows)]).
     """
+    if isinstance(z, dict):
+        # the rows of each precision through the same definition, with that
+        # precision's offsets
+        xa = _as_half_bits(x)
+        if xa.ndim == 1:
+            xa = xa[None, :]
+        pr = np.full(xa.shape[0], int(p)) if p is not None else np.asarray(p_row, dtype=np.int64)
+        out = None
+        for q in sorted(set(int(v) for v in pr)):
+            sel = np.nonzero(pr == q)[0]
+            yq = gemm(xa[sel], planes, alphas, z.get(q), p=q, group=group, rows=rows)
+            if out is None:
+                out = np.empty((xa.shape[0], yq.shape[1]), dtype=np.float64)
+            out[sel] = yq
+        return out
     x = _as_half_bits(x)
     if x.ndim == 1:
         x = x[None, :]

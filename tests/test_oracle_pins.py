@@ -303,3 +303,22 @@ def test_greedy_bcq_scale_is_mean_abs_and_error_monotone():
     assert abs(a[0] - np.mean(np.abs(w))) < 1e-12
     errs = [float(np.sum((w - (a[:q, None] * B[:q]).sum(axis=0)) ** 2)) for q in range(1, 5)]
     assert all(e2 <= e1 + 1e-12 for e1, e2 in zip(errs, errs[1:]))
+
+
+def test_gemm_per_precision_offsets_closed_forms():
+    # alpha = 0: y[m][n] = sum_g z^(p_m)[n][g] * (sum of x[m] over group g),
+    # the group sums taken directly with numpy; one shared array in every
+    # slot of the dict is the single-offset call
+    prob = synth.make_problem(48, 384, 5, seed=23)
+    rng = np.random.default_rng(24)
+    zq = {q: rng.normal(0.0, 0.01, size=(48, 3)).astype(np.float16) for q in (2, 3, 4)}
+    zero = {q: np.zeros_like(a) for q, a in prob.alphas.items()}
+    p_row = np.array([2, 4, 3, 3, 2], dtype=np.int32)
+    y = oracle.gemm(prob.x, prob.planes, zero, zq, p_row=p_row)
+    xs = prob.x.astype(np.float64).reshape(5, 3, 128).sum(axis=2)
+    for m in range(5):
+        ref = zq[int(p_row[m])].astype(np.float64) @ xs[m]
+        assert np.allclose(y[m], ref, rtol=1e-12, atol=1e-12)
+    same = {q: prob.z for q in (2, 3, 4)}
+    assert np.array_equal(oracle.gemm(prob.x, prob.planes, prob.alphas, same, p_row=p_row),
+                          oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=p_row))

@@ -93,6 +93,8 @@ def lib():
         L.bcq_debug_wait_timeout.argtypes = [I, P]
         L.bcq_quantize.restype = I
         L.bcq_quantize.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
+        L.bcq_quantize_zp.restype = I
+        L.bcq_quantize_zp.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -101,7 +103,7 @@ EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
             "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl",
             "bcq_gemm_host", "bcq_gemm_noalloc", "bcq_build_lut", "bcq_device_error",
-            "bcq_debug_wait_timeout", "bcq_quantize", "bcq_gemm_zp")
+            "bcq_debug_wait_timeout", "bcq_quantize", "bcq_gemm_zp", "bcq_quantize_zp")
 
 
 def status_string(status: int) -> str:
@@ -186,11 +188,15 @@ def pack_scales(src: torch.Tensor, q: int, stream=None) -> torch.Tensor:
 
 
 def quantize(w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
-             with_sse: bool = False, stream=None):
+             with_sse: bool = False, offsets: str = "shared", stream=None):
     """Offline quantiser (bcq_quantize): fp16 CUDA weights [N][K] ->
     (planes int32 [p_H][N][K/32] holding the uint32 words, {p: alpha^(p) fp16
     [N][K/128][p]} for p = p_L..p_H, z fp16 [N][K/128], and with_sse: fp64
-    [p_H - p_L + 1][N][K/128] squared error per group, else None)."""
+    [p_H - p_L + 1][N][K/128] squared error per group, else None).
+    offsets="per_precision" (bcq_quantize_zp): z is {p: z^(p) fp16 [N][K/128]}
+    for the per-precision offsets of bcq_gemm_zp."""
+    if offsets not in ("shared", "per_precision"):
+        raise ValueError("offsets must be 'shared' or 'per_precision'")
     _need_cuda(w, "w", torch.float16)
     if w.dim() != 2:
         raise ValueError("w must be [N][K]")
@@ -200,9 +206,15 @@ def quantize(w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
     planes = torch.empty((p_H, N, K // 32), dtype=torch.int32, device=dev)
     alphas = {p: torch.empty((N, G, p), dtype=torch.float16, device=dev)
               for p in range(p_L, p_H + 1)} if 1 <= p_L <= p_H <= 4 else {}
-    z = torch.empty((N, G), dtype=torch.float16, device=dev)
     sse = (torch.empty((max(p_H - p_L + 1, 0), N, G), dtype=torch.float64, device=dev)
            if with_sse else None)
+    if offsets == "per_precision":
+        z = {p: torch.empty((N, G), dtype=torch.float16, device=dev) for p in alphas}
+        _check(lib().bcq_quantize_zp(_ptr(w), N, K, int(p_L), int(p_H), int(rounds),
+                                     _ptr(planes), _alpha_array(alphas), _alpha_array(z, "z"),
+                                     _ptr(sse), _stream(stream)), "bcq_quantize_zp")
+        return planes, alphas, z, sse
+    z = torch.empty((N, G), dtype=torch.float16, device=dev)
     _check(lib().bcq_quantize(_ptr(w), N, K, int(p_L), int(p_H), int(rounds), _ptr(planes),
                               _alpha_array(alphas), _ptr(z), _ptr(sse), _stream(stream)),
            "bcq_quantize")
@@ -299,10 +311,11 @@ class BcqWeights:
 
     @classmethod
     def quantize(cls, w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
-                 stream=None):
-        """Quantise fp16 CUDA weights [N][K] on the device (bcq_quantize) and
-        pack the result for bcq_gemm."""
-        planes, alphas, z, _ = quantize(w, p_L, p_H, rounds, stream=stream)
+                 offsets: str = "shared", stream=None):
+        """Quantise fp16 CUDA weights [N][K] on the device (bcq_quantize, or
+        bcq_quantize_zp for offsets="per_precision") and pack the result for
+        bcq_gemm (bcq_gemm_zp)."""
+        planes, alphas, z, _ = quantize(w, p_L, p_H, rounds, offsets=offsets, stream=stream)
         return cls.from_canonical(planes, alphas, z, device=w.device, stream=stream)
 
     @classmethod

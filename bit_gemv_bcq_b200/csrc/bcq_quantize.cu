@@ -48,7 +48,8 @@ struct QuantParams {
   const __half* w;       // fp16 [N][K]
   uint32_t* planes;      // uint32 [p_H][N][K/32]
   __half* alpha[4];      // alpha[q-1]: fp16 [N][G][q] (q = p_L..p_H)
-  __half* z;             // fp16 [N][G]
+  __half* z;             // fp16 [N][G] (shared offsets)
+  __half* zq[4];         // per-precision offsets: zq[p-1] fp16 [N][G] (p = p_L..p_H)
   double* sse;           // fp64 [p_H - p_L + 1][N][G], or nullptr
   long long groups;      // N * G
   int N, K, G, rounds;
@@ -393,10 +394,12 @@ __device__ __forceinline__ void base_precision(const QuantParams& q, const doubl
   lsq_with_offset<PL>(w, sumw, code, alpha, z);
 }
 
-template <int P, int PH>
+// Expansion p -> p + 1: B_{p+1} = sign(R_p), then every scale refit with z
+// kept (shared offsets) or refit with it (q.zp: offsets per precision).
+template <int P, int PH, bool ZP>
 __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int lane, int p_L,
-                                       const double (&w)[4], double z, unsigned (&code)[4],
-                                       const double (&alpha)[P]) {
+                                       const double (&w)[4], double sumw, double z,
+                                       unsigned (&code)[4], const double (&alpha)[P]) {
   if constexpr (P < PH) {
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
@@ -404,14 +407,20 @@ __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int 
       code[s] |= (res >= 0.0 ? 1u : 0u) << P;
     }
     double next[P + 1];
-    lsq_fixed_offset<P + 1>(w, z, code, next);
-    const double e = q.sse ? group_sse<P + 1>(w, next, z, code) : 0.0;
+    double zn = z;
+    if constexpr (ZP) {
+      lsq_with_offset<P + 1>(w, sumw, code, next, zn);
+      if (lane == 0) q.zq[P][gid] = __double2half(zn);
+    } else {
+      lsq_fixed_offset<P + 1>(w, z, code, next);
+    }
+    const double e = q.sse ? group_sse<P + 1>(w, next, zn, code) : 0.0;
     store_scales<P + 1>(q, gid, lane, next, e, p_L);
-    expand<P + 1, PH>(q, gid, lane, p_L, w, z, code, next);
+    expand<P + 1, PH, ZP>(q, gid, lane, p_L, w, sumw, zn, code, next);
   }
 }
 
-template <int PL, int PH>
+template <int PL, int PH, bool ZP>
 __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinBlocks) quantize_kernel(QuantParams q) {
   const int lane = threadIdx.x & 31;
   const long long gid = (long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
@@ -429,8 +438,8 @@ __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinBlocks) quantize_ke
   base_precision<PL>(q, w, sumw, code, alpha, z);
   const double e = q.sse ? group_sse<PL>(w, alpha, z, code) : 0.0;
   store_scales<PL>(q, gid, lane, alpha, e, PL);
-  if (lane == 0) q.z[gid] = __double2half(z);
-  expand<PL, PH>(q, gid, lane, PL, w, z, code, alpha);
+  if (lane == 0) (ZP ? q.zq[PL - 1] : q.z)[gid] = __double2half(z);
+  expand<PL, PH, ZP>(q, gid, lane, PL, w, sumw, z, code, alpha);
 
   // planes: lane 4 i + s writes word s of plane i
   uint32_t pw[PH][4];
@@ -445,9 +454,9 @@ __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinBlocks) quantize_ke
 
 using QuantKernel = void (*)(QuantParams);
 
-QuantKernel quantize_kernel_for(int p_L, int p_H) {
+QuantKernel quantize_kernel_for(int p_L, int p_H, bool zp) {
 #define BCQ_Q(a, b) \
-  if (p_L == a && p_H == b) return quantize_kernel<a, b>;
+  if (p_L == a && p_H == b) return zp ? quantize_kernel<a, b, true> : quantize_kernel<a, b, false>;
   BCQ_Q(1, 1) BCQ_Q(1, 2) BCQ_Q(1, 3) BCQ_Q(1, 4)
   BCQ_Q(2, 2) BCQ_Q(2, 3) BCQ_Q(2, 4)
   BCQ_Q(3, 3) BCQ_Q(3, 4)
@@ -461,28 +470,35 @@ bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 }  // namespace
 }  // namespace bcq
 
-extern "C" bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int p_H,
-                                   int rounds, uint32_t* planes, uint16_t* const alpha[4],
-                                   uint16_t* z, double* sse, void* stream) {
-  using namespace bcq;
+namespace bcq {
+namespace {
+
+bcq_status quantize_common(const uint16_t* w, int N, int K, int p_L, int p_H, int rounds,
+                           uint32_t* planes, uint16_t* const alpha[4], uint16_t* z,
+                           uint16_t* const zq[4], double* sse, void* stream) {
   if (!alpha) return BCQ_ERR_NULL;
   if (p_H < 1 || p_H > BCQ_MAX_PLANES || p_L < 1 || p_L > p_H) return BCQ_ERR_PRECISION;
   if (N < 0 || K < 0 || K % BCQ_GROUP != 0 || rounds < 0 || rounds > 1000) return BCQ_ERR_SHAPE;
   if ((long long)N * (K / BCQ_GROUP) > (1ll << 33)) return BCQ_ERR_SHAPE;
   if (N == 0 || K == 0) return BCQ_OK;
-  if (!w || !planes || !z) return BCQ_ERR_NULL;
-  for (int p = p_L; p <= p_H; ++p)
+  if (!w || !planes || (!z && !zq)) return BCQ_ERR_NULL;
+  for (int p = p_L; p <= p_H; ++p) {
     if (!alpha[p - 1]) return BCQ_ERR_PRECISION;
-  if (!aligned_to(w, 2) || !aligned_to(planes, 4) || !aligned_to(z, 2) ||
+    if (zq && !zq[p - 1]) return BCQ_ERR_NULL;
+  }
+  if (!aligned_to(w, 2) || !aligned_to(planes, 4) || (z && !aligned_to(z, 2)) ||
       (sse && !aligned_to(sse, 8)))
     return BCQ_ERR_ALIGN;
   for (int p = p_L; p <= p_H; ++p)
-    if (!aligned_to(alpha[p - 1], 2)) return BCQ_ERR_ALIGN;
+    if (!aligned_to(alpha[p - 1], 2) || (zq && !aligned_to(zq[p - 1], 2))) return BCQ_ERR_ALIGN;
   QuantParams q{};
   q.w = reinterpret_cast<const __half*>(w);
   q.planes = planes;
-  for (int p = 1; p <= 4; ++p)
-    q.alpha[p - 1] = (p >= p_L && p <= p_H) ? reinterpret_cast<__half*>(alpha[p - 1]) : nullptr;
+  for (int p = 1; p <= 4; ++p) {
+    const bool used = p >= p_L && p <= p_H;
+    q.alpha[p - 1] = used ? reinterpret_cast<__half*>(alpha[p - 1]) : nullptr;
+    q.zq[p - 1] = used && zq ? reinterpret_cast<__half*>(zq[p - 1]) : nullptr;
+  }
   q.z = reinterpret_cast<__half*>(z);
   q.sse = sse;
   q.N = N;
@@ -490,9 +506,26 @@ extern "C" bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int
   q.G = K / BCQ_GROUP;
   q.groups = (long long)N * q.G;
   q.rounds = rounds;
-  const QuantKernel fn = quantize_kernel_for(p_L, p_H);
+  const QuantKernel fn = quantize_kernel_for(p_L, p_H, zq != nullptr);
   if (!fn) return BCQ_ERR_UNSUPPORTED;
   const long long blocks = (q.groups + kQuantWarps - 1) / kQuantWarps;
   fn<<<(unsigned)blocks, 32 * kQuantWarps, 0, (cudaStream_t)stream>>>(q);
   return cudaGetLastError() == cudaSuccess ? BCQ_OK : BCQ_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace bcq
+
+extern "C" bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int p_H,
+                                   int rounds, uint32_t* planes, uint16_t* const alpha[4],
+                                   uint16_t* z, double* sse, void* stream) {
+  if (!z && N > 0 && K > 0) return BCQ_ERR_NULL;
+  return bcq::quantize_common(w, N, K, p_L, p_H, rounds, planes, alpha, z, nullptr, sse, stream);
+}
+
+extern "C" bcq_status bcq_quantize_zp(const uint16_t* w, int N, int K, int p_L, int p_H,
+                                      int rounds, uint32_t* planes, uint16_t* const alpha[4],
+                                      uint16_t* const z[4], double* sse, void* stream) {
+  if (!z && N > 0 && K > 0) return BCQ_ERR_NULL;
+  return bcq::quantize_common(w, N, K, p_L, p_H, rounds, planes, alpha, nullptr, z, sse, stream);
 }

@@ -314,6 +314,22 @@ bcq_status bcq_quantize(const uint16_t* w, int N, int K, int p_L, int p_H, int r
                         double* sse, void* stream);
 
 /*
+ * bcq_quantize for the per-precision offsets of bcq_gemm_zp: the same steps,
+ * except that each expansion p -> p + 1 refits the offset z^(p+1) jointly
+ * with the p + 1 scales (least squares with the all-ones column first, as at
+ * the base precision) and the residual of precision p uses z^(p).
+ *
+ *   z   HOST array of 4 device pointers; z[p-1] for p = p_L..p_H receives
+ *       fp16 [N][K/128] (2-byte aligned), the others are ignored; z^(p_L) is
+ *       the offset bcq_quantize would write.
+ * Every other argument and error is that of bcq_quantize (a NULL z or a
+ * NULL z[p-1] in p_L..p_H -> BCQ_ERR_NULL).
+ */
+bcq_status bcq_quantize_zp(const uint16_t* w, int N, int K, int p_L, int p_H, int rounds,
+                           uint32_t* planes, uint16_t* const alpha[4], uint16_t* const z[4],
+                           double* sse, void* stream);
+
+/*
  * The lookup table and group sums exactly as the GEMV kernel builds them in
  * shared memory (AnyBCQ page, "直接bit-plane运算的CUDA内核": cached signed
  * partial sums of x).  For test and inspection.

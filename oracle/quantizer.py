@@ -50,7 +50,12 @@ Readings (the pages leave them open):
   * candidate values and residuals are formed in fp64 as
     z + (((alpha_1 b_1) + alpha_2 b_2) + ...), left to right;
   * sign(0) = +1; inputs are fp16 weights widened to fp64; scales and offsets
-    are rounded to fp16 (nearest even) only when stored.
+    are rounded to fp16 (nearest even) only when stored;
+  * variant with offsets per precision (offsets="per_precision", for the
+    format in which every precision keeps its own z^(p) as it keeps its own
+    scales): each expansion refits z jointly with all p + 1 scales (the
+    all-ones column first, as at the base precision); the residual of
+    precision p uses z^(p).
 """
 from __future__ import annotations
 
@@ -180,15 +185,19 @@ def group_sse(W, B, alpha, z):
     return np.sum(residual(W, B, alpha, z) ** 2, axis=1)
 
 
-def quantize_groups(W, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None):
+def quantize_groups(W, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None,
+                    offsets: str = "shared"):
     """Quantise P independent groups W [P][n] (fp64).
 
     Returns (B [P][p_H][n] in {-1,+1}, {p: alpha^(p) [P][p]} for p = p_L..p_H,
-    z [P]).  trace, if a list, receives (stage, sse [P]) after every step."""
+    z [P]; with offsets="per_precision", z is {p: z^(p) [P]}).  trace, if a
+    list, receives (stage, sse [P]) after every step."""
     W = np.asarray(W, dtype=np.float64)
     P, n = W.shape
     if not 1 <= p_L <= p_H:
         raise ValueError("need 1 <= p_L <= p_H")
+    if offsets not in ("shared", "per_precision"):
+        raise ValueError("offsets must be 'shared' or 'per_precision'")
 
     def record(stage, B, alpha, z):
         if trace is not None:
@@ -218,32 +227,40 @@ def quantize_groups(W, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None)
         B = best_codes(W, alpha, z)
         record("codes", B, alpha, z)
     alpha, z = lsq(W, B)
-    out_alpha = {p_L: alpha}
+    out_alpha, out_z = {p_L: alpha}, {p_L: z}
     record(f"p{p_L}", B, alpha, z)
-    # progressive expansion: codes and z frozen, the residual's sign appended
+    # progressive expansion: codes (and shared z) frozen, the residual's sign appended
     for p in range(p_L, p_H):
         B = np.concatenate([B, sign_pm1(residual(W, B, alpha, z))[:, None, :]], axis=1)
-        alpha, _ = lsq(W, B, z)
+        if offsets == "shared":
+            alpha, _ = lsq(W, B, z)
+        else:
+            alpha, z = lsq(W, B)
         out_alpha[p + 1] = alpha
+        out_z[p + 1] = z
         record(f"p{p + 1}", B, alpha, z)
-    return B, out_alpha, z
+    return B, out_alpha, (z if offsets == "shared" else out_z)
 
 
-def quantize(W, group: int = 128, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None):
+def quantize(W, group: int = 128, p_L: int = 2, p_H: int = 4, rounds: int = 20, trace=None,
+             offsets: str = "shared"):
     """Quantise a weight W [N][K] (K a multiple of the group size and of 32)
     into the canonical format the GEMV reads.
 
     Returns (planes uint32 [p_H][N][K/32], bit j of word w = column 32w + j,
     bit 1 = +1; {p: alpha^(p) fp64 [N][K/group][p]} for p = p_L..p_H;
-    z fp64 [N][K/group]).  trace: as for quantize_groups (groups row-major)."""
+    z fp64 [N][K/group], or {p: z^(p)} with offsets="per_precision").  trace:
+    as for quantize_groups (groups row-major)."""
     W = np.asarray(W, dtype=np.float64)
     N, K = W.shape
     if K % group or K % 32:
         raise ValueError("K must be a multiple of the group size and of 32")
     G = K // group
-    B, alphas, z = quantize_groups(W.reshape(N * G, group), p_L, p_H, rounds, trace)
+    B, alphas, z = quantize_groups(W.reshape(N * G, group), p_L, p_H, rounds, trace, offsets)
     bits = (B > 0).reshape(N, G, p_H, group).transpose(2, 0, 1, 3).reshape(p_H, N, K)
     words = bits.reshape(p_H, N, K // 32, 32).astype(np.uint64)
     planes = np.sum(words << np.arange(32, dtype=np.uint64), axis=3).astype(np.uint32)
     out = {p: a.reshape(N, G, p) for p, a in alphas.items()}
+    if isinstance(z, dict):
+        return planes, out, {p: zp.reshape(N, G) for p, zp in z.items()}
     return planes, out, z.reshape(N, G)

@@ -168,3 +168,52 @@ def test_empty_and_bad_arguments():
     with pytest.raises(api.BcqError) as e:
         api.quantize(torch.zeros((4, 200), dtype=torch.float16, device="cuda"))
     assert e.value.status == api.BCQ_ERR_SHAPE
+
+
+# ------------------------------------------------- variant: offsets per precision
+
+def _gpu_zp(w16, p_L=2, p_H=4, rounds=20):
+    w = torch.from_numpy(w16.view(np.int16)).view(torch.float16).cuda()
+    planes, alphas, z, sse = api.quantize(w, p_L, p_H, rounds, with_sse=True,
+                                          offsets="per_precision")
+    torch.cuda.synchronize()
+    return (planes.cpu().numpy().view(np.uint32), {p: a.cpu().numpy() for p, a in alphas.items()},
+            {p: v.cpu().numpy() for p, v in z.items()}, sse.cpu().numpy())
+
+
+@pytest.mark.parametrize("p_L,p_H", [(2, 4), (1, 4), (3, 4), (1, 2)])
+def test_parity_per_precision_offsets(p_L, p_H):
+    structured = np.tile(_structured(6), (1, 2))[:, :384]   # 5 rows of special groups
+    w16 = np.concatenate([synth.make_weights(37, 384, seed=40 + p_L), structured])
+    gp, ga, gz, gs = _gpu_zp(w16, p_L, p_H)
+    tr = []
+    rp, ra, rz = Q.quantize(w16.astype(np.float64), 128, p_L, p_H, 20, trace=tr,
+                            offsets="per_precision")
+    rs = np.stack([e for s, e in tr if s.startswith("p")]).reshape(p_H - p_L + 1, 42, 3)
+    assert np.array_equal(gp, rp)
+    for p in range(p_L, p_H + 1):
+        assert np.array_equal(ga[p].view(np.uint16), ra[p].astype(np.float16).view(np.uint16))
+        assert np.array_equal(gz[p].view(np.uint16), rz[p].astype(np.float16).view(np.uint16))
+    assert np.allclose(gs, rs, rtol=1e-9, atol=1e-30)
+    # the base precision equals the shared-offset quantiser's
+    sp, sa, sz, _ = _gpu(w16, p_L, p_H)
+    assert np.array_equal(gz[p_L].view(np.uint16), sz.view(np.uint16))
+    assert np.array_equal(ga[p_L].view(np.uint16), sa[p_L].view(np.uint16))
+
+
+def test_per_precision_weights_feed_gemm_zp():
+    import oracle
+    N, K = 128, 512
+    w16 = synth.make_weights(N, K, seed=51)
+    w = torch.from_numpy(w16.view(np.int16)).view(torch.float16).cuda()
+    bw = api.BcqWeights.quantize(w, offsets="per_precision")
+    planes, alphas, z, _ = api.quantize(w, offsets="per_precision")
+    pl = planes.cpu().numpy().view(np.uint32)
+    al = {p: a.cpu().numpy() for p, a in alphas.items()}
+    zq = {p: v.cpu().numpy() for p, v in z.items()}
+    x16 = synth.make_x(5, K, seed=52)
+    x = torch.from_numpy(x16.view(np.int16)).view(torch.float16).cuda()
+    p_row = np.array([2, 4, 3, 2, 4], dtype=np.int32)
+    y = bw.gemm(x, p_row=p_row).float().cpu().numpy().astype(np.float64)
+    ref = oracle.gemm(x16, pl, al, zq, p_row=p_row)
+    assert np.all(np.abs(y - ref) <= 1e-2 + 2e-3 * np.abs(ref))

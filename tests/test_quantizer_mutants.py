@@ -21,13 +21,15 @@ PINS = os.path.join(ROOT, "tests", "test_quantizer_oracle.py")
 MUTANTS = {
     # expansion refits only the new plane's scale, the old ones stay
     "expansion_new_scale_only": (
-        "        alpha, _ = lsq(W, B, z)\n",
-        "        a_new, _ = lsq(W - code_values(alpha, z, B[:, :-1]) + z[:, None], B[:, -1:], z)\n"
-        "        alpha = np.concatenate([alpha, a_new], axis=1)\n"),
+        "            alpha, _ = lsq(W, B, z)\n",
+        "            a_new, _ = lsq(W - code_values(alpha, z, B[:, :-1]) + z[:, None], B[:, -1:], z)\n"
+        "            alpha = np.concatenate([alpha, a_new], axis=1)\n"),
     "expansion_residual_sign_flipped": (
         "sign_pm1(residual(W, B, alpha, z))", "sign_pm1(-residual(W, B, alpha, z))"),
     "expansion_refits_offset": (
-        "        alpha, _ = lsq(W, B, z)\n", "        alpha, z = lsq(W, B)\n"),
+        "            alpha, _ = lsq(W, B, z)\n", "            alpha, z = lsq(W, B)\n"),
+    "per_precision_variant_keeps_offset": (
+        "            alpha, z = lsq(W, B)\n", "            alpha, _ = lsq(W, B)\n"),
     "code_update_farthest": ("idx = np.argmin(err, axis=2)", "idx = np.argmax(err, axis=2)"),
     "code_ties_to_last": (
         "idx = np.argmin(err, axis=2)",

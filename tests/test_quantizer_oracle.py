@@ -392,3 +392,31 @@ def test_quantize_rejects_ragged_k():
         Q.quantize(np.zeros((2, 200)))
     with pytest.raises(ValueError):
         Q.quantize_groups(np.zeros((2, 128)), p_L=3, p_H=2)
+
+
+# ------------------------------------------------- variant: offsets per precision
+
+def test_per_precision_offsets_variant():
+    w = _weights((24, 128), 17)
+    tr_s, tr_v = [], []
+    Bs, als, zs = Q.quantize_groups(w, 2, 4, trace=tr_s)
+    Bv, alv, zv = Q.quantize_groups(w, 2, 4, trace=tr_v, offsets="per_precision")
+    # the base precision is the same; z^(p_L) is the shared z
+    assert np.array_equal(Bv[:, :3], Bs[:, :3]) and np.array_equal(alv[2], als[2])
+    assert np.array_equal(zv[2], zs)
+    # every precision: (z^(p), alpha^(p)) jointly least squares for its codes
+    for p in (2, 3, 4):
+        res = w - zv[p][:, None] - np.einsum("qi,qin->qn", alv[p], Bv[:, :p])
+        assert np.max(np.abs(res.sum(axis=1))) < 1e-12
+        assert np.max(np.abs(np.einsum("qin,qn->qi", Bv[:, :p], res))) < 1e-12
+    # B_{p+1} = sign of the residual with z^(p); the error falls with p and is
+    # never above the shared-offset variant's (a larger least-squares space)
+    for p in (2, 3):
+        res = w - zv[p][:, None] - np.einsum("qi,qin->qn", alv[p], Bv[:, :p])
+        assert np.array_equal(Bv[:, p], np.where(res >= 0, 1.0, -1.0))
+    e = [t for s, t in tr_v if s in ("p2", "p3", "p4")]
+    assert np.all(e[1] <= e[0] * (1 + 1e-12)) and np.all(e[2] <= e[1] * (1 + 1e-12))
+    es = [t for s, t in tr_s if s == "p3"][0]
+    assert np.all(e[1] <= es * (1 + 1e-12))
+    with pytest.raises(ValueError):
+        Q.quantize_groups(w, 2, 4, offsets="bogus")

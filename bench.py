@@ -104,6 +104,34 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+# ------------------------------------------------------------- ranks (N > 1)
+
+def rank_barrier(world):
+    """Barrier of all ranks (no-op on one GPU)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (the job's time is its slowest
+    rank's); `device` is where the process group's backend reduces (cuda for
+    NCCL, cpu for gloo)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbps(bytes_per_rank_step, ms_per_step, world):
+    """Whole-job throughput: every rank processes its own bytes_per_rank_step
+    per step (weak scaling, replicas), in ms_per_step (the max over ranks)."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -217,9 +245,7 @@ def run_gpu(args, rank, world, local_rank):
         case_graphs[(p, M)] = capture(one)
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+        rank_barrier(world)
 
     with torch.cuda.stream(stream):
         for k in range(args.warmup):
@@ -247,11 +273,7 @@ def run_gpu(args, rank, world, local_rank):
     if err != api.BCQ_OK:
         raise RuntimeError(f"device error {api.status_string(err)}")
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
 
     # per-case microseconds (same stream, events around each replay)
     per_case = []
@@ -347,11 +369,7 @@ def run_gpu(args, rank, world, local_rank):
         b.record(stream)
         b.synchronize()
         e2e_ms = a.elapsed_time(b)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
         result["e2e"] = {"ms": e2e_ms, "steps": e2e_steps, "h2d": h2d, "d2h": d2h}
     return result
 
@@ -544,7 +562,7 @@ def main():
 
     peak, peak_kind = measured_peaks()
     ms_step = res["ms_total"] / args.steps
-    value = world * res["bytes_step"] / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbps(res["bytes_step"], ms_step, world)
     achieved_per_gpu = res["bytes_step"] / (ms_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -590,7 +608,7 @@ def main():
                                           "frac": round(c["GBps"] / peak, 4)} for c in m1}
     if "e2e" in res:
         e = res["e2e"]
-        line["e2e"] = {"value": round(world * res["bytes_step"] * e["steps"] / (e["ms"] * 1e-3) / 1e9, 2),
+        line["e2e"] = {"value": round(whole_job_gbps(res["bytes_step"], e["ms"] / e["steps"], world), 2),
                        "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": round(e["ms"] / e["steps"], 4),
                        "path": "bcq_gemm_host (pinned host x/y, copies on the stream)"}

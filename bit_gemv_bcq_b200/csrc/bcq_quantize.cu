@@ -7,19 +7,22 @@
 // scale of alpha^(p+1) by least squares.  "训练策略": asymmetric, group 128,
 // 20 refinement rounds.
 //
-// One warp quantises one 128-weight group; lane l holds columns l + 32 s,
-// s = 0..3, so a ballot over the lanes of plane bit i in slot s is word s of
-// the group's canonical plane i.  Everything is fp64 (the weights are fp16,
+// Half a warp quantises one 128-weight group (two groups per warp, so the
+// per-group work every lane repeats -- Gram counts, the solve, candidate
+// values -- is shared by two groups); lane j of a half holds columns
+// j + 16 s, s = 0..7, so the ballot of plane bit i over slot s carries 16
+// columns of each half's group, and one byte permute of two ballots gives a
+// canonical 32-column plane word.  Everything is fp64 (the weights are fp16,
 // widened exactly).  Per step:
 //   * the Gram matrix of the +-1 planes (and the all-ones column of z) is
-//     integer-valued and comes exactly from popcounts of the ballot words;
-//   * right-hand sides are warp sums (xor butterfly: every lane ends with the
-//     same bits, since a + b == b + a), so every lane solves the same system
-//     and holds the same scales without a broadcast;
+//     integer-valued and comes exactly from popcounts of the plane words;
+//   * right-hand sides are sums over the half (xor butterfly: every lane ends
+//     with the same bits, since a + b == b + a), so every lane solves the same
+//     system and holds the same scales without a broadcast;
 //   * columns exactly dependent on the columns before them (a plane equal to
 //     another, to its negation or to the all-ones column, or any exact linear
-//     dependence) get scale 0: fraction-free integer elimination decides it,
-//     then an LDL^T solve in fp64 on the kept columns gives the scales;
+//     dependence) get scale 0; the normal equations of the kept columns are
+//     solved by Cramer's rule with the exact integer adjugate;
 //   * the code update gives every weight the code whose value
 //     z + (((alpha_1 b_1) + alpha_2 b_2) + ...) is nearest, first code in
 //     enumeration order on ties (code c: b_i = +1 where bit i of c is set).
@@ -37,12 +40,14 @@ namespace bcq {
 namespace {
 
 constexpr int kQuantGroup = 128;
-constexpr int kQuantWarps = 8;  // groups per CTA
-// Four CTAs (32 warps) per SM: 64 registers a thread.  The code is a chain
-// of dependent fp64 steps per group, so resident warps, not registers, set
-// the speed (measured: 3.8 ms against 4.4 ms at two CTAs per SM for a
-// 14336 x 4096 weight); the spills sit on the rare general-solve path.
-constexpr int kQuantMinBlocks = 4;
+constexpr int kGroupLanes = 16;                       // lanes per group (half a warp)
+constexpr int kSlots = kQuantGroup / kGroupLanes;     // weights per lane
+constexpr int kQuantWarps = 8;                        // warps per CTA (two groups each)
+// Two CTAs (16 warps, 32 groups) per SM: 128 registers a thread and no
+// spills.  Measured on a 14336 x 4096 weight (p_L = 2 -> p_H = 4): 3.07 ms,
+// against 3.1 ms at three or four CTAs per SM (80 / 64 registers, spills)
+// and 3.77 ms for one group per warp (the per-group work each lane repeats
+// is then paid once per group instead of once per two).
 
 struct QuantParams {
   const __half* w;       // fp16 [N][K]
@@ -55,23 +60,26 @@ struct QuantParams {
   int N, K, G, rounds;
 };
 
-__device__ __forceinline__ double warp_sum(double v) {
+// Sum over the 16 lanes of this lane's group (xor butterfly within the half).
+__device__ __forceinline__ double group_sum(double v) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  for (int o = kGroupLanes / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// Two warp sums at once (lanes 0-15 reduce a, lanes 16-31 reduce b, then
-// both are broadcast).  Only for sums that are exact in any order: sums of
-// +-fp16 weights, whose partial sums are multiples of 2^-24 below 2^23.
-__device__ __forceinline__ void warp_sum2_exact(double a, double b, double& sa, double& sb) {
-  const bool hi = (threadIdx.x & 16) != 0;
+// Two group sums at once (lanes 0-7 of the half reduce a, lanes 8-15 reduce
+// b, then both are broadcast within the half).  Only for sums that are exact
+// in any order: sums of +-fp16 weights, whose partial sums are multiples of
+// 2^-24 below 2^23.
+__device__ __forceinline__ void group_sum2_exact(double a, double b, double& sa, double& sb) {
+  const bool hi = (threadIdx.x & 8) != 0;
   double keep = hi ? b : a;
-  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 16);
+  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 8);
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-  sa = __shfl_sync(0xffffffffu, keep, 0);
-  sb = __shfl_sync(0xffffffffu, keep, 16);
+  for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  const int base = threadIdx.x & 16;
+  sa = __shfl_sync(0xffffffffu, keep, base);
+  sb = __shfl_sync(0xffffffffu, keep, base + 8);
 }
 
 __device__ __forceinline__ double signed_val(bool plus, double a) { return plus ? a : -a; }
@@ -222,13 +230,23 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
   if constexpr (M >= 2) solve_general<M>(G, r, x);
 }
 
-// Ballot words of the first P planes: P[i][s] = plane i, columns 32 s..32 s + 31.
+// Canonical words of plane i of this lane's group: word t = columns
+// 32 t..32 t + 31 = slots 2t (low half) and 2t + 1 (high half), the group's
+// 16 bits of each ballot picked by one byte permute.
+__device__ __forceinline__ void plane_word(const unsigned (&code)[kSlots], int i,
+                                           uint32_t (&cw)[4]) {
+  const uint32_t sel = (threadIdx.x & 16) ? 0x7632u : 0x5410u;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t lo = __ballot_sync(0xffffffffu, (code[2 * t] >> i) & 1u);
+    const uint32_t hi = __ballot_sync(0xffffffffu, (code[2 * t + 1] >> i) & 1u);
+    cw[t] = __byte_perm(lo, hi, sel);
+  }
+}
 template <int P>
-__device__ __forceinline__ void plane_words(const unsigned (&code)[4], uint32_t (&pw)[P][4]) {
+__device__ __forceinline__ void plane_words(const unsigned (&code)[kSlots], uint32_t (&pw)[P][4]) {
 #pragma unroll
-  for (int i = 0; i < P; ++i)
-#pragma unroll
-    for (int s = 0; s < 4; ++s) pw[i][s] = __ballot_sync(0xffffffffu, (code[s] >> i) & 1u);
+  for (int i = 0; i < P; ++i) plane_word(code, i, pw[i]);
 }
 
 __device__ __forceinline__ int dot_pm1(const uint32_t (&a)[4], const uint32_t (&b)[4]) {
@@ -241,25 +259,25 @@ __device__ __forceinline__ int sum_pm1(const uint32_t (&a)[4]) {
 
 // Exact sums sum(b_i w) of the first P planes, i = 0..P-1.
 template <int P>
-__device__ __forceinline__ void signed_sums(const double (&w)[4], const unsigned (&code)[4],
+__device__ __forceinline__ void signed_sums(const double (&w)[kSlots], const unsigned (&code)[kSlots],
                                             double (&S)[P]) {
   double t[P];
 #pragma unroll
   for (int i = 0; i < P; ++i) {
     t[i] = 0.0;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) t[i] += signed_val((code[s] >> i) & 1u, w[s]);
+    for (int s = 0; s < kSlots; ++s) t[i] += signed_val((code[s] >> i) & 1u, w[s]);
   }
 #pragma unroll
-  for (int i = 0; i + 1 < P; i += 2) warp_sum2_exact(t[i], t[i + 1], S[i], S[i + 1]);
-  if constexpr (P % 2 == 1) S[P - 1] = warp_sum(t[P - 1]);
+  for (int i = 0; i + 1 < P; i += 2) group_sum2_exact(t[i], t[i + 1], S[i], S[i + 1]);
+  if constexpr (P % 2 == 1) S[P - 1] = group_sum(t[P - 1]);
 }
 
 // Joint least squares for (z, alpha_1..alpha_P): columns [ones, b_1..b_P],
 // right-hand sides sum(w) and sum(b_i w).
 template <int P>
-__device__ __forceinline__ void lsq_with_offset(const double (&w)[4], double sumw,
-                                                const unsigned (&code)[4], double (&alpha)[P],
+__device__ __forceinline__ void lsq_with_offset(const double (&w)[kSlots], double sumw,
+                                                const unsigned (&code)[kSlots], double (&alpha)[P],
                                                 double& z) {
   uint32_t pw[P][4];
   plane_words<P>(code, pw);
@@ -284,8 +302,8 @@ __device__ __forceinline__ void lsq_with_offset(const double (&w)[4], double sum
 // Least squares for alpha_1..alpha_P with z fixed: columns [b_1..b_P],
 // right-hand sides sum(b_i (w - z)) = sum(b_i w) - z sum(b_i).
 template <int P>
-__device__ __forceinline__ void lsq_fixed_offset(const double (&w)[4], double z,
-                                                 const unsigned (&code)[4], double (&alpha)[P]) {
+__device__ __forceinline__ void lsq_fixed_offset(const double (&w)[kSlots], double z,
+                                                 const unsigned (&code)[kSlots], double (&alpha)[P]) {
   uint32_t pw[P][4];
   plane_words<P>(code, pw);
   int G[P][P];
@@ -310,14 +328,14 @@ __device__ __forceinline__ double code_value(const double (&alpha)[P], double z,
 }
 
 template <int P>
-__device__ __forceinline__ void nearest_codes(const double (&w)[4], const double (&alpha)[P],
-                                              double z, unsigned (&code)[4]) {
+__device__ __forceinline__ void nearest_codes(const double (&w)[kSlots], const double (&alpha)[P],
+                                              double z, unsigned (&code)[kSlots]) {
   constexpr int C = 1 << P;
   double v[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) v[c] = code_value<P>(alpha, z, (unsigned)c);
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
+  for (int s = 0; s < kSlots; ++s) {
     unsigned best = 0;
     double be = fabs(w[s] - v[0]);
 #pragma unroll
@@ -333,37 +351,40 @@ __device__ __forceinline__ void nearest_codes(const double (&w)[4], const double
 }
 
 template <int P>
-__device__ __forceinline__ double group_sse(const double (&w)[4], const double (&alpha)[P],
-                                            double z, const unsigned (&code)[4]) {
+__device__ __forceinline__ double group_sse(const double (&w)[kSlots], const double (&alpha)[P],
+                                            double z, const unsigned (&code)[kSlots]) {
   double t = 0.0;
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
+  for (int s = 0; s < kSlots; ++s) {
     const double e = w[s] - code_value<P>(alpha, z, code[s]);
     t += e * e;
   }
-  return warp_sum(t);
+  return group_sum(t);
 }
 
-// alpha^(P) of the group rounded to fp16 (nearest even), and its error.
+// alpha^(P) of the group rounded to fp16 (nearest even), and its error;
+// j = the lane within the group, valid = the half holds a real group.
 template <int P>
-__device__ __forceinline__ void store_scales(const QuantParams& q, long long gid, int lane,
-                                             const double (&alpha)[P], double sse, int p_L) {
+__device__ __forceinline__ void store_scales(const QuantParams& q, long long gid, int j,
+                                             bool valid, const double (&alpha)[P], double sse,
+                                             int p_L) {
+  if (!valid) return;
   __half* a = q.alpha[P - 1] + gid * P;
 #pragma unroll
   for (int i = 0; i < P; ++i)
-    if (lane == i) a[i] = __double2half(alpha[i]);
-  if (q.sse && lane == 0) q.sse[(long long)(P - p_L) * q.groups + gid] = sse;
+    if (j == i) a[i] = __double2half(alpha[i]);
+  if (q.sse && j == 0) q.sse[(long long)(P - p_L) * q.groups + gid] = sse;
 }
 
 // Base precision PL: greedy start, refinement rounds, final refit.
 template <int PL>
-__device__ __forceinline__ void base_precision(const QuantParams& q, const double (&w)[4],
-                                               double sumw, unsigned (&code)[4],
+__device__ __forceinline__ void base_precision(const QuantParams& q, const double (&w)[kSlots],
+                                               double sumw, unsigned (&code)[kSlots],
                                                double (&alpha)[PL], double& z) {
   z = sumw / kQuantGroup;  // exact: the sum is exact, 128 a power of two
-  double r[4];
+  double r[kSlots];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
+  for (int s = 0; s < kSlots; ++s) {
     r[s] = w[s] - z;
     code[s] = 0;
   }
@@ -371,20 +392,19 @@ __device__ __forceinline__ void base_precision(const QuantParams& q, const doubl
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
 #pragma unroll
-    for (int s = 0; s < 4; ++s) code[s] |= (r[s] >= 0.0 ? 1u : 0u) << i;  // b_i = sign(r)
-#pragma unroll
-    for (int s = 0; s < 4; ++s) pw[i][s] = __ballot_sync(0xffffffffu, (code[s] >> i) & 1u);
+    for (int s = 0; s < kSlots; ++s) code[s] |= (r[s] >= 0.0 ? 1u : 0u) << i;  // b_i = sign(r)
+    plane_word(code, i, pw[i]);
     // <b_i, r> = sum(b_i w) - z sum(b_i) - sum_j alpha_j <b_i, b_j>, left to right
     double t = 0.0;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) t += signed_val((code[s] >> i) & 1u, w[s]);
-    t = warp_sum(t);
+    for (int s = 0; s < kSlots; ++s) t += signed_val((code[s] >> i) & 1u, w[s]);
+    t = group_sum(t);
     t = __dsub_rn(t, __dmul_rn(z, (double)sum_pm1(pw[i])));
 #pragma unroll
     for (int j = 0; j < i; ++j) t = __dsub_rn(t, __dmul_rn(alpha[j], (double)dot_pm1(pw[i], pw[j])));
     const double a = t / kQuantGroup;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) r[s] = ((code[s] >> i) & 1u) ? r[s] - a : r[s] + a;
+    for (int s = 0; s < kSlots; ++s) r[s] = ((code[s] >> i) & 1u) ? r[s] - a : r[s] + a;
     alpha[i] = a;
   }
   for (int it = 0; it < q.rounds; ++it) {
@@ -397,12 +417,13 @@ __device__ __forceinline__ void base_precision(const QuantParams& q, const doubl
 // Expansion p -> p + 1: B_{p+1} = sign(R_p), then every scale refit with z
 // kept (shared offsets) or refit with it (q.zp: offsets per precision).
 template <int P, int PH, bool ZP>
-__device__ __forceinline__ void expand(const QuantParams& q, long long gid, int lane, int p_L,
-                                       const double (&w)[4], double sumw, double z,
-                                       unsigned (&code)[4], const double (&alpha)[P]) {
+__device__ __forceinline__ void expand(const QuantParams& q, long long gid, int j, bool valid,
+                                       int p_L,
+                                       const double (&w)[kSlots], double sumw, double z,
+                                       unsigned (&code)[kSlots], const double (&alpha)[P]) {
   if constexpr (P < PH) {
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       const double res = w[s] - code_value<P>(alpha, z, code[s]);
       code[s] |= (res >= 0.0 ? 1u : 0u) << P;
     }
@@ -410,46 +431,55 @@ __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int 
     double zn = z;
     if constexpr (ZP) {
       lsq_with_offset<P + 1>(w, sumw, code, next, zn);
-      if (lane == 0) q.zq[P][gid] = __double2half(zn);
+      if (valid && j == 0) q.zq[P][gid] = __double2half(zn);
     } else {
       lsq_fixed_offset<P + 1>(w, z, code, next);
     }
     const double e = q.sse ? group_sse<P + 1>(w, next, zn, code) : 0.0;
-    store_scales<P + 1>(q, gid, lane, next, e, p_L);
-    expand<P + 1, PH, ZP>(q, gid, lane, p_L, w, sumw, zn, code, next);
+    store_scales<P + 1>(q, gid, j, valid, next, e, p_L);
+    expand<P + 1, PH, ZP>(q, gid, j, valid, p_L, w, sumw, zn, code, next);
   }
 }
 
 template <int PL, int PH, bool ZP>
-__global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinBlocks) quantize_kernel(QuantParams q) {
-  const int lane = threadIdx.x & 31;
-  const long long gid = (long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
-  if (gid >= q.groups) return;  // uniform per warp
-  const long long n = gid / q.G;
-  const int g = (int)(gid - n * q.G);
+__global__ void __launch_bounds__(32 * kQuantWarps, 2) quantize_kernel(QuantParams q) {
+  const int j = threadIdx.x & (kGroupLanes - 1);
+  const long long gid0 = ((long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5)) * 2;
+  if (gid0 >= q.groups) return;  // uniform per warp
+  const long long gid = gid0 + ((threadIdx.x >> 4) & 1);
+  // the second half of the last warp may have no group: it computes on its
+  // partner's weights (every lane takes part in the ballots and shuffles)
+  // and stores nothing
+  const bool valid = gid < q.groups;
+  const long long gl = valid ? gid : gid0;
+  const long long n = gl / q.G;
+  const int g = (int)(gl - n * q.G);
   const __half* src = q.w + n * q.K + (long long)g * kQuantGroup;
-  double w[4];
+  double w[kSlots];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) w[s] = (double)__half2float(src[lane + 32 * s]);
-  const double sumw = warp_sum(((w[0] + w[1]) + w[2]) + w[3]);
+  for (int s = 0; s < kSlots; ++s) w[s] = (double)__half2float(src[j + kGroupLanes * s]);
+  double tw = 0.0;
+#pragma unroll
+  for (int s = 0; s < kSlots; ++s) tw += w[s];
+  const double sumw = group_sum(tw);  // exact in any order
 
-  unsigned code[4];
+  unsigned code[kSlots];
   double alpha[PL], z;
   base_precision<PL>(q, w, sumw, code, alpha, z);
   const double e = q.sse ? group_sse<PL>(w, alpha, z, code) : 0.0;
-  store_scales<PL>(q, gid, lane, alpha, e, PL);
-  if (lane == 0) (ZP ? q.zq[PL - 1] : q.z)[gid] = __double2half(z);
-  expand<PL, PH, ZP>(q, gid, lane, PL, w, sumw, z, code, alpha);
+  store_scales<PL>(q, gid, j, valid, alpha, e, PL);
+  if (valid && j == 0) (ZP ? q.zq[PL - 1] : q.z)[gid] = __double2half(z);
+  expand<PL, PH, ZP>(q, gid, j, valid, PL, w, sumw, z, code, alpha);
 
-  // planes: lane 4 i + s writes word s of plane i
+  // planes: lane 4 i + t of the group writes word t of plane i
   uint32_t pw[PH][4];
   plane_words<PH>(code, pw);
   const int KW = q.K / 32;
 #pragma unroll
   for (int i = 0; i < PH; ++i)
 #pragma unroll
-    for (int s = 0; s < 4; ++s)
-      if (lane == 4 * i + s) q.planes[((long long)i * q.N + n) * KW + 4 * g + s] = pw[i][s];
+    for (int t = 0; t < 4; ++t)
+      if (valid && j == 4 * i + t) q.planes[((long long)i * q.N + n) * KW + 4 * g + t] = pw[i][t];
 }
 
 using QuantKernel = void (*)(QuantParams);
@@ -508,7 +538,7 @@ bcq_status quantize_common(const uint16_t* w, int N, int K, int p_L, int p_H, in
   q.rounds = rounds;
   const QuantKernel fn = quantize_kernel_for(p_L, p_H, zq != nullptr);
   if (!fn) return BCQ_ERR_UNSUPPORTED;
-  const long long blocks = (q.groups + kQuantWarps - 1) / kQuantWarps;
+  const long long blocks = (q.groups + 2 * kQuantWarps - 1) / (2 * kQuantWarps);
   fn<<<(unsigned)blocks, 32 * kQuantWarps, 0, (cudaStream_t)stream>>>(q);
   return cudaGetLastError() == cudaSuccess ? BCQ_OK : BCQ_ERR_CUDA;
 }

@@ -1,4 +1,5 @@
-// bcq_quantize.cu -- the offline multi-precision BCQ quantiser (bcq_quantize).
+// bcq_quantize.cu -- the offline multi-precision BCQ quantiser (bcq_quantize,
+// and bcq_quantize_zp for offsets per precision).
 //
 // "AnyBCQ ..." (Paper-Notes page), "关键设计 / 渐进式精度扩展": at the base
 // precision p_L the codes start greedy and are refined by alternating a
@@ -28,7 +29,8 @@
 //     enumeration order on ties (code c: b_i = +1 where bit i of c is set).
 // The greedy start peels b = sign(r), alpha = <b, r> / 128 off r = w - mean(w);
 // sign(0) = +1.  z is fitted jointly with the base precision's scales and
-// kept for the expansions.
+// kept for the expansions (bcq_quantize_zp: refit with the scales at every
+// expansion, giving z^(p) per precision).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -43,11 +45,12 @@ constexpr int kQuantGroup = 128;
 constexpr int kGroupLanes = 16;                       // lanes per group (half a warp)
 constexpr int kSlots = kQuantGroup / kGroupLanes;     // weights per lane
 constexpr int kQuantWarps = 8;                        // warps per CTA (two groups each)
-// Two CTAs (16 warps, 32 groups) per SM: 128 registers a thread and no
-// spills.  Measured on a 14336 x 4096 weight (p_L = 2 -> p_H = 4): 3.07 ms,
+// kQuantMinCtas: two CTAs (16 warps, 32 groups) per SM, 128 registers a
+// thread and no spills.  Measured on a 14336 x 4096 weight (p_L = 2 -> p_H = 4): 3.07 ms,
 // against 3.1 ms at three or four CTAs per SM (80 / 64 registers, spills)
 // and 3.77 ms for one group per warp (the per-group work each lane repeats
 // is then paid once per group instead of once per two).
+constexpr int kQuantMinCtas = 2;
 
 struct QuantParams {
   const __half* w;       // fp16 [N][K]
@@ -442,7 +445,7 @@ __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int 
 }
 
 template <int PL, int PH, bool ZP>
-__global__ void __launch_bounds__(32 * kQuantWarps, 2) quantize_kernel(QuantParams q) {
+__global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinCtas) quantize_kernel(QuantParams q) {
   const int j = threadIdx.x & (kGroupLanes - 1);
   const long long gid0 = ((long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5)) * 2;
   if (gid0 >= q.groups) return;  // uniform per warp

@@ -159,7 +159,11 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
   const size_t part_stride = (size_t)RB * kRowBlock;
   const size_t kstride = (size_t)Mrows * part_stride;  // one K-block of partials
   const bool live = *abort_flag == 0;
-  int task = 0, mine = warp;  // tasks dealt round-robin: no division
+  // Tasks are dealt round-robin (no division), starting at the first warp of
+  // the second team: the first team takes the odd group out of an odd
+  // number, so the second team is done first and polls earlier (measured:
+  // M = 1 calls 1-3 % faster than dealing from warp 0).
+  int task = 0, mine = warp ^ (nwarps >> 1);
   for (int kb = R.kb0; kb <= R.kb_last && live; ++kb) {
     const int a = kb == R.kb0 ? R.u0 - kb * RB : 0;
     const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;

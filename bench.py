@@ -431,7 +431,7 @@ def run_quantizer(args, dev, rows=N_OUT):
     assert api.device_error(stream) == api.BCQ_OK
     groups = rows * G
     out = {"workload": f"bcq_quantize fp16 {rows}x{K_IN}, g=128, p_L=2 -> p_H=4, 20 rounds "
-                       f"({groups} groups, half a warp each)",
+                       f"({groups} groups, a quarter warp each)",
            "ms": round(ms, 4), "groups_per_s": round(groups / (ms * 1e-3), 1),
            "weights_GBps": round(rows * K_IN * 2 / (ms * 1e-3) / 1e9, 2),
            "launches_per_call": 1, "reps": reps, "l2": "flushed before every call"}

@@ -8,18 +8,18 @@
 // scale of alpha^(p+1) by least squares.  "训练策略": asymmetric, group 128,
 // 20 refinement rounds.
 //
-// Half a warp quantises one 128-weight group (two groups per warp, so the
-// per-group work every lane repeats -- Gram counts, the solve, candidate
-// values -- is shared by two groups); lane j of a half holds columns
-// j + 16 s, s = 0..7, so the ballot of plane bit i over slot s carries 16
-// columns of each half's group, and one byte permute of two ballots gives a
-// canonical 32-column plane word.  Everything is fp64 (the weights are fp16,
+// A quarter warp (8 lanes) quantises one 128-weight group (four groups per
+// warp, so the per-group work every lane repeats -- Gram counts, the solve,
+// candidate values -- is shared by four groups); lane j of a group holds
+// columns j + 8 s, s = 0..15, so the ballot of plane bit i over slot s
+// carries 8 columns of each of the warp's groups, and three byte permutes of
+// four ballots give a canonical 32-column plane word.  Everything is fp64 (the weights are fp16,
 // widened exactly).  Per step:
 //   * the Gram matrix of the +-1 planes (and the all-ones column of z) is
 //     integer-valued and comes exactly from popcounts of the plane words;
-//   * right-hand sides are sums over the half (xor butterfly: every lane ends
-//     with the same bits, since a + b == b + a), so every lane solves the same
-//     system and holds the same scales without a broadcast;
+//   * right-hand sides are sums over the group's lanes (xor butterfly: every
+//     lane ends with the same bits, since a + b == b + a), so every lane
+//     solves the same system and holds the same scales without a broadcast;
 //   * columns exactly dependent on the columns before them (a plane equal to
 //     another, to its negation or to the all-ones column, or any exact linear
 //     dependence) get scale 0; the normal equations of the kept columns are
@@ -42,14 +42,14 @@ namespace bcq {
 namespace {
 
 constexpr int kQuantGroup = 128;
-constexpr int kGroupLanes = 16;                       // lanes per group (half a warp)
+constexpr int kGroupLanes = 8;                        // lanes per group (quarter warp)
 constexpr int kSlots = kQuantGroup / kGroupLanes;     // weights per lane
-constexpr int kQuantWarps = 8;                        // warps per CTA (two groups each)
-// kQuantMinCtas: two CTAs (16 warps, 32 groups) per SM, 128 registers a
-// thread and no spills.  Measured on a 14336 x 4096 weight (p_L = 2 -> p_H = 4): 3.07 ms,
-// against 3.1 ms at three or four CTAs per SM (80 / 64 registers, spills)
-// and 3.77 ms for one group per warp (the per-group work each lane repeats
-// is then paid once per group instead of once per two).
+constexpr int kQuantWarps = 8;                        // warps per CTA (four groups each)
+// kQuantMinCtas: two CTAs (16 warps, 64 groups) per SM, 128 registers a
+// thread.  Measured on a 14336 x 4096 weight (p_L = 2 -> p_H = 4): 2.53 ms
+// with four groups per warp, against 2.83 ms at one CTA per SM (230
+// registers), 3.07 ms with two groups per warp and 3.77 ms with one (the
+// per-group work each lane repeats is paid once per warp).
 constexpr int kQuantMinCtas = 2;
 
 struct QuantParams {
@@ -63,26 +63,26 @@ struct QuantParams {
   int N, K, G, rounds;
 };
 
-// Sum over the 16 lanes of this lane's group (xor butterfly within the half).
+// Sum over the 8 lanes of this lane's group (xor butterfly within the group).
 __device__ __forceinline__ double group_sum(double v) {
 #pragma unroll
   for (int o = kGroupLanes / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// Two group sums at once (lanes 0-7 of the half reduce a, lanes 8-15 reduce
-// b, then both are broadcast within the half).  Only for sums that are exact
-// in any order: sums of +-fp16 weights, whose partial sums are multiples of
-// 2^-24 below 2^23.
+// Two group sums at once (lanes 0-3 of the group reduce a, lanes 4-7 reduce
+// b, then both are broadcast within the group).  Only for sums that are
+// exact in any order: sums of +-fp16 weights, whose partial sums are
+// multiples of 2^-24 below 2^23.
 __device__ __forceinline__ void group_sum2_exact(double a, double b, double& sa, double& sb) {
-  const bool hi = (threadIdx.x & 8) != 0;
+  const bool hi = (threadIdx.x & 4) != 0;
   double keep = hi ? b : a;
-  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 8);
+  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 4);
 #pragma unroll
-  for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-  const int base = threadIdx.x & 16;
+  for (int o = 2; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  const int base = threadIdx.x & 24;
   sa = __shfl_sync(0xffffffffu, keep, base);
-  sb = __shfl_sync(0xffffffffu, keep, base + 8);
+  sb = __shfl_sync(0xffffffffu, keep, base + 4);
 }
 
 __device__ __forceinline__ double signed_val(bool plus, double a) { return plus ? a : -a; }
@@ -234,16 +234,19 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
 }
 
 // Canonical words of plane i of this lane's group: word t = columns
-// 32 t..32 t + 31 = slots 2t (low half) and 2t + 1 (high half), the group's
-// 16 bits of each ballot picked by one byte permute.
+// 32 t..32 t + 31 = slots 4t..4t + 3 (bytes 0..3), the group's byte of each
+// ballot picked by byte permutes.
 __device__ __forceinline__ void plane_word(const unsigned (&code)[kSlots], int i,
                                            uint32_t (&cw)[4]) {
-  const uint32_t sel = (threadIdx.x & 16) ? 0x7632u : 0x5410u;
+  const uint32_t gq = (threadIdx.x >> 3) & 3u;
+  const uint32_t sel = gq | ((gq + 4u) << 4);
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    const uint32_t lo = __ballot_sync(0xffffffffu, (code[2 * t] >> i) & 1u);
-    const uint32_t hi = __ballot_sync(0xffffffffu, (code[2 * t + 1] >> i) & 1u);
-    cw[t] = __byte_perm(lo, hi, sel);
+    const uint32_t b0 = __ballot_sync(0xffffffffu, (code[4 * t] >> i) & 1u);
+    const uint32_t b1 = __ballot_sync(0xffffffffu, (code[4 * t + 1] >> i) & 1u);
+    const uint32_t b2 = __ballot_sync(0xffffffffu, (code[4 * t + 2] >> i) & 1u);
+    const uint32_t b3 = __ballot_sync(0xffffffffu, (code[4 * t + 3] >> i) & 1u);
+    cw[t] = __byte_perm(__byte_perm(b0, b1, sel), __byte_perm(b2, b3, sel), 0x5410u);
   }
 }
 template <int P>
@@ -366,7 +369,7 @@ __device__ __forceinline__ double group_sse(const double (&w)[kSlots], const dou
 }
 
 // alpha^(P) of the group rounded to fp16 (nearest even), and its error;
-// j = the lane within the group, valid = the half holds a real group.
+// j = the lane within the group, valid = the lanes hold a real group.
 template <int P>
 __device__ __forceinline__ void store_scales(const QuantParams& q, long long gid, int j,
                                              bool valid, const double (&alpha)[P], double sse,
@@ -447,12 +450,12 @@ __device__ __forceinline__ void expand(const QuantParams& q, long long gid, int 
 template <int PL, int PH, bool ZP>
 __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinCtas) quantize_kernel(QuantParams q) {
   const int j = threadIdx.x & (kGroupLanes - 1);
-  const long long gid0 = ((long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5)) * 2;
+  const long long gid0 = ((long long)blockIdx.x * kQuantWarps + (threadIdx.x >> 5)) * 4;
   if (gid0 >= q.groups) return;  // uniform per warp
-  const long long gid = gid0 + ((threadIdx.x >> 4) & 1);
-  // the second half of the last warp may have no group: it computes on its
-  // partner's weights (every lane takes part in the ballots and shuffles)
-  // and stores nothing
+  const long long gid = gid0 + ((threadIdx.x >> 3) & 3);
+  // the last warp may hold fewer than four groups: a lane without a group
+  // computes on the warp's first group (every lane takes part in the
+  // ballots and shuffles) and stores nothing
   const bool valid = gid < q.groups;
   const long long gl = valid ? gid : gid0;
   const long long n = gl / q.G;
@@ -474,7 +477,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinCtas) quantize_kern
   if (valid && j == 0) (ZP ? q.zq[PL - 1] : q.z)[gid] = __double2half(z);
   expand<PL, PH, ZP>(q, gid, j, valid, PL, w, sumw, z, code, alpha);
 
-  // planes: lane 4 i + t of the group writes word t of plane i
+  // planes: lane (4 i + t) mod 8 of the group writes word t of plane i
   uint32_t pw[PH][4];
   plane_words<PH>(code, pw);
   const int KW = q.K / 32;
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps, kQuantMinCtas) quantize_kern
   for (int i = 0; i < PH; ++i)
 #pragma unroll
     for (int t = 0; t < 4; ++t)
-      if (valid && j == 4 * i + t) q.planes[((long long)i * q.N + n) * KW + 4 * g + t] = pw[i][t];
+      if (valid && j == ((4 * i + t) & 7)) q.planes[((long long)i * q.N + n) * KW + 4 * g + t] = pw[i][t];
 }
 
 using QuantKernel = void (*)(QuantParams);
@@ -541,7 +544,7 @@ bcq_status quantize_common(const uint16_t* w, int N, int K, int p_L, int p_H, in
   q.rounds = rounds;
   const QuantKernel fn = quantize_kernel_for(p_L, p_H, zq != nullptr);
   if (!fn) return BCQ_ERR_UNSUPPORTED;
-  const long long blocks = (q.groups + 2 * kQuantWarps - 1) / (2 * kQuantWarps);
+  const long long blocks = (q.groups + 4 * kQuantWarps - 1) / (4 * kQuantWarps);
   fn<<<(unsigned)blocks, 32 * kQuantWarps, 0, (cudaStream_t)stream>>>(q);
   return cudaGetLastError() == cudaSuccess ? BCQ_OK : BCQ_ERR_CUDA;
 }

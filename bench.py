@@ -342,9 +342,48 @@ def run_gpu(args, rank, world, local_rank):
         del scopies, sbase
         assert api.device_error(stream) == api.BCQ_OK
 
+    # offsets per precision (bcq_gemm_zp): M = 1 at each precision and one
+    # two-row launch with two precisions (row 1's offsets read apart), against
+    # the same calls with shared offsets
+    zp = None
+    if not args.cases:
+        rng = np.random.default_rng(args.seed + 3)
+        zq = {q: rng.normal(0.0, 0.005, size=prob.z.shape).astype(np.float16) for q in PRECISIONS}
+        zbase = api.BcqWeights.from_canonical(prob.planes, prob.alphas, zq, device=dev)
+        zcopies = [zbase] + [api.BcqWeights(packed=c.packed, alphas=c.alphas, z=None, N=c.N, K=c.K,
+                                            p_H=c.p_H, zq={q: v.clone() for q, v in zbase.zq.items()})
+                             for c in copies[1:]]
+        zp = {"weights": "the bench weight with one offset array per precision"}
+        single = {(c["p"], c["M"]): c["us"] for c in per_case}
+        for label, M, pr in [("M1p2", 1, [2]), ("M1p3", 1, [3]), ("M1p4", 1, [4]),
+                             ("M2p2p4", 2, [2, 4])]:
+            def zone(M=M, pr=pr):
+                for w in zcopies:
+                    w.gemm(x[:M], p_row=pr, out=ys[M], stream=stream)
+            with torch.cuda.stream(stream):
+                zone()
+            stream.synchronize()
+            g = capture(zone)
+            with torch.cuda.stream(stream):
+                g.replay()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+            b.synchronize()
+            us = a.elapsed_time(b) * 1000.0 / (reps * R)
+            shared = single.get((pr[0], M)) if len(set(pr)) == 1 else None
+            zp[label] = {"us": round(us, 3), "us_shared_offsets": shared}
+            del g
+        del zcopies, zbase
+        assert api.device_error(stream) == api.BCQ_OK
+
     result = {"ms_total": ms_total, "bytes_step": bytes_step, "R": R,
               "per_copy_bytes": per_copy, "launches_per_step": launches_per_step,
-              "per_case": per_case, "clocks": clocks, "stacked": stacked}
+              "per_case": per_case, "clocks": clocks, "stacked": stacked,
+              "per_precision_offsets": zp}
 
     # end to end through bcq_gemm_host: pinned host x and y, copies inside
     # the timed region.  Calls alternate between two streams, each with its
@@ -405,9 +444,16 @@ def run_quantizer(args, dev, rows=N_OUT):
     stream = torch.cuda.Stream(device=dev)
     arr = api._alpha_array(alphas)
 
-    def call():
-        st = api.lib().bcq_quantize(api._ptr(w), rows, K_IN, 2, P_H, 20, api._ptr(planes), arr,
-                                    api._ptr(z), None, api._stream(stream))
+    zq = {p: torch.empty((rows, G), dtype=torch.float16, device=dev) for p in PRECISIONS}
+    zarr = api._alpha_array(zq, "z")
+
+    def call(per_precision=False):
+        if per_precision:
+            st = api.lib().bcq_quantize_zp(api._ptr(w), rows, K_IN, 2, P_H, 20, api._ptr(planes),
+                                           arr, zarr, None, api._stream(stream))
+        else:
+            st = api.lib().bcq_quantize(api._ptr(w), rows, K_IN, 2, P_H, 20, api._ptr(planes), arr,
+                                        api._ptr(z), None, api._stream(stream))
         if st != api.BCQ_OK:
             raise api.BcqError(st, "bcq_quantize")
 
@@ -428,13 +474,29 @@ def run_quantizer(args, dev, rows=N_OUT):
         b.synchronize()
         ms += a.elapsed_time(b)
     ms /= reps
+    # the per-precision-offset variant (bcq_quantize_zp), same method
+    with torch.cuda.stream(stream):
+        call(True)
+    ms_zp = 0.0
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call(True)
+            b.record(stream)
+        b.synchronize()
+        ms_zp += a.elapsed_time(b)
+    ms_zp /= reps
     assert api.device_error(stream) == api.BCQ_OK
     groups = rows * G
     out = {"workload": f"bcq_quantize fp16 {rows}x{K_IN}, g=128, p_L=2 -> p_H=4, 20 rounds "
                        f"({groups} groups, a quarter warp each)",
            "ms": round(ms, 4), "groups_per_s": round(groups / (ms * 1e-3), 1),
            "weights_GBps": round(rows * K_IN * 2 / (ms * 1e-3) / 1e9, 2),
-           "launches_per_call": 1, "reps": reps, "l2": "flushed before every call"}
+           "launches_per_call": 1, "reps": reps, "l2": "flushed before every call",
+           "ms_per_precision_offsets": round(ms_zp, 4)}
     # issue-bound fp64/integer code: achieved warp instructions per second
     # (ncu's count per group x groups / event time) against the issue peak
     # of 148 SMs x 4 schedulers x one warp instruction per cycle at 1965 MHz
@@ -618,6 +680,8 @@ def main():
     line["roofline"]["by_kernel"] = by_kernel
     if res.get("stacked"):
         line["stacked_gate_up"] = res["stacked"]
+    if res.get("per_precision_offsets"):
+        line["per_precision_offsets"] = res["per_precision_offsets"]
     m1 = [c for c in res["per_case"] if c["M"] == 1]
     line["headline_m1"] = {f"p{c['p']}": {"us": c["us"], "GBps": c["GBps"],
                                           "frac": round(c["GBps"] / peak, 4)} for c in m1}

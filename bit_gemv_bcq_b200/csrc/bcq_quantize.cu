@@ -166,9 +166,30 @@ __device__ __forceinline__ void solve_general(const int (&G)[M][M], const double
   for (int j = 0; j < M; ++j) x[j] = xs[j];
 }
 
+// Determinant of the 4x4 minor of a 5x5 integer matrix without row SR and
+// column SC, by Laplace expansion over the 2x2 minors of its first two rows
+// (s) and last two rows (c).  |G| <= 128: 2x2 minors below 2^15, the result
+// below 2^33 (64-bit).
+template <int SR, int SC>
+__device__ __forceinline__ long long minor4(const int (&G)[5][5]) {
+  int a[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) a[r][c] = G[r < SR ? r : r + 1][c < SC ? c : c + 1];
+  const int s0 = a[0][0] * a[1][1] - a[1][0] * a[0][1], s1 = a[0][0] * a[1][2] - a[1][0] * a[0][2],
+            s2 = a[0][0] * a[1][3] - a[1][0] * a[0][3], s3 = a[0][1] * a[1][2] - a[1][1] * a[0][2],
+            s4 = a[0][1] * a[1][3] - a[1][1] * a[0][3], s5 = a[0][2] * a[1][3] - a[1][2] * a[0][3];
+  const int c5 = a[2][2] * a[3][3] - a[3][2] * a[2][3], c4 = a[2][1] * a[3][3] - a[3][1] * a[2][3],
+            c3 = a[2][1] * a[3][2] - a[3][1] * a[2][2], c2 = a[2][0] * a[3][3] - a[3][0] * a[2][3],
+            c1 = a[2][0] * a[3][2] - a[3][0] * a[2][2], c0 = a[2][0] * a[3][1] - a[3][0] * a[2][1];
+  return (long long)s0 * c5 - (long long)s1 * c4 + (long long)s2 * c3 + (long long)s3 * c2 -
+         (long long)s4 * c1 + (long long)s5 * c0;
+}
+
 // Least squares on M columns with integer Gram matrix G and right-hand
 // sides r, by Cramer's rule with the exact adjugate; columns dependent on
-// earlier ones get 0.  Full-rank systems of 1 to 4 columns (every leading
+// earlier ones get 0.  Full-rank systems of 1 to 5 columns (every leading
 // principal minor non-zero) take closed forms; the rest solve_general.
 template <int M>
 __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (&r)[M],
@@ -227,6 +248,43 @@ __device__ __forceinline__ void solve_exact(const int (&G)[M][M], const double (
       x[1] = cramer_row<4>(r1, r, det);
       x[2] = cramer_row<4>(r2, r, det);
       x[3] = cramer_row<4>(r3, r, det);
+      return;
+    }
+  }
+  else if constexpr (M == 5) {
+    // adj[i][j] = (-1)^(i+j) det(G without row j, column i); G symmetric, so
+    // adj is symmetric: 15 distinct 4x4 minors (below 2^33)
+    long long A[5][5];
+    A[0][0] = minor4<0, 0>(G);
+    A[0][1] = -minor4<1, 0>(G);
+    A[0][2] = minor4<2, 0>(G);
+    A[0][3] = -minor4<3, 0>(G);
+    A[0][4] = minor4<4, 0>(G);
+    A[1][1] = minor4<1, 1>(G);
+    A[1][2] = -minor4<2, 1>(G);
+    A[1][3] = minor4<3, 1>(G);
+    A[1][4] = -minor4<4, 1>(G);
+    A[2][2] = minor4<2, 2>(G);
+    A[2][3] = -minor4<3, 2>(G);
+    A[2][4] = minor4<4, 2>(G);
+    A[3][3] = minor4<3, 3>(G);
+    A[3][4] = -minor4<4, 3>(G);
+    A[4][4] = minor4<4, 4>(G);
+#pragma unroll
+    for (int i = 1; i < 5; ++i)
+#pragma unroll
+      for (int j = 0; j < i; ++j) A[i][j] = A[j][i];
+    long long det = 0;  // expansion along row 0: sum_j G[0][j] adj[j][0]
+#pragma unroll
+    for (int j = 0; j < 5; ++j) det += (long long)G[0][j] * A[j][0];
+    // leading minors: G[0][0] = 128, 2x2, 3x3, 4x4 (= adj[4][4]), det
+    const long long d2 = (long long)G[0][0] * G[1][1] - (long long)G[0][1] * G[1][0];
+    const long long d3 = (long long)G[0][0] * ((long long)G[1][1] * G[2][2] - (long long)G[1][2] * G[2][1]) -
+                         (long long)G[0][1] * ((long long)G[1][0] * G[2][2] - (long long)G[1][2] * G[2][0]) +
+                         (long long)G[0][2] * ((long long)G[1][0] * G[2][1] - (long long)G[1][1] * G[2][0]);
+    if (d2 != 0 && d3 != 0 && A[4][4] != 0 && det != 0) {
+#pragma unroll
+      for (int a = 0; a < 5; ++a) x[a] = cramer_row<5>(A[a], r, det);
       return;
     }
   }

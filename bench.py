@@ -146,9 +146,9 @@ class ClockSampler:
 
     def start(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
-            self.f = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="bcq_clocks_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-i", str(self.dev), "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
@@ -180,6 +180,10 @@ class ClockSampler:
                 for name, val in zip(names, parts[5:9]):
                     if val.lower().startswith("active"):
                         reasons.add(name)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sms:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),

@@ -19,7 +19,7 @@
  *     section "核心思路：修正项只用 +1 和 −1": a +-1 vector times x is a signed
  *     sum of the entries of x.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   bit value 1 -> +1 and 0 -> -1; bit j of 32-bit word w holds column 32w+j
  *   (LSB first); canonical planes are [p_H][N][K/32]; alpha for precision q is
  *   its own fp16 array [N][G][q]; one offset z[N][G] shared by all precisions;

@@ -540,8 +540,13 @@ def launches_per_call(M):
     return -(-M // 16) if M >= MMA_MIN_ROWS else -(-M // 2)
 
 
-def kernel_of(M):
-    return "gemv_mma_kernel" if M >= MMA_MIN_ROWS else "gemv_lut_kernel"
+LUT4_MIN_BITS = 3  # bcq_gemm's four-row lookup launches: 3-4 rows of >= 3 bits
+
+
+def kernel_of(M, p):
+    if M < MMA_MIN_ROWS or (M <= 4 and p >= LUT4_MIN_BITS):
+        return "gemv_lut_kernel"
+    return "gemv_mma_kernel"
 
 
 # ------------------------------------------------------------- CPU oracle arm
@@ -660,8 +665,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
                      "peak_kind": peak_kind, "traffic": None,
-                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 2, "
-                               "gemv_mma_kernel for M >= 3)"},
+                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 2 and for "
+                               "M = 4 at p >= 3, gemv_mma_kernel for the other batches)"},
         "per_call": res["per_case"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
@@ -674,7 +679,7 @@ def main():
         line["roofline"]["traffic_source"] = tr["source"]
     by_kernel = {}
     for c in res["per_case"]:
-        k = by_kernel.setdefault(kernel_of(c["M"]), {"us": 0.0, "bytes": 0})
+        k = by_kernel.setdefault(kernel_of(c["M"], c["p"]), {"us": 0.0, "bytes": 0})
         k["us"] += c["us"]
         k["bytes"] += c["bytes"]
     for name, k in by_kernel.items():

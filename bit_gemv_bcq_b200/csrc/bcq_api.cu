@@ -26,7 +26,7 @@ constexpr int kDefaultMmaMinRows = 3;
 
 // Kernels: the lookup-table kernel (one or two rows), and for batches a
 // tensor-core kernel: mma.sync (default) or tcgen05 (BCQ_MMA_KIND=tcgen05).
-enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2 };
+enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2, kPathLut4 = 3 };
 
 int batch_path() {
   const char* v = std::getenv("BCQ_MMA_KIND");
@@ -122,7 +122,7 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
     return path == kPathUmma      ? (NN == kMmaRows ? umma_dyn_bytes<16>(d, P)
                                                      : umma_dyn_bytes<64>(d, P))
            : path == kPathMmaSync ? mma_dyn_bytes(d, P)
-                                  : gemv_dyn_bytes(d, P);
+                                  : gemv_dyn_bytes(d, P, M);
   };
   const long long RB = (long long)row_blocks(N);
   const long long KB = (long long)k_blocks(K);
@@ -278,6 +278,14 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
   const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
   if (M >= mma_min) {
     const int path = batch_path();
+    // batches of 3-4 rows of one precision of at least 3 bits: one lookup
+    // launch over two pair tables (measured on 14336 x 4096: p = 3 / 4 in
+    // 26.1 / 29.7 us against 29.6 / 36.6 us on the tensor-core kernel; at
+    // p = 2 building two tables costs more than the shorter loop saves:
+    // 23.8 against 22.9 us).  BCQ_LUT4_MAX_ROWS=0 turns it off,
+    // BCQ_LUT4_MIN_BITS moves the precision threshold.
+    const int lut4_max = std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4));
+    const int lut4_bits = env_int("BCQ_LUT4_MIN_BITS", 3);
     for (int q = 1; q <= 4; ++q) {
       int rows[BCQ_MAX_M];
       int n = 0;
@@ -289,6 +297,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
         if (left >= 2 * kMmaRows) {
           cnt = std::min(kMaxLaunchRows, left);
           qpath = kPathUmma;
+        } else if (left >= mma_min && left <= lut4_max && q >= lut4_bits) {
+          cnt = left;  // one lookup launch over four-row pair tables
+          qpath = kPathLut4;
         } else if (left >= mma_min) {
           cnt = std::min(kMmaRows, left);
           qpath = path;
@@ -297,7 +308,8 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
           qpath = kPathLut;
         }
         Plan pl;
-        bcq_status s = plan_gemv(cnt, N, K, q, false, qpath, &pl);
+        bcq_status s = qpath == kPathLut4 ? plan_gemv(4, N, K, q, false, kPathLut, &pl)
+                                          : plan_gemv(cnt, N, K, q, false, qpath, &pl);
         if (s != BCQ_OK) return s;
         GemvParams g{};
         fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);

@@ -96,14 +96,16 @@ __global__ void pack_scales_kernel(const uint16_t* __restrict__ src,
 // Loads this lane's 8 activations of K-block kb for rows 0..M-1: the chunk
 // c = lane % 16 of group h = lane / 16 (zero past K).  x was written before
 // this grid started (or by a grid it waited for), so it is read through L2.
+// Rows m >= nrows are zero; rowmap (or nullptr: row m) gives the row of x.
 template <int M>
 __device__ __forceinline__ void load_x(const uint16_t* x, int K, int kb, int lane,
-                                       uint4 (&xv)[M]) {
+                                       uint4 (&xv)[M], int nrows = M,
+                                       const int* rowmap = nullptr) {
   const int k = kb * kKBlock + (lane >> 4) * kGroup + (lane & 15) * 8;
 #pragma unroll
   for (int m = 0; m < M; ++m) {
-    if (k < K) {
-      const uint16_t* p = x + (size_t)m * K + k;
+    if (k < K && m < nrows) {
+      const uint16_t* p = x + (size_t)(rowmap ? rowmap[m] : m) * K + k;
       asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
                    : "=r"(xv[m].x), "=r"(xv[m].y), "=r"(xv[m].z), "=r"(xv[m].w)
                    : "l"(p));
@@ -258,6 +260,7 @@ __device__ __forceinline__ float plane_sum1(const uint4& w, const uint32_t (&cr)
 }
 
 // The same for two activation rows (entries are pairs).
+template <uint32_t kBase = kDynBase>
 __device__ __forceinline__ void plane_sum2(const uint4& w, const uint32_t (&cr)[4][2],
                                            float& r0, float& r1) {
   const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
@@ -266,7 +269,7 @@ __device__ __forceinline__ void plane_sum2(const uint4& w, const uint32_t (&cr)[
   for (int u = 0; u < 4; ++u) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float2 e = lds_f32x2<kDynBase>(prmt(wd[u], cr[u][j >> 1], sel_of(j)));
+      const float2 e = lds_f32x2<kBase>(prmt(wd[u], cr[u][j >> 1], sel_of(j)));
       s0[j & 1] += e.x;
       s1[j & 1] += e.y;
     }
@@ -368,9 +371,9 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   const int warp = tid >> 5;
   const int D = prm.D, NP = prm.NP, RB = prm.RB;
   constexpr uint32_t kStage = gemv_stage_bytes(P);
-  const uint32_t full0 = sbase + gemv_off_bar(D, P);
+  const uint32_t full0 = sbase + gemv_off_bar(D, P, M);
   const uint32_t empty0 = full0 + 8u * (uint32_t)D;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + gemv_off_misc(D, P));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + gemv_off_misc(D, P, M));
   constexpr int kConsumers = kConsumerWarps * 32;
 
   // The table is addressed through load immediates: the dynamic shared
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   uint4 xv[M];
   if (warp < kConsumerWarps) {
     grid_dependency_wait();
-    load_x<M>(prm.x, prm.K, R.kb0, lane, xv);
+    load_x<M>(prm.x, prm.K, R.kb0, lane, xv, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
   }
   if (warp == 0) {
     if (cfg_ok && lane < D) {  // one lane per ring slot
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   if (*abort_flag) return;  // set before the barrier: uniform
 
   if (warp >= kConsumerWarps) {
-    produce_stages<P>(prm, R, warp - kConsumerWarps, lane, sbase + kLutBytes, full0, empty0,
+    produce_stages<P>(prm, R, warp - kConsumerWarps, lane, sbase + gemv_lut_bytes(M), full0, empty0,
                       abort_flag);
     return;
   }
@@ -471,10 +474,15 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     if (prm.KB > 1) {
 #pragma unroll
       for (int m = 0; m < M; ++m)
-        st_partial(prm.part + ((size_t)pend_kb[J] * M + m) * part_stride + (size_t)row, r[m]);
+        if (M < 4 || m < prm.M)
+          st_partial(prm.part + ((size_t)pend_kb[J] * (M == 4 ? prm.M : M) + m) * part_stride +
+                         (size_t)row,
+                     r[m]);
     } else if (row < prm.N) {
 #pragma unroll
-      for (int m = 0; m < M; ++m) prm.y[(size_t)m * prm.N + row] = f2h_rn(r[m]);
+      for (int m = 0; m < M; ++m)
+        if (M < 4 || m < prm.M)
+          prm.y[(size_t)(M == 4 ? prm.rows[m] : m) * prm.N + row] = f2h_rn(r[m]);
     }
   };
 
@@ -492,19 +500,34 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 #pragma unroll
           for (int m = 0; m < M; ++m) xv[m] = xn[m];
         } else {
-          load_x<M>(prm.x, prm.K, kbn, lane, xv);
+          load_x<M>(prm.x, prm.K, kbn, lane, xv, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
         }
       }
       if (kbn < R.kb_last) {
-        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn);
+        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
         xn_kb = kbn + 1;
       }
       // M = 2 has one table: every warp must be done with the old one.
       // M = 1 alternates two slots; the one rebuilt was last read two
       // K-blocks ago, before the previous build's barrier.
-      if (M == 2 && cur_kb >= 0) named_barrier_sync(1, kConsumers);
+      if (M >= 2 && cur_kb >= 0) named_barrier_sync(1, kConsumers);
       const int slot = M == 1 ? (kbn & 1) : 0;
-      build_lut<M, 1>(xv, slot, sbase, warp, lane, gs);
+      if constexpr (M == 4) {
+        // two pair tables: rows 0-1 at the start, rows 2-3 kLutBytes on
+        uint4 xa[2] = {xv[0], xv[1]}, xb[2] = {xv[2], xv[3]};
+        float ga[2][2], gb[2][2];
+        build_lut<2, 1>(xa, 0, sbase, warp, lane, ga);
+        build_lut<2, 1>(xb, 0, sbase + kLutBytes, warp, lane, gb);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          gs[0][h] = ga[0][h];
+          gs[1][h] = ga[1][h];
+          gs[2][h] = gb[0][h];
+          gs[3][h] = gb[1][h];
+        }
+      } else {
+        build_lut<M, 1>(xv, slot, sbase, warp, lane, gs);
+      }
       if (M == 1 && slot != cr_slot) {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -534,7 +557,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
       *abort_flag = 1;
     }
     const bool live = ok && active;
-    const uint32_t st = sbase + kLutBytes + (uint32_t)s * kStage +
+    const uint32_t st = sbase + gemv_lut_bytes(M) + (uint32_t)s * kStage +
                         (uint32_t)tw * kUnitPlaneBytes + (uint32_t)lane * 16u;
     // planes in batches of two: their plane words, then the lookups of both;
     // the stage is released once all its words are in registers
@@ -560,11 +583,24 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
         const int i = i0 + t;
         if (i < P && live) {
           // half (pass * P + i) of the lane's scales of row m
-          if (M == 1) {
+          if constexpr (M == 1) {
             const float p0 = plane_sum1(w[t][0], cr0);
             const float p1 = plane_sum1(w[t][1], cr1);
             acc[J][0] = fmaf(half_at(sc.a[0][i >> 1], i & 1), p0, acc[J][0]);
             acc[J][0] = fmaf(half_at(sc.a[0][(P + i) >> 1], (P + i) & 1), p1, acc[J][0]);
+          } else if constexpr (M == 4) {
+            // one precision: the scales of row 0 serve every row
+            float a0, a1, b0, b1, c0, c1, d0, d1;
+            plane_sum2(w[t][0], cr0, a0, a1);
+            plane_sum2<kDynBase + kLutBytes>(w[t][0], cr0, c0, c1);
+            plane_sum2(w[t][1], cr1, b0, b1);
+            plane_sum2<kDynBase + kLutBytes>(w[t][1], cr1, d0, d1);
+            const float s0 = half_at(sc.a[0][i >> 1], i & 1);
+            const float s1 = half_at(sc.a[0][(P + i) >> 1], (P + i) & 1);
+            acc[J][0] = fmaf(s1, b0, fmaf(s0, a0, acc[J][0]));
+            acc[J][1] = fmaf(s1, b1, fmaf(s0, a1, acc[J][1]));
+            acc[J][2] = fmaf(s1, d0, fmaf(s0, c0, acc[J][2]));
+            acc[J][3] = fmaf(s1, d1, fmaf(s0, c1, acc[J][3]));
           } else {
             float a0, a1, b0, b1;
             plane_sum2(w[t][0], cr0, a0, a1);
@@ -613,7 +649,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   // (no barrier: a warp starts its reduction tasks as soon as it is done;
   // the partials it waits for are polled, not counted)
   if (prm.KB > 1) {
-    splitk_tail<M == 1 ? 16 : 8>(prm, R, M, nullptr, tid, kConsumers, abort_flag);
+    // (rows: compile-time for one- and two-row launches, so the tail keeps
+    // only the loads it needs in registers)
+    splitk_tail<M == 1 ? 16 : 8>(prm, R, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr, tid,
+                                 kConsumers, abort_flag);
   }
 }
 
@@ -711,6 +750,15 @@ GemvKernel gemv_kernel_for(int M, int P, bool mixed) {
       case 2: return gemv_lut_kernel<1, 2, false>;
       case 3: return gemv_lut_kernel<1, 3, false>;
       case 4: return gemv_lut_kernel<1, 4, false>;
+      default: return nullptr;
+    }
+  }
+  if (M == 4 && !mixed) {
+    switch (P) {
+      case 1: return gemv_lut_kernel<4, 1, false>;
+      case 2: return gemv_lut_kernel<4, 2, false>;
+      case 3: return gemv_lut_kernel<4, 3, false>;
+      case 4: return gemv_lut_kernel<4, 4, false>;
       default: return nullptr;
     }
   }

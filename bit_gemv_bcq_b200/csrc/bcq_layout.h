@@ -71,18 +71,22 @@ constexpr int kReduceBatch = 128;        // units per round of arrival counting
 // without clusters and without static shared memory (checked at run time).
 constexpr uint32_t kDynBase = 0x400;
 
-// Dynamic shared memory of a GEMV launch with D ring stages of P planes.
+// Dynamic shared memory of a lookup launch of M rows with D ring stages of
+// P planes: the table (two pair tables for M = 4), the ring, the barriers.
 __host__ __device__ constexpr uint32_t gemv_stage_bytes(int P) {
   return (uint32_t)P * kPlaneGroupBytes;
 }
-__host__ __device__ constexpr uint32_t gemv_off_bar(int D, int P) {
-  return kLutBytes + (uint32_t)D * gemv_stage_bytes(P);
+__host__ __device__ constexpr uint32_t gemv_lut_bytes(int M) {
+  return M == 4 ? 2u * kLutBytes : kLutBytes;
 }
-__host__ __device__ constexpr uint32_t gemv_off_misc(int D, int P) {
-  return gemv_off_bar(D, P) + 16u * (uint32_t)D;
+__host__ __device__ constexpr uint32_t gemv_off_bar(int D, int P, int M = 1) {
+  return gemv_lut_bytes(M) + (uint32_t)D * gemv_stage_bytes(P);
 }
-__host__ __device__ constexpr uint32_t gemv_dyn_bytes(int D, int P) {
-  return gemv_off_misc(D, P) + 16u + 4u * kReduceBatch;
+__host__ __device__ constexpr uint32_t gemv_off_misc(int D, int P, int M = 1) {
+  return gemv_off_bar(D, P, M) + 16u * (uint32_t)D;
+}
+__host__ __device__ constexpr uint32_t gemv_dyn_bytes(int D, int P, int M = 1) {
+  return gemv_off_misc(D, P, M) + 16u + 4u * kReduceBatch;
 }
 
 // Units of one CTA, computed on the host: [u0, u1), its group count and

@@ -540,7 +540,7 @@ def launches_per_call(M):
     return -(-M // 16) if M >= MMA_MIN_ROWS else -(-M // 2)
 
 
-LUT4_MIN_BITS = 3  # bcq_gemm's four-row lookup launches: 3-4 rows of >= 3 bits
+LUT4_MIN_BITS = 1  # bcq_gemm's four-row lookup launches: 3-4 rows of any precision
 
 
 def kernel_of(M, p):
@@ -665,8 +665,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
                      "peak_kind": peak_kind, "traffic": None,
-                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 2 and for "
-                               "M = 4 at p >= 3, gemv_mma_kernel for the other batches)"},
+                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 4, "
+                               "gemv_mma_kernel for M = 8 and 16)"},
         "per_call": res["per_case"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],

@@ -278,14 +278,13 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
   const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
   if (M >= mma_min) {
     const int path = batch_path();
-    // batches of 3-4 rows of one precision of at least 3 bits: one lookup
-    // launch over two pair tables (measured on 14336 x 4096: p = 3 / 4 in
-    // 26.1 / 29.7 us against 29.6 / 36.6 us on the tensor-core kernel; at
-    // p = 2 building two tables costs more than the shorter loop saves:
-    // 23.8 against 22.9 us).  BCQ_LUT4_MAX_ROWS=0 turns it off,
-    // BCQ_LUT4_MIN_BITS moves the precision threshold.
+    // batches of 3-4 rows of one precision: one lookup launch over two pair
+    // tables (measured on 14336 x 4096: p = 2 / 3 / 4 in 17.2 / 23.6 /
+    // 26.2 us against 22.9 / 29.6 / 36.6 us on the tensor-core kernel).
+    // BCQ_LUT4_MAX_ROWS=0 turns it off, BCQ_LUT4_MIN_BITS sets a precision
+    // threshold.
     const int lut4_max = std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4));
-    const int lut4_bits = env_int("BCQ_LUT4_MIN_BITS", 3);
+    const int lut4_bits = env_int("BCQ_LUT4_MIN_BITS", 1);
     for (int q = 1; q <= 4; ++q) {
       int rows[BCQ_MAX_M];
       int n = 0;

@@ -503,8 +503,10 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
           load_x<M>(prm.x, prm.K, kbn, lane, xv, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
         }
       }
-      if (kbn < R.kb_last) {
-        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
+      // the next K-block's x is fetched a table ahead (four-row launches
+      // load it when needed: its registers would spill in the main loop)
+      if (M != 4 && kbn < R.kb_last) {
+        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn);
         xn_kb = kbn + 1;
       }
       // M = 2 has one table: every warp must be done with the old one.

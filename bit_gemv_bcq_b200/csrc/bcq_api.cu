@@ -432,13 +432,19 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
   if (M < 1 || M > kMaxLaunchRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
   if (p_load < 1 || p_load > 4) return BCQ_ERR_PRECISION;
   if (mixed && (M != 2 || p_load < 2)) return BCQ_ERR_PRECISION;
-  const int path = M > kMmaRows ? kPathUmma : M > kMaxMPerLaunch ? batch_path() : kPathLut;
+  // 3-4 rows: the four-row lookup launch bcq_gemm would use (same switches)
+  const bool lut4 = !mixed && M > kMaxMPerLaunch &&
+                    M <= std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4)) &&
+                    p_load >= env_int("BCQ_LUT4_MIN_BITS", 1);
+  const int path = lut4 ? kPathLut
+                   : M > kMmaRows ? kPathUmma
+                   : M > kMaxMPerLaunch ? batch_path() : kPathLut;
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;
   if (t_virtual) (void)cudaGetLastError();
   Plan pl;
-  bcq_status st = plan_gemv(M, N, K, p_load, mixed != 0, path, &pl);
+  bcq_status st = plan_gemv(lut4 ? 4 : M, N, K, p_load, mixed != 0, path, &pl);
   t_virtual = false;
   if (st != BCQ_OK) return st;
   out[0] = pl.C;

@@ -195,10 +195,10 @@ bcq_status bcq_gemm_zp(const uint16_t* x, const uint32_t* planes,
 /*
  * The launch plan bcq_gemm would use for one launch of M (1..64) activation
  * rows streaming p_load planes (mixed = 1: two rows of different
- * precisions).  M <= 2 plans the lookup-table kernel, 3 <= M <= 16 the
- * tensor-core kernel that bcq_gemm would use for a batch (BCQ_MMA_KIND), and
- * M >= 17 the 64-row tcgen05 launch.  (bcq_gemm itself sends 3-4 rows of
- * one precision to a four-row lookup launch.)  use_device = 1
+ * precisions).  M <= 2 plans the lookup-table kernel, 3 <= M <= 4 its
+ * four-row launch (two pair tables), 5 <= M <= 16 the tensor-core kernel
+ * that bcq_gemm would use for a batch (BCQ_MMA_KIND), and M >= 17 the
+ * 64-row tcgen05 launch.  use_device = 1
  * plans for the current device; 0 (or no usable device) plans for a nominal
  * 148-SM B200 without touching CUDA.  out[8] receives: CTAs, consumer warps,
  * producer warps, ring stages, dynamic shared memory bytes, bytes per ring

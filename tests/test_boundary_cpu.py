@@ -74,7 +74,8 @@ def test_workspace_bytes_formula(L):
                                            (1, 4096, 14336, 3, False), (2, 4096, 4096, 2, False),
                                            (2, 28672, 8192, 4, True), (1, 256, 512, 4, False),
                                            (1, 1, 128, 1, False), (2, 33, 640, 2, False),
-                                           (64, 14336, 4096, 4, False), (33, 4096, 4096, 2, False)])
+                                           (64, 14336, 4096, 4, False), (33, 4096, 4096, 2, False),
+                                           (4, 14336, 4096, 4, False), (3, 4096, 4096, 2, False)])
 def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     """Plans for a nominal 148-SM B200 (no GPU needed): one CTA per SM at
     most (never more CTAs than units), whole K-blocks per CTA when the CTAs
@@ -95,7 +96,7 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     assert pl["dyn_bytes"] <= 232448
     assert pl["stage_bytes"] == 8192 * p    # the p planes of one row group
     tiles = 2 * (16 if M <= 16 else 64) * 256 * 2        # two activation tiles
-    table = 65536 if M <= 2 else tiles                    # or the lookup table
+    table = 65536 if M <= 2 else 131072 if M <= 4 else tiles  # or the lookup table(s)
     assert pl["dyn_bytes"] >= table + pl["D"] * pl["stage_bytes"]
     assert pl["D"] % 2 == 0 and pl["D"] % pl["NP"] == 0 and 2 <= pl["D"] <= 20
     # as deep as the shared memory allows

@@ -244,7 +244,8 @@ _WS: dict = {}
 def workspace(M: int, N: int, K: int, device, stream=None) -> torch.Tensor | None:
     """The zero-filled workspace of (device, stream), at least
     bcq_workspace_bytes(M, N, K) bytes; None when none is needed.  Every call
-    that completes leaves it zero-filled again."""
+    that completes leaves it zero-filled again.  Calls that may run at the
+    same time (other streams) get workspaces of their own."""
     need = workspace_bytes(M, N, K)
     if need == 0:
         return None
@@ -261,7 +262,7 @@ def workspace(M: int, N: int, K: int, device, stream=None) -> torch.Tensor | Non
 
 def drop_workspaces() -> None:
     """Forget the cached workspaces (after a device error they may hold
-    stale counters; new ones are zero-filled)."""
+    partial sums; new ones are zero-filled)."""
     _WS.clear()
 
 
@@ -473,7 +474,7 @@ def build_lut(x: torch.Tensor, stream=None):
 
 def device_error(stream=None) -> int:
     """Synchronise the stream, return and clear the device error word.  After
-    an error the cached workspaces are dropped (their counters may be stale)."""
+    an error the cached workspaces are dropped (they may hold partial sums)."""
     st = int(lib().bcq_device_error(_stream(stream)))
     if st != BCQ_OK:
         drop_workspaces()

@@ -26,7 +26,14 @@ constexpr int kDefaultMmaMinRows = 3;
 
 // Kernels: the lookup-table kernel (one or two rows), and for batches a
 // tensor-core kernel: mma.sync (default) or tcgen05 (BCQ_MMA_KIND=tcgen05).
-enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2, kPathLut4 = 3 };
+enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2, kPathLut4 = 3, kPathM1 = 4 };
+
+// One-row launches: the dense-table kernel (bcq_m1.cuh) unless
+// BCQ_M1_KIND=pair asks for the pair-table kernel with one row.
+bool use_m1_kernel() {
+  const char* v = std::getenv("BCQ_M1_KIND");
+  return !(v && std::strcmp(v, "pair") == 0);
+}
 
 int batch_path() {
   const char* v = std::getenv("BCQ_MMA_KIND");
@@ -96,7 +103,7 @@ bcq_status get_device(DeviceCache** dc) {
 
 struct Plan {
   GemvKernel fn = nullptr;
-  int C = 0, D = 0, NP = 0, MW = 0;
+  int C = 0, D = 0, NP = 0, MW = 0, CW = kConsumerWarps;
   size_t dyn = 0;
   long long units_max = 0;
   int KB = 0;
@@ -116,12 +123,14 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   const int NN = M > kMmaRows ? kMaxLaunchRows : kMmaRows;  // tcgen05: 16 or 64 rows
   pl.fn = path == kPathUmma      ? gemv_umma_kernel_for(P, NN)
           : path == kPathMmaSync ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P)
+          : path == kPathM1      ? gemv_m1_kernel_for(P)
                                  : gemv_kernel_for(M, P, mixed);
   if (!pl.fn) return BCQ_ERR_UNSUPPORTED;
   auto dyn_of = [&](int d) {
     return path == kPathUmma      ? (NN == kMmaRows ? umma_dyn_bytes<16>(d, P)
                                                      : umma_dyn_bytes<64>(d, P))
            : path == kPathMmaSync ? mma_dyn_bytes(d, P)
+           : path == kPathM1      ? m1_dyn_bytes(d, P)
                                   : gemv_dyn_bytes(d, P, M);
   };
   const long long RB = (long long)row_blocks(N);
@@ -129,13 +138,16 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   const long long U = RB * KB;
   pl.KB = (int)KB;
   pl.NP = std::max(1, std::min(2, env_int("BCQ_FORCE_NP", kDefaultProducers)));
-  const int step = 2;  // even, and a multiple of NP <= 2
+  // ring stages: even (the two teams alternate) and a multiple of NP
+  const int step = 2;
+  const size_t dyn_cap = kMaxDynSmem;
   int D = env_int("BCQ_FORCE_D", kMaxStages);
   D = std::min(kMaxStages, D) / step * step;
   if (D < step) D = step;
-  while (D > step && dyn_of(D) > kMaxDynSmem) D -= step;
+  while (D > step && dyn_of(D) > dyn_cap) D -= step;
   pl.MW = path == kPathUmma ? kUmmaGroups : 0;
-  const int nthreads = 32 * (kConsumerWarps + pl.MW + pl.NP);
+  pl.CW = path == kPathM1 ? kM1Warps : kConsumerWarps;
+  const int nthreads = 32 * (pl.CW + pl.MW + pl.NP);
   while (true) {
     pl.dyn = dyn_of(D);
     int per_sm = 0;
@@ -156,9 +168,15 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   pl.D = D;
   // With no more K-blocks than SMs, every K-block gets the same number of
   // CTAs and no CTA spans two K-blocks (a second table build would make it
-  // the slowest CTA, and the last to arrive for all of its row-blocks).
+  // the slowest CTA, and the last to arrive for all of its row-blocks).  The
+  // one-row kernel keeps that split only while it leaves at most a tenth of
+  // the SMs idle; otherwise every SM takes an equal share of the units and
+  // some CTAs rebuild the table once (4096 x 14336: 148 CTAs, not 112).
   long long C = std::min<long long>(U, std::min(dc->sm_count, kMaxCtas));
-  if (KB <= C) C = std::min<long long>(U, KB * std::min<long long>(RB, C / KB));
+  if (KB <= C) {
+    const long long even = std::min<long long>(U, KB * std::min<long long>(RB, C / KB));
+    if (path != kPathM1 || even * 10 >= C * 9) C = even;
+  }
   const int force_C = env_int("BCQ_FORCE_C", 0);
   if (force_C > 0) C = std::min<long long>(U, std::min(force_C, kMaxCtas));
   pl.C = (int)C;
@@ -240,8 +258,8 @@ void plan_units(int RB, int KB, int C, CtaWork* work) {
 }
 
 // Fills the fields every launch shares.
-void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes,
-                 int N, int K, int p_H, void* ws, int pdl_mode, int wait_us) {
+void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, int N, int K, int p_H,
+                 void* ws, int pdl_mode, int wait_us) {
   const int RB = (int)row_blocks(N);
   const int KB = (int)k_blocks(K);
   g.planes = planes;
@@ -261,6 +279,11 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes,
   g.early_weights = pdl_mode == 2 ? 1 : 0;
   g.timeout_ns = wait_us > 0 ? (unsigned long long)wait_us * 1000ull : kDefaultWaitNs;
 }
+
+// Cooperative launches (all CTAs of a grid resident at once, which the
+// split-K tail's polling relies on); BCQ_COOPERATIVE=0 turns the attribute
+// off (for comparison only: the tail then assumes the grid fits at once).
+bool cooperative_launch() { return env_int("BCQ_COOPERATIVE", 1) != 0; }
 
 // Small batches: lookup-table launches of at most two rows, in order; two
 // rows with different precisions share one launch (planes streamed up to
@@ -306,6 +329,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
           cnt = 1;
           qpath = kPathLut;
         }
+        if (qpath == kPathLut && use_m1_kernel()) qpath = kPathM1;
         Plan pl;
         bcq_status s = qpath == kPathLut4 ? plan_gemv(4, N, K, q, false, kPathLut, &pl)
                                           : plan_gemv(cnt, N, K, q, false, qpath, &pl);
@@ -316,7 +340,7 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
         g.z = g.z1 = zq[q - 1];
         g.M = cnt;
         g.q[0] = g.q[1] = q;
-        if (qpath == kPathLut) {  // one row, addressed directly
+        if (qpath == kPathLut || qpath == kPathM1) {  // one row, addressed directly
           g.x = x + (size_t)rows[r0] * K;
           g.y = y + (size_t)rows[r0] * N;
         } else {
@@ -324,7 +348,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
           g.y = y;
           for (int j = 0; j < cnt; ++j) g.rows[j] = rows[r0 + j];
         }
-        if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st) != cudaSuccess) return BCQ_ERR_CUDA;
+        if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st, pl.CW, cooperative_launch()) !=
+            cudaSuccess)
+          return BCQ_ERR_CUDA;
         r0 += cnt;
       }
     }
@@ -337,8 +363,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
       q[r] = p > 0 ? p : p_row[m0 + std::min(r, rows - 1)];
     const int P = std::max(q[0], q[1]);
     const bool mixed = q[0] != q[1];
+    const int path = rows == 1 && use_m1_kernel() ? kPathM1 : kPathLut;
     Plan pl;
-    bcq_status s = plan_gemv(rows, N, K, P, mixed, kPathLut, &pl);
+    bcq_status s = plan_gemv(rows, N, K, P, mixed, path, &pl);
     if (s != BCQ_OK) return s;
     GemvParams g{};
     fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);
@@ -351,7 +378,9 @@ bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* c
     g.M = rows;
     g.q[0] = q[0];
     g.q[1] = q[1];
-    if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st) != cudaSuccess) return BCQ_ERR_CUDA;
+    if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st, pl.CW, cooperative_launch()) !=
+        cudaSuccess)
+      return BCQ_ERR_CUDA;
     m0 += rows;
   }
   return BCQ_OK;
@@ -438,7 +467,8 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
                     p_load >= env_int("BCQ_LUT4_MIN_BITS", 1);
   const int path = lut4 ? kPathLut
                    : M > kMmaRows ? kPathUmma
-                   : M > kMaxMPerLaunch ? batch_path() : kPathLut;
+                   : M > kMaxMPerLaunch ? batch_path()
+                   : M == 1 && !mixed && use_m1_kernel() ? kPathM1 : kPathLut;
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;
@@ -448,11 +478,11 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
   t_virtual = false;
   if (st != BCQ_OK) return st;
   out[0] = pl.C;
-  out[1] = kConsumerWarps;
+  out[1] = pl.CW;
   out[2] = pl.NP;
   out[3] = pl.D;
   out[4] = (int)pl.dyn;
-  out[5] = (int)gemv_stage_bytes(p_load);
+  out[5] = (int)(path == kPathM1 ? m1_stage_bytes(p_load) : gemv_stage_bytes(p_load));
   out[6] = (int)pl.units_max;
   out[7] = pl.KB;
   return BCQ_OK;

@@ -62,6 +62,18 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t lds_u32v(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds_v2u(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -75,6 +87,10 @@ template <uint32_t OFF>
 __device__ __forceinline__ void sts_f32x2_at(uint32_t addr, float a, float b) {
   asm volatile("st.shared.v2.f32 [%0+%1], {%2, %3};" ::"r"(addr), "n"(OFF), "f"(a), "f"(b)
                : "memory");
+}
+
+__device__ __forceinline__ void stg_cg_zero(float* p) {
+  asm volatile("st.global.cg.f32 [%0], %1;" ::"l"(p), "f"(0.f) : "memory");
 }
 
 // Read-only global loads that do not allocate in L1 (streamed data).
@@ -101,10 +117,6 @@ __device__ __forceinline__ uint16_t ldg_nc_u16(const void* p) {
   uint16_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
-}
-
-__device__ __forceinline__ void stg_cg_zero(float* p) {
-  asm volatile("st.global.cg.f32 [%0], %1;" ::"l"(p), "f"(0.f) : "memory");
 }
 
 // Split-K partial sums travel as the complement of their fp32 bits, so a
@@ -210,6 +222,24 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src,
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
       "[%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// L2 policy for data read once per call (planes, scales, offsets): evicted
+// first, so they do not push x and the split-K workspace out of L2.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// bulk_g2s with an L2 cache policy.
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
       : "memory");
 }
 

@@ -5,8 +5,10 @@
 //   gemv_lut_kernel      producer warps stream plane stages by bulk copy;
 //                        consumer warps build the K-block's lookup table,
 //                        look up and accumulate, fuse alpha and z, and write
-//                        split-K partial sums; the last CTA to finish a
-//                        row-block sums its partials in K order -> fp16 y
+//                        split-K partial sums; the CTA that computed a
+//                        row-block's unit in K-block rb mod KB sums its
+//                        partials in K order -> fp16 y
+//   gemv_m1_kernel       the one-row GEMV (bcq_m1.cuh)
 //   lut_dump_kernel      the same table build, written out for inspection
 //   wait_probe_kernel    exercises the bounded mbarrier wait
 //
@@ -60,7 +62,7 @@ __global__ void pack_planes_kernel(const uint32_t* __restrict__ canon,
         const size_t cb = kb * 32 + h * 16 + c;  // canonical byte index in the row
         if (cb * 8 < (size_t)K) {
           const uint32_t byte = (row[cb >> 2] >> (8 * (cb & 3))) & 0xFFu;
-          out |= byte << (8 * j);
+          out |= (((byte >> 1) | (byte << 7)) & 0xFFu) << (8 * j);  // rotr8(byte, 1)
         }
       }
     }
@@ -173,11 +175,21 @@ struct LutRows2<16, HH> {
                                              float, float, float, float) {}
 };
 
-// Builds the table of one K-block at shared address lut (layout in
-// bcq_layout.h): 16 / HH warps of the caller each write the entries of high
-// nibbles HH * warp .. HH * warp + HH - 1 for all 32 columns (lane = column).
-// Entry b of a column with activations v0..v7 is sum_j (2 bit_j(b) - 1) v_j,
-// formed as L[b & 15] + H[b >> 4].  Also returns the group sums of this
+// Activations of one chunk in the bit order of a stored plane byte: bit j of
+// the stored byte is column (j + 1) mod 8 of the chunk (bcq_layout.h).
+__device__ __forceinline__ void unpack8_stored(const uint4& r, float (&v)[8]) {
+  float c[8];
+  unpack8(r, c);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = c[(j + 1) & 7];
+}
+
+// Builds the pair-layout table of one K-block at shared address lut (layout
+// in bcq_layout.h), indexed by the stored byte s: 16 / HH warps of the
+// caller each write the entries of high nibbles HH * warp .. HH * warp +
+// HH - 1 for all 32 columns (lane = column).  Entry s of a column with
+// activations v0..v7 (in stored bit order) is sum_j (2 bit_j(s) - 1) v_j,
+// formed as L[s & 15] + H[s >> 4].  Also returns the group sums of this
 // lane's pass-0 group (gs[m][0]) and of the other group (gs[m][1]).  The
 // caller synchronises before the table is read.
 template <int M, int HH>
@@ -185,7 +197,7 @@ __device__ __forceinline__ void build_lut(const uint4 (&xv)[M], int slot, uint32
                                           int warp, int lane, float (&gs)[M][2]) {
   float v[M][8];
 #pragma unroll
-  for (int m = 0; m < M; ++m) unpack8(xv[m], v[m]);
+  for (int m = 0; m < M; ++m) unpack8_stored(xv[m], v[m]);
   float L[M][16];
 #pragma unroll
   for (int m = 0; m < M; ++m) low_sums(v[m], L[m]);
@@ -660,6 +672,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 
 }  // namespace bcq
 
+#include "bcq_m1.cuh"
 #include "bcq_mma.cuh"
 #include "bcq_umma.cuh"
 
@@ -667,8 +680,10 @@ namespace bcq {
 
 // ============================================================ LUT dump
 
-// One CTA per K-block: the table exactly as the GEMV kernel builds it, read
-// back to global memory in the canonical [M][K/8][256] order.
+// One CTA per K-block: the table exactly as the GEMV kernels build it (M = 1:
+// the one-row kernel's dense table, indexed by the canonical byte; M = 2:
+// the pair table, indexed by the stored byte rotr8(b, 1)), read back to
+// global memory in the canonical [M][K/8][256] order.
 template <int M>
 __global__ void __launch_bounds__(256) lut_dump_kernel(const __grid_constant__ LutParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -679,8 +694,11 @@ __global__ void __launch_bounds__(256) lut_dump_kernel(const __grid_constant__ L
   uint4 xv[M];
   load_x<M>(P.x, P.K, kb, lane, xv);
   float gs[M][2];
-  const int slot = M == 1 ? (kb & 1) : 0;
-  build_lut<M, 2>(xv, slot, sbase, warp, lane, gs);
+  if constexpr (M == 1) {
+    build_lut1c<2>(xv[0], sbase, warp, lane, gs[0]);  // 8 warps
+  } else {
+    build_lut<M, 2>(xv, 0, sbase, warp, lane, gs);
+  }
   __syncthreads();
   const int C8 = P.K / 8;
   for (int e = threadIdx.x; e < M * 32 * 256; e += blockDim.x) {
@@ -689,9 +707,9 @@ __global__ void __launch_bounds__(256) lut_dump_kernel(const __grid_constant__ L
     const int m = e >> 13;
     const int k = kb * kKBlock + (col >> 4) * kGroup + (col & 15) * 8;
     if (k >= P.K) continue;
-    const uint32_t a = sbase + (uint32_t)b * 256u +
-                       (M == 1 ? (uint32_t)slot * 128u + (uint32_t)col * 4u
-                               : (uint32_t)col * 8u + (uint32_t)m * 4u);
+    const uint32_t sb = ((uint32_t)b >> 1) | (((uint32_t)b & 1u) << 7);  // stored byte
+    const uint32_t a = M == 1 ? sbase + (uint32_t)b * 128u + (uint32_t)col * 4u
+                              : sbase + sb * 256u + (uint32_t)col * 8u + (uint32_t)m * 4u;
     P.lut[((size_t)m * C8 + k / 8) * 256 + b] = lds_f32_dyn(a);
   }
   if (P.gsum && warp == 0 && (lane & 15) == 0) {
@@ -784,6 +802,16 @@ GemvKernel gemv_kernel_for(int M, int P, bool mixed) {
   return nullptr;
 }
 
+GemvKernel gemv_m1_kernel_for(int P) {
+  switch (P) {
+    case 1: return gemv_m1_kernel<1>;
+    case 2: return gemv_m1_kernel<2>;
+    case 3: return gemv_m1_kernel<3>;
+    case 4: return gemv_m1_kernel<4>;
+    default: return nullptr;
+  }
+}
+
 GemvKernel gemv_mma_kernel_for(int NT, int P) {
   if (NT == 1) {
     switch (P) {
@@ -829,17 +857,22 @@ GemvKernel gemv_umma_kernel_for(int P, int NN) {
 }
 
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,
-                        cudaStream_t st) {
+                        cudaStream_t st, int consumer_warps, bool cooperative) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.C, 1, 1);
-  cfg.blockDim = dim3((unsigned)(32 * (kConsumerWarps + p.MW + p.NP)), 1, 1);
+  cfg.blockDim = dim3((unsigned)(32 * (consumer_warps + p.MW + p.NP)), 1, 1);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   int na = 0;
   if (pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cooperative) {  // every CTA resident at once: the split-K tail polls other CTAs
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
     ++na;
   }
   cfg.attrs = attr;

@@ -22,6 +22,10 @@ cudaError_t launch_pack_scales(const uint16_t* src, uint16_t* dst, int q, int N,
 // the rows use different precisions.  nullptr if there is none.
 GemvKernel gemv_kernel_for(int M, int P, bool mixed);
 
+// The one-row lookup GEMV kernel (bcq_m1.cuh) for precision P; nullptr if
+// there is none.
+GemvKernel gemv_m1_kernel_for(int P);
+
 // The tensor-core GEMV kernel for NT n-tiles of 8 activation rows (1 or 2)
 // streaming P planes (one precision); nullptr if there is none.
 GemvKernel gemv_mma_kernel_for(int NT, int P);
@@ -30,9 +34,10 @@ GemvKernel gemv_mma_kernel_for(int NT, int P);
 // P planes (one precision); nullptr if there is none.
 GemvKernel gemv_umma_kernel_for(int P, int NN);
 
-// p.C CTAs of 32 * (16 + p.MW + p.NP) threads.
+// p.C CTAs of 32 * (consumer_warps + p.MW + p.NP) threads; cooperative: all
+// CTAs resident at once (the launch fails rather than run fewer).
 cudaError_t launch_gemv(GemvKernel fn, const GemvParams& p, size_t dyn, bool pdl,
-                        cudaStream_t st);
+                        cudaStream_t st, int consumer_warps, bool cooperative);
 
 // CTAs of this shape that fit on one SM (also raises the kernel's dynamic
 // shared-memory limit to dyn).

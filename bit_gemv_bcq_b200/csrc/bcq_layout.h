@@ -25,6 +25,10 @@
 // lanes 0-15 walk group A and lanes 16-31 group B; in pass 1 they swap.  At
 // every step the 32 lanes touch 32 different (group, chunk) columns of the
 // lookup table, one per shared-memory bank, whatever the bit values.
+// Inside a byte the chunk's 8 bits are rotated right by one: bit j of the
+// stored byte is column 8c + ((j + 1) mod 8), i.e. stored = rotr8(canonical,
+// 1).  The one-row kernel then forms the address b * 128 + column * 4 of a
+// dense 32 KiB table directly from the stored byte (see below).
 // Row-blocks past N and columns past K are zero.
 //
 // Packed scales (written by bcq_pack_scales, read by the GEMV kernel)
@@ -41,12 +45,22 @@
 // Lookup table in shared memory
 // -----------------------------
 // The table of one K-block sits at the start of the dynamic shared memory.
-// Entry (byte value b, column col = h * 16 + c) is at
-//   M = 1: b * 256 + slot * 128 + col * 4    (fp32; slot = kb & 1)
-//   M = 2: b * 256 + col * 8                 (fp32 pair: row 0, row 1)
-// One prmt forms b * 256 + (column byte) from a plane word and a per-lane
-// register holding the column bytes; the table's shared address is the
-// immediate offset of the load, so the table needs no alignment.
+// For the stored byte s of a chunk (s = rotr8(b, 1) for the canonical byte
+// b) and column col = h * 16 + c, the entry sum_j (2 bit_j(b) - 1) x[8c + j]
+// is at
+//   M = 1 (gemv_m1_kernel):  b * 128 + col * 4    (fp32, dense 32 KiB)
+//   M = 2, 4 (pair tables):  s * 256 + col * 8    (fp32 pair: row 0, row 1)
+// Pair tables: one prmt forms s * 256 + (column byte) from a plane word and
+// a per-lane register holding the column bytes.  M = 1: with a = s & 0x7F
+// and e = (s & 0x80) | (column byte), one prmt forms a * 256 + e =
+// rotl8(s, 1) * 128 + col * 4 = b * 128 + col * 4 (two lop3 per word make
+// a and e for its four bytes).  The table's shared address is the immediate
+// offset of the load, so the table needs no alignment.
+//
+// One-row kernel (gemv_m1_kernel) ring stage: the P planes of a row group
+// (plane i at i * 8 KiB, row-block w at w KiB), then its packed alpha^(P)
+// (row-block w at w * 128 P bytes), then its packed offsets (w * 128
+// bytes): three bulk copies of the packed arrays, 16-byte aligned.
 #pragma once
 
 #include <cstdint>
@@ -66,7 +80,6 @@ constexpr uint32_t kLutBytes = 65536;
 constexpr int kMaxStages = 20;
 constexpr int kMaxProducerWarps = 4;
 constexpr int kMaxMPerLaunch = 2;        // activation rows per GEMV launch
-constexpr int kReduceBatch = 128;        // units per round of arrival counting
 // Shared-window address of the dynamic shared memory of a CTA launched
 // without clusters and without static shared memory (checked at run time).
 constexpr uint32_t kDynBase = 0x400;
@@ -86,7 +99,33 @@ __host__ __device__ constexpr uint32_t gemv_off_misc(int D, int P, int M = 1) {
   return gemv_off_bar(D, P, M) + 16u * (uint32_t)D;
 }
 __host__ __device__ constexpr uint32_t gemv_dyn_bytes(int D, int P, int M = 1) {
-  return gemv_off_misc(D, P, M) + 16u + 4u * kReduceBatch;
+  return gemv_off_misc(D, P, M) + 16u;
+}
+
+// The one-row kernel: 16 consumer warps in two teams of 8 (team t takes
+// stages t, t + 2, ...; warp w of a team takes row-block w of the stage)
+// and NP producer warps; a dense 32 KiB table; ring stages of planes +
+// scales + offsets; then the full / empty barriers and the abort flag.
+constexpr int kM1Warps = 16;
+constexpr int kM1TeamWarps = 8;
+constexpr uint32_t kLut1Bytes = 32768;
+__host__ __device__ constexpr uint32_t m1_alpha_off(int P) {
+  return (uint32_t)P * kPlaneGroupBytes;
+}
+__host__ __device__ constexpr uint32_t m1_z_off(int P) {
+  return m1_alpha_off(P) + (uint32_t)kRowGroup * 128u * (uint32_t)P;
+}
+__host__ __device__ constexpr uint32_t m1_stage_bytes(int P) {
+  return m1_z_off(P) + (uint32_t)kRowGroup * 128u;
+}
+__host__ __device__ constexpr uint32_t m1_off_bar(int D, int P) {
+  return kLut1Bytes + (uint32_t)D * m1_stage_bytes(P);
+}
+__host__ __device__ constexpr uint32_t m1_off_misc(int D, int P) {
+  return m1_off_bar(D, P) + 16u * (uint32_t)D;
+}
+__host__ __device__ constexpr uint32_t m1_dyn_bytes(int D, int P) {
+  return m1_off_misc(D, P) + 16u;
 }
 
 // Units of one CTA, computed on the host: [u0, u1), its group count and

@@ -139,15 +139,16 @@ __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, i
 // byte (4v - rho) mod 16, rho = r mod 16: it is the funnel shift of rotated
 // words (v - R) mod 4 and (v - R + 1) mod 4 by 8 delta bits, with
 // R = ceil(rho / 4) mod 4 and delta = (-rho) mod 4 -- per-thread constants.
-// A fragment element pair (columns 2q, 2q + 1 of an 8-column chunk) becomes
-// +-alpha by moving the two bits to bit 7 of their byte (shifts by 7 - 2q and
-// 6 - 2q), replicating each into a sign byte (prmt) and xoring the fp16 sign
+// A fragment element pair (columns 2q, 2q + 1 of an 8-column chunk; stored
+// bits (2q + 7) mod 8 and 2q, the bytes being rotated) becomes +-alpha by
+// moving the two bits to bit 7 of their byte (shifts by (8 - 2q) mod 8 and
+// 7 - 2q), replicating each into a sign byte (prmt) and xoring the fp16 sign
 // bits of alpha2 (lop3).
 template <int NT, int P>
 __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sbuf, int i,
                                           int g, int q, uint32_t ra0, uint32_t ra1, uint32_t dsh,
                                           float (&acc)[2][2][NT][4]) {
-  const uint32_t sh1 = 7u - 2u * (uint32_t)q, sh2 = 6u - 2u * (uint32_t)q;
+  const uint32_t sh1 = (8u - 2u * (uint32_t)q) & 7u, sh2 = 7u - 2u * (uint32_t)q;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     // activation fragments of the group's 8 k-steps, off the critical path

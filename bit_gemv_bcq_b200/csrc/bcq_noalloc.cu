@@ -5,9 +5,9 @@
 // takes from its caller comes from a static array of this library instead.
 //
 // The array lives in this translation unit.  Host code sees only a host-side
-// stand-in under its name, so its device address is looked up here, once per
-// device with that device current, and passed to the kernels as the
-// workspace pointer of bcq_gemm.
+// stand-in under its name, so its device address is looked up here, with the
+// call's device current, and passed to the kernels as the workspace pointer
+// of bcq_gemm.
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -27,14 +27,18 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (looked up on
-// the first call for that device).
-bcq_status scratch_address(void** out) {
+// Device address of g_noalloc_scratch on the current device: looked up on
+// every call (cheap, and right again after a device or context reset loads
+// the module anew) except while `stream` is capturing a graph, when the last
+// address found on this device is used.
+bcq_status scratch_address(cudaStream_t stream, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BCQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return BCQ_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return BCQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_scratch_addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BCQ_ERR_CUDA;
     g_scratch_addr[dev] = p;
@@ -52,7 +56,7 @@ extern "C" bcq_status bcq_gemm_noalloc(const uint16_t* x, const uint32_t* planes
   const size_t need = (M > 0) ? bcq_workspace_bytes(M, N, K) : 0;
   void* ws = nullptr;
   if (need > 0) {
-    bcq_status s = scratch_address(&ws);
+    bcq_status s = scratch_address(static_cast<cudaStream_t>(stream), &ws);
     if (s != BCQ_OK) return s;
   }
   // bcq_gemm's checks, with the scratch standing in for the workspace, so

@@ -140,7 +140,10 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
 // its warp has stored its own partial sums (no barrier).  Every unit's fp32
 // partials [kb][m][row] go to the workspace as tagged words (st_partial: zero
 // = not written yet), so no fence or arrival counter is needed: a reducer
-// polls the partials themselves.  Row-block rb is reduced by the CTA that
+// polls the partials themselves.  The polling needs every CTA of the grid
+// to run: the GEMV kernels are launched cooperatively (one CTA per SM at
+// most, cudaLaunchAttributeCooperative), so the launch makes all of them
+// resident at once, whatever else holds the GPU.  Row-block rb is reduced by the CTA that
 // computed its unit in K-block rb mod KB, so the work is spread evenly
 // whatever the order in which CTAs finish.  The (row-block, two launch rows)
 // tasks of the CTA are dealt to its warps in turn; a warp loads all KB
@@ -208,7 +211,9 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
                   have = have && v[mm][j] != 0u;
                 }
               if (__all_sync(0xFFFFFFFFu, have)) break;
-              if (*abort_flag || globaltimer_ns() - t0 > prm.timeout_ns) {
+              // (warp-uniform: every lane leaves the loop together)
+              if (__any_sync(0xFFFFFFFFu,
+                             *abort_flag != 0 || globaltimer_ns() - t0 > prm.timeout_ns)) {
                 ok = false;
                 break;
               }

@@ -21,8 +21,10 @@
 // K order.  Inside a 256-column K-block the A operand holds the columns in
 // the order the expansion produces them: tensor-memory column
 // c = 64 h + 16 U + s (group h, 32-column word U of the group, shift s)
-// holds columns 128 h + 32 U + 15 - s (low half) and 128 h + 32 U + 31 - s
-// (high half).  The activation tile is stored with the same permutation.
+// holds the columns of bits 15 - s (low half) and 31 - s (high half) of the
+// group's natural word U, where bit t is column 128 h + 32 U + 8 (t / 8) +
+// ((t + 1) mod 8) (the packed bytes are rotated by one bit).  The activation
+// tile is stored with the same permutation.
 #pragma once
 
 #include <cstdint>
@@ -153,8 +155,9 @@ __device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int n,
 #pragma unroll
   for (int e8 = 0; e8 < 8; ++e8) {
     const int t = t0 + e8;                   // column 128 h + 32 U + t
-    const int e = t >> 4;                    // low (t < 16) or high half
-    const int s = (e ? 31 : 15) - t;         // the shift that brings bit t to a sign
+    const int bt = (t & ~7) | ((t + 7) & 7); // its bit in the natural (rotated-byte) word
+    const int e = bt >> 4;                   // low (bit < 16) or high half
+    const int s = (e ? 31 : 15) - bt;        // the shift that brings that bit to a sign
     const int j = 2 * (64 * h + 16 * U + s) + e;
     const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
     asm volatile("st.shared.u16 [%0], %1;" ::"r"(tile + (uint32_t)((j >> 3) * (NN * 16) + (j & 7) * 2)),

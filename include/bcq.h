@@ -134,14 +134,16 @@ size_t bcq_workspace_bytes(int M, int N, int K);
  *
  *   x        device, fp16 [M][K] row-major, 16-byte aligned.
  *   planes   device, packed planes from bcq_pack_planes (p_H, N, K).
- *   alpha    HOST array of 4 device pointers; alpha[q-1] -> the scales of
- *            precision q (alpha^(q)[n][g][i], i = plane, canonically fp16
- *            [N][K/128][q]) packed by bcq_pack_scales(.., q, ..).  It must be
+ *   alpha    PACKED scales only: canonical [N][K/128][q] arrays are not
+ *            accepted (they would be read in the wrong order, with no error);
+ *            pass each through bcq_pack_scales(.., q, ..) first.  HOST array
+ *            of 4 device pointers; alpha[q-1] -> the packed scales of
+ *            precision q (alpha^(q)[n][g][i], i = plane).  It must be
  *            non-NULL for every precision used by the call; the others may be
  *            NULL.  16-byte aligned.
- *   z        device, the per-(row, group) offsets (canonically fp16
- *            [N][K/128]) packed by bcq_pack_scales(.., 1, ..), or NULL (= 0).
- *            16-byte aligned.
+ *   z        PACKED offsets only (canonical [N][K/128] arrays go through
+ *            bcq_pack_scales(.., 1, ..) first), or NULL (= 0).  16-byte
+ *            aligned.
  *   p        uniform precision 1..p_H for every row, or 0 to use p_row.
  *   p_row    HOST array int32 [M] of precisions 1..p_H (read during the call
  *            only), or NULL when p > 0.
@@ -158,10 +160,14 @@ size_t bcq_workspace_bytes(int M, int N, int K);
  *            BCQ_ERR_TIMEOUT).  Calls that may run at the same time (other
  *            streams) need workspaces of their own; calls in one stream may
  *            share one.
+ * Launches: one GEMV kernel per group of rows, each a cooperative launch of
+ * at most one CTA per SM: all its CTAs are resident at once, so the split-K
+ * reduction at its end (a CTA polls the partial sums other CTAs of the grid
+ * store) completes whatever else runs on the GPU.
  * The call reads planes 0..max_m(p_m)-1 only.  Accumulation is fp32; each
  * output is rounded once to fp16 (round to nearest even).  Partial sums over
- * 256-column K-blocks are added in K order, so for a given device and shape
- * the result does not depend on scheduling: results are reproducible.
+ * 256-column K-blocks are added in a fixed order, so for a given device and
+ * shape the result does not depend on scheduling: results are reproducible.
  * Errors: as listed above; workspace too small or NULL -> BCQ_ERR_NULL;
  * misaligned workspace -> BCQ_ERR_ALIGN.
  */
@@ -253,9 +259,12 @@ bcq_status bcq_gemm_host(const uint16_t* x_host, const uint32_t* planes,
  *     (16 MiB), held on every GPU that loads the library until the process
  *     exits.  A call whose bcq_workspace_bytes(M, N, K) exceeds it returns
  *     BCQ_ERR_SCRATCH and launches nothing; use bcq_gemm for such shapes.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on that device.
+ *   - Each call looks up the array's device address (cudaGetSymbolAddress,
+ *     with the call's device current) unless `stream` is capturing a CUDA
+ *     graph, when the address found by the last such lookup on that device
+ *     is used: make one call on a device before any stream capture on it.
+ *     (Looking it up again on every call keeps it right after a device or
+ *     context reset, which loads the library's device code anew.)
  *   - Each call clears the part of the scratch it uses (cudaMemsetAsync on
  *     `stream`) before its kernels.  Nothing is allocated, by this call or
  *     by any routine it calls.

@@ -59,7 +59,7 @@ def test_workspace_bytes_formula(L):
     # one K-block: no split over K, no workspace
     assert api.workspace_bytes(1, 4096, 256) == 0
     assert api.workspace_bytes(4, 4096, 128) == 0
-    # KB x min(M, 64) x rows (padded to 32) x 4 B of tagged partial sums
+    # KB x min(M, 64) x rows (padded to 32) x 4 B of partial sums
     assert api.workspace_bytes(1, 14336, 4096) == 16 * 1 * 14336 * 4
     assert api.workspace_bytes(8, 14336, 4096) == 16 * 8 * 14336 * 4
     assert api.workspace_bytes(64, 14336, 4096) == 16 * 64 * 14336 * 4
@@ -86,8 +86,25 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
     pl = api.plan_query(M, N, K, p, mixed=mixed, use_device=False)
     RB, KB = -(-N // 32), -(-K // 256)
     U = RB * KB
+    one_row = M == 1 and not mixed
+    even = min(U, KB * min(RB, 148 // KB)) if KB <= 148 else None
+    if one_row:
+        # the one-row kernel keeps whole K-blocks per CTA only while that
+        # leaves at most a tenth of the SMs idle, else every SM takes a share
+        assert pl["C"] == (even if even is not None and 10 * even >= 9 * min(U, 148)
+                           else min(U, 148))
+        # planes, scales alpha^(p) and offsets of one row group per stage,
+        # two teams of 8 consumer warps alternating stages, a 32 KiB table
+        assert pl["stage_bytes"] == 8192 * p + 1024 * p + 1024
+        assert pl["consumer_warps"] == 16
+        assert pl["dyn_bytes"] <= 232448
+        assert pl["dyn_bytes"] >= 32768 + pl["D"] * pl["stage_bytes"]
+        assert pl["D"] % 2 == 0 and pl["D"] % pl["NP"] == 0 and 2 <= pl["D"] <= 20
+        assert pl["D"] == 20 or pl["dyn_bytes"] + 2 * pl["stage_bytes"] > 232448
+        assert pl["units_max"] == -(-U // pl["C"])
+        return
     if KB <= 148:
-        assert pl["C"] == min(U, KB * min(RB, 148 // KB))   # whole K-blocks per CTA group
+        assert pl["C"] == even   # whole K-blocks per CTA group
         assert pl["C"] % KB == 0 or pl["C"] == U
     else:
         assert pl["C"] == 148

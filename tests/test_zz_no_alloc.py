@@ -4,15 +4,17 @@ Some callers cannot call cudaMalloc (code inside an allocator or memory pool,
 a plug-in whose host framework owns every device allocation, a loop that must
 not block on the driver's allocator), yet bcq_gemm needs split-K scratch from
 its caller.  bcq_gemm_noalloc takes that scratch from a static array built
-into the library.  These tests call it through the C ABI and check its output
-against bcq_gemm's (with a caller workspace) on two calls in a row, within
-the tolerance of the other parity tests.  The file is named to be collected
-last.
+into the library.  These tests call it through the C ABI on two calls in a
+row and check each result against the fp64 oracle (within the tolerance of
+the other parity tests) and bit for bit against bcq_gemm with a caller
+workspace: both run the same kernels in the same order, only the scratch
+differs.  The file is named to be collected last.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from bit_gemv_bcq_b200 import api, synth
 
 pytestmark = pytest.mark.gpu
@@ -29,11 +31,10 @@ def _cuda():
     assert api.device_error() == api.BCQ_OK
 
 
-def _close(y, y_ref, what):
+def _check_oracle(y, y_ref, what):
     a = y.float().cpu().numpy().astype(np.float64)
-    b = y_ref.float().cpu().numpy().astype(np.float64)
-    bad = np.abs(a - b) > ATOL + RTOL * np.abs(b)
-    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outputs differ"
+    bad = np.abs(a - y_ref) > ATOL + RTOL * np.abs(y_ref)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outputs outside tolerance"
 
 
 @pytest.mark.parametrize("N,K,M", [(4096, 4096, 1), (4096, 4096, 2), (1000, 2048, 5),
@@ -44,6 +45,7 @@ def test_noalloc_matches_gemm_twice_in_a_row(N, K, M):
     x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).cuda()
     assert api.workspace_bytes(M, N, K) <= api.NOALLOC_SCRATCH_BYTES
     for p in (2, 4):
+        y_ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p=p)
         ref = w.gemm(x, p=p)
         y1 = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
         y2 = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
@@ -51,8 +53,9 @@ def test_noalloc_matches_gemm_twice_in_a_row(N, K, M):
         api.gemm_noalloc(x, w, p=p, out=y2)   # second call reuses the same scratch
         torch.cuda.synchronize()
         assert api.device_error() == api.BCQ_OK
-        _close(y1, ref, f"first call N={N} K={K} M={M} p={p}")
-        _close(y2, ref, f"second call N={N} K={K} M={M} p={p}")
+        for y, which in ((y1, "first"), (y2, "second")):
+            _check_oracle(y, y_ref, f"{which} call N={N} K={K} M={M} p={p}")
+            assert torch.equal(y, ref), f"{which} call N={N} K={K} M={M} p={p}: not bcq_gemm's bits"
 
 
 def test_noalloc_mixed_precision_rows():
@@ -60,12 +63,14 @@ def test_noalloc_mixed_precision_rows():
     prob = synth.make_problem(N, K, M, seed=11)
     w = api.BcqWeights.from_canonical(prob.planes, prob.alphas, prob.z)
     x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).cuda()
-    p_row = [2, 4, 3, 2]
+    p_row = np.array([2, 4, 3, 2], dtype=np.int32)
+    y_ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=p_row)
     ref = w.gemm(x, p_row=p_row)
     for _ in range(2):
         y = api.gemm_noalloc(x, w, p_row=p_row)
         torch.cuda.synchronize()
-        _close(y, ref, "mixed precisions")
+        _check_oracle(y, y_ref, "mixed precisions")
+        assert torch.equal(y, ref)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

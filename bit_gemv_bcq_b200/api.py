@@ -71,6 +71,8 @@ def lib():
         L.bcq_packed_scales_bytes.argtypes = [I, I, I]
         L.bcq_pack_scales.restype = I
         L.bcq_pack_scales.argtypes = [P, I, I, I, P, P]
+        L.bcq_route_query.restype = I
+        L.bcq_route_query.argtypes = [I, I, P, I, I, P, I]
         L.bcq_set_pdl.restype = I
         L.bcq_set_pdl.argtypes = [I]
         L.bcq_workspace_bytes.restype = S
@@ -101,7 +103,7 @@ def lib():
 
 EXPORTED = ("bcq_status_string", "bcq_version", "bcq_packed_planes_bytes",
             "bcq_pack_planes", "bcq_packed_scales_bytes", "bcq_pack_scales",
-            "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_set_pdl",
+            "bcq_workspace_bytes", "bcq_gemm", "bcq_plan_query", "bcq_route_query", "bcq_set_pdl",
             "bcq_gemm_host", "bcq_gemm_noalloc", "bcq_build_lut", "bcq_device_error",
             "bcq_debug_wait_timeout", "bcq_quantize", "bcq_gemm_zp", "bcq_quantize_zp")
 
@@ -232,6 +234,22 @@ def plan_query(M: int, N: int, K: int, p_load: int, mixed: bool = False,
     _check(lib().bcq_plan_query(M, N, K, p_load, int(mixed), int(use_device),
                                 ctypes.cast(out, ctypes.c_void_p)), "bcq_plan_query")
     return dict(zip(PLAN_FIELDS, list(out)))
+
+
+KERNEL_NAMES = {1: "lut_pair", 2: "lut_one", 3: "lut_four", 4: "mma", 5: "mma_mixed",
+                6: "tcgen05"}
+
+
+def route_query(M: int, N: int, K: int, p: int | None = None, p_row=None) -> list:
+    """The launches bcq_gemm makes for M rows (see bcq_route_query):
+    [(kernel name, rows, planes streamed), ...]."""
+    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
+    out = (ctypes.c_int * (1 + 3 * 64))()
+    _check(lib().bcq_route_query(M, pv, pr_ptr, N, K, ctypes.cast(out, ctypes.c_void_p), 64),
+           "bcq_route_query")
+    del pr_keep
+    return [(KERNEL_NAMES[out[1 + 3 * i]], out[2 + 3 * i], out[3 + 3 * i])
+            for i in range(min(out[0], 64))]
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:

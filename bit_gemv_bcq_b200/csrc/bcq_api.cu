@@ -30,7 +30,7 @@ enum GemvPath { kPathLut = 0, kPathMmaSync = 1, kPathUmma = 2, kPathLut4 = 3, kP
 
 // One-row launches: the dense-table kernel (bcq_m1.cuh) unless
 // BCQ_M1_KIND=pair asks for the pair-table kernel with one row.
-bool use_m1_kernel() {
+bool use_m1_kernel(int /*K*/) {
   const char* v = std::getenv("BCQ_M1_KIND");
   return !(v && std::strcmp(v, "pair") == 0);
 }
@@ -122,14 +122,14 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   Plan pl;
   const int NN = M > kMmaRows ? kMaxLaunchRows : kMmaRows;  // tcgen05: 16 or 64 rows
   pl.fn = path == kPathUmma      ? gemv_umma_kernel_for(P, NN)
-          : path == kPathMmaSync ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P)
+          : path == kPathMmaSync ? gemv_mma_kernel_for(M > 8 ? 2 : 1, P, mixed)
           : path == kPathM1      ? gemv_m1_kernel_for(P)
                                  : gemv_kernel_for(M, P, mixed);
   if (!pl.fn) return BCQ_ERR_UNSUPPORTED;
   auto dyn_of = [&](int d) {
     return path == kPathUmma      ? (NN == kMmaRows ? umma_dyn_bytes<16>(d, P)
                                                      : umma_dyn_bytes<64>(d, P))
-           : path == kPathMmaSync ? mma_dyn_bytes(d, P)
+           : path == kPathMmaSync ? mma_dyn_bytes(d, P, mixed)
            : path == kPathM1      ? m1_dyn_bytes(d, P)
                                   : gemv_dyn_bytes(d, P, M);
   };
@@ -285,103 +285,158 @@ void fill_common(GemvParams& g, const Plan& pl, const uint32_t* planes, int N, i
 // off (for comparison only: the tail then assumes the grid fits at once).
 bool cooperative_launch() { return env_int("BCQ_COOPERATIVE", 1) != 0; }
 
-// Small batches: lookup-table launches of at most two rows, in order; two
-// rows with different precisions share one launch (planes streamed up to
-// the larger one).  Larger batches, per precision (rows grouped by
-// precision, in order): tcgen05 launches of up to 64 rows while at least 32
-// rows are left (measured: 64 rows in one launch cost 0.6 of four 16-row
-// launches), then tensor-core launches of 16 rows, then one for a
-// remainder of at least BCQ_MMA_MIN_ROWS rows, else a lookup launch per
-// remaining row.
+// One launch of a call: the kernel, the rows of x and y it takes (in launch
+// order) and their precisions.
+struct Launch {
+  int path = kPathLut;  // kPathLut (pair tables, 1-2 rows), kPathM1, kPathLut4, kPathMmaSync, kPathUmma
+  bool mixed = false;   // rows of several precisions
+  int n = 0;            // rows
+  int P = 0;            // planes streamed: the largest precision
+  int row[kMaxLaunchRows];
+  int q[kMaxLaunchRows];
+};
+
+// The launches of one call (no device work; bcq_gemm and the queries share
+// it).  Rows of one precision, M >= BCQ_MMA_MIN_ROWS (3): tcgen05 launches
+// of up to 64 rows while at least 32 are left (measured: 64 rows in one
+// launch cost 0.6 of four 16-row launches), a four-row lookup launch for a
+// group of 3-4 rows (measured on 14336 x 4096: p = 2 / 3 / 4 in 17.2 / 23.6 /
+// 26.2 us against 22.9 / 29.6 / 36.6 us on the tensor-core kernel;
+// BCQ_LUT4_MAX_ROWS=0 turns it off, BCQ_LUT4_MIN_BITS sets a precision
+// threshold), tensor-core launches of up to 16 rows, lookup launches for a
+// remainder of 1-2 rows.  Rows of several precisions (per-request
+// precision): up to 16 rows are one mixed tensor-core launch that streams
+// the planes once, up to the largest precision, each row applying its own
+// scales and offsets; larger batches are grouped by precision as above and
+// the rows left over in every group share mixed launches (16 rows at most
+// each).  Fewer than BCQ_MMA_MIN_ROWS rows: lookup launches of two rows,
+// mixed or not.  One-row lookup launches use the dense-table kernel.
+int route_call(int M, int p, const int32_t* p_row, int K, Launch* out) {
+  const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
+  const int lut4_max = std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4));
+  const int lut4_bits = env_int("BCQ_LUT4_MIN_BITS", 1);
+  const int tc = batch_path();
+  auto qof = [&](int m) { return p > 0 ? p : p_row[m]; };
+  int n = 0;
+  auto add = [&](int path, const int* rows, int cnt) {
+    Launch& L = out[n++];
+    L.path = path;
+    L.n = cnt;
+    L.P = 0;
+    bool mixed = false;
+    for (int j = 0; j < cnt; ++j) {
+      L.row[j] = rows[j];
+      L.q[j] = qof(rows[j]);
+      L.P = std::max(L.P, L.q[j]);
+      mixed = mixed || L.q[j] != L.q[0];
+    }
+    L.mixed = mixed;
+    if (path == kPathLut && cnt == 1 && use_m1_kernel(K)) L.path = kPathM1;
+  };
+  auto pairs = [&](const int* rows, int cnt) {
+    for (int j = 0; j < cnt; j += kMaxMPerLaunch) add(kPathLut, rows + j, std::min(kMaxMPerLaunch, cnt - j));
+  };
+  int all[BCQ_MAX_M];
+  bool uniform = true;
+  for (int m = 0; m < M; ++m) {
+    all[m] = m;
+    uniform = uniform && qof(m) == qof(0);
+  }
+  if (M < mma_min) {
+    pairs(all, M);
+    return n;
+  }
+  // (BCQ_MIXED_LAUNCH=0: mixed batches grouped by precision, for comparison)
+  const bool mixed_launch = env_int("BCQ_MIXED_LAUNCH", 1) != 0;
+  if (!uniform && mixed_launch && M <= kMmaRows) {
+    add(kPathMmaSync, all, M);
+    return n;
+  }
+  int left_rows[BCQ_MAX_M];
+  int nleft = 0;
+  for (int q = 1; q <= 4; ++q) {
+    int rows[BCQ_MAX_M];
+    int cnt = 0;
+    for (int m = 0; m < M; ++m)
+      if (qof(m) == q) rows[cnt++] = m;
+    for (int r0 = 0; r0 < cnt;) {
+      const int left = cnt - r0;
+      if (left >= 2 * kMmaRows) {
+        const int c = std::min(kMaxLaunchRows, left);
+        add(kPathUmma, rows + r0, c);
+        r0 += c;
+      } else if (left >= mma_min && left <= lut4_max && q >= lut4_bits) {
+        add(kPathLut4, rows + r0, left);
+        r0 += left;
+      } else if (left >= mma_min) {
+        const int c = std::min(kMmaRows, left);
+        add(tc, rows + r0, c);
+        r0 += c;
+      } else {
+        for (int j = r0; j < cnt; ++j) left_rows[nleft++] = rows[j];
+        r0 = cnt;
+      }
+    }
+  }
+  // rows left over in every precision group
+  if (mixed_launch) {
+    int r0 = 0;
+    while (nleft - r0 >= mma_min) {
+      const int c = std::min(kMmaRows, nleft - r0);
+      add(kPathMmaSync, left_rows + r0, c);
+      r0 += c;
+    }
+    pairs(left_rows + r0, nleft - r0);
+  } else {
+    pairs(left_rows, nleft);
+  }
+  return n;
+}
+
 bcq_status run_gemm(const uint16_t* x, const uint32_t* planes, const uint16_t* const alpha[4],
                     const uint16_t* const zq[4], int p, const int32_t* p_row, int M, int N, int K,
                     int p_H, uint16_t* y, void* ws, cudaStream_t st) {
   const int pdl_mode = g_pdl_mode.load();
   const int wait_us = env_int("BCQ_WAIT_LIMIT_US", 0);
-  const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
-  if (M >= mma_min) {
-    const int path = batch_path();
-    // batches of 3-4 rows of one precision: one lookup launch over two pair
-    // tables (measured on 14336 x 4096: p = 2 / 3 / 4 in 17.2 / 23.6 /
-    // 26.2 us against 22.9 / 29.6 / 36.6 us on the tensor-core kernel).
-    // BCQ_LUT4_MAX_ROWS=0 turns it off, BCQ_LUT4_MIN_BITS sets a precision
-    // threshold.
-    const int lut4_max = std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4));
-    const int lut4_bits = env_int("BCQ_LUT4_MIN_BITS", 1);
-    for (int q = 1; q <= 4; ++q) {
-      int rows[BCQ_MAX_M];
-      int n = 0;
-      for (int m = 0; m < M; ++m)
-        if ((p > 0 ? p : p_row[m]) == q) rows[n++] = m;
-      for (int r0 = 0; r0 < n;) {
-        const int left = n - r0;
-        int cnt, qpath;
-        if (left >= 2 * kMmaRows) {
-          cnt = std::min(kMaxLaunchRows, left);
-          qpath = kPathUmma;
-        } else if (left >= mma_min && left <= lut4_max && q >= lut4_bits) {
-          cnt = left;  // one lookup launch over four-row pair tables
-          qpath = kPathLut4;
-        } else if (left >= mma_min) {
-          cnt = std::min(kMmaRows, left);
-          qpath = path;
-        } else {
-          cnt = 1;
-          qpath = kPathLut;
-        }
-        if (qpath == kPathLut && use_m1_kernel()) qpath = kPathM1;
-        Plan pl;
-        bcq_status s = qpath == kPathLut4 ? plan_gemv(4, N, K, q, false, kPathLut, &pl)
-                                          : plan_gemv(cnt, N, K, q, false, qpath, &pl);
-        if (s != BCQ_OK) return s;
-        GemvParams g{};
-        fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);
-        g.alpha[0] = g.alpha[1] = alpha[q - 1];
-        g.z = g.z1 = zq[q - 1];
-        g.M = cnt;
-        g.q[0] = g.q[1] = q;
-        if (qpath == kPathLut || qpath == kPathM1) {  // one row, addressed directly
-          g.x = x + (size_t)rows[r0] * K;
-          g.y = y + (size_t)rows[r0] * N;
-        } else {
-          g.x = x;
-          g.y = y;
-          for (int j = 0; j < cnt; ++j) g.rows[j] = rows[r0 + j];
-        }
-        if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st, pl.CW, cooperative_launch()) !=
-            cudaSuccess)
-          return BCQ_ERR_CUDA;
-        r0 += cnt;
-      }
-    }
-    return BCQ_OK;
-  }
-  for (int m0 = 0; m0 < M;) {
-    const int rows = std::min(kMaxMPerLaunch, M - m0);
-    int q[2];
-    for (int r = 0; r < kMaxMPerLaunch; ++r)
-      q[r] = p > 0 ? p : p_row[m0 + std::min(r, rows - 1)];
-    const int P = std::max(q[0], q[1]);
-    const bool mixed = q[0] != q[1];
-    const int path = rows == 1 && use_m1_kernel() ? kPathM1 : kPathLut;
+  static thread_local Launch launches[BCQ_MAX_M];
+  const int n = route_call(M, p, p_row, K, launches);
+  for (int li = 0; li < n; ++li) {
+    const Launch& L = launches[li];
     Plan pl;
-    bcq_status s = plan_gemv(rows, N, K, P, mixed, path, &pl);
+    const int plan_rows = L.path == kPathLut4 ? 4 : L.n;
+    const int plan_path = L.path == kPathLut4 ? kPathLut : L.path;
+    bcq_status s = plan_gemv(plan_rows, N, K, L.P, L.mixed, plan_path, &pl);
     if (s != BCQ_OK) return s;
     GemvParams g{};
     fill_common(g, pl, planes, N, K, p_H, ws, pdl_mode, wait_us);
-    g.z = zq[q[0] - 1];
-    g.z1 = zq[q[1] - 1];
-    g.x = x + (size_t)m0 * K;
-    g.y = y + (size_t)m0 * N;
-    g.alpha[0] = alpha[q[0] - 1];
-    g.alpha[1] = alpha[q[1] - 1];
-    g.M = rows;
-    g.q[0] = q[0];
-    g.q[1] = q[1];
+    g.M = L.n;
+    g.q[0] = L.q[0];
+    g.q[1] = L.q[L.n > 1 ? 1 : 0];
+    g.alpha[0] = alpha[g.q[0] - 1];
+    g.alpha[1] = alpha[g.q[1] - 1];
+    g.z = zq[g.q[0] - 1];
+    g.z1 = zq[g.q[1] - 1];
+    if (L.path == kPathM1 || (L.path == kPathLut && L.n == 1)) {  // one row, addressed directly
+      g.x = x + (size_t)L.row[0] * K;
+      g.y = y + (size_t)L.row[0] * N;
+    } else {
+      g.x = x;
+      g.y = y;
+      for (int j = 0; j < L.n; ++j) {
+        g.rows[j] = L.row[j];
+        g.qrow[j] = L.q[j];
+      }
+    }
+    if (L.mixed && L.path == kPathMmaSync) {
+      for (int q = 1; q <= 4; ++q) {
+        g.alpha_q[q - 1] = alpha[q - 1];
+        g.z_q[q - 1] = zq[q - 1];
+      }
+      for (int j = 0; j < L.n; ++j) g.qmask |= 1 << L.q[j];
+    }
     if (launch_gemv(pl.fn, g, pl.dyn, pdl_mode != 0, st, pl.CW, cooperative_launch()) !=
         cudaSuccess)
       return BCQ_ERR_CUDA;
-    m0 += rows;
   }
   return BCQ_OK;
 }
@@ -460,15 +515,18 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
   if (!out) return BCQ_ERR_NULL;
   if (M < 1 || M > kMaxLaunchRows || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
   if (p_load < 1 || p_load > 4) return BCQ_ERR_PRECISION;
-  if (mixed && (M != 2 || p_load < 2)) return BCQ_ERR_PRECISION;
-  // 3-4 rows: the four-row lookup launch bcq_gemm would use (same switches)
-  const bool lut4 = !mixed && M > kMaxMPerLaunch &&
+  if (mixed && (M < 2 || M > kMmaRows || p_load < 2)) return BCQ_ERR_PRECISION;
+  // the kernel bcq_gemm gives a launch of M rows (route_call's rules)
+  const int mma_min = std::max(1, env_int("BCQ_MMA_MIN_ROWS", kDefaultMmaMinRows));
+  const bool lut4 = !mixed && M > kMaxMPerLaunch && M >= mma_min &&
                     M <= std::min(4, env_int("BCQ_LUT4_MAX_ROWS", 4)) &&
                     p_load >= env_int("BCQ_LUT4_MIN_BITS", 1);
-  const int path = lut4 ? kPathLut
-                   : M > kMmaRows ? kPathUmma
-                   : M > kMaxMPerLaunch ? batch_path()
-                   : M == 1 && !mixed && use_m1_kernel() ? kPathM1 : kPathLut;
+  int path;
+  if (M <= kMaxMPerLaunch) path = M == 1 && !mixed && use_m1_kernel(K) ? kPathM1 : kPathLut;
+  else if (mixed) path = kPathMmaSync;
+  else if (lut4) path = kPathLut;
+  else if (M > kMmaRows) path = kPathUmma;
+  else path = batch_path();
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   t_virtual = !use_device || cudaGetDevice(&dev) != cudaSuccess;
@@ -485,6 +543,30 @@ int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, i
   out[5] = (int)(path == kPathM1 ? m1_stage_bytes(p_load) : gemv_stage_bytes(p_load));
   out[6] = (int)pl.units_max;
   out[7] = pl.KB;
+  return BCQ_OK;
+}
+
+int bcq_route_query(int M, int p, const int32_t* p_row, int N, int K, int* out,
+                    int max_launches) {
+  if (!out || max_launches < 0) return BCQ_ERR_NULL;
+  if (M < 1 || M > BCQ_MAX_M || !shape_ok(N, K)) return BCQ_ERR_SHAPE;
+  if (p < 0 || p > 4 || (p == 0 && !p_row)) return BCQ_ERR_PRECISION;
+  for (int m = 0; m < M && p == 0; ++m)
+    if (p_row[m] < 1 || p_row[m] > 4) return BCQ_ERR_PRECISION;
+  static thread_local Launch launches[BCQ_MAX_M];
+  const int n = route_call(M, p, p_row, K, launches);
+  out[0] = n;
+  for (int i = 0; i < n && i < max_launches; ++i) {
+    const Launch& L = launches[i];
+    int kind = BCQ_KERNEL_LUT_PAIR;
+    if (L.path == kPathM1) kind = BCQ_KERNEL_LUT_ONE;
+    else if (L.path == kPathLut4) kind = BCQ_KERNEL_LUT_FOUR;
+    else if (L.path == kPathMmaSync) kind = L.mixed ? BCQ_KERNEL_MMA_MIXED : BCQ_KERNEL_MMA;
+    else if (L.path == kPathUmma) kind = BCQ_KERNEL_TCGEN05;
+    out[1 + 3 * i] = kind;
+    out[2 + 3 * i] = L.n;
+    out[3 + 3 * i] = L.P;
+  }
   return BCQ_OK;
 }
 

@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   uint4 xv[M];
   if (warp < kConsumerWarps) {
     grid_dependency_wait();
-    load_x<M>(prm.x, prm.K, R.kb0, lane, xv, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
+    load_x<M>(prm.x, prm.K, R.kb0, lane, xv, M == 4 ? prm.M : M, M >= 2 ? prm.rows : nullptr);
   }
   if (warp == 0) {
     if (cfg_ok && lane < D) {  // one lane per ring slot
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 #pragma unroll
       for (int m = 0; m < M; ++m)
         if (M < 4 || m < prm.M)
-          prm.y[(size_t)(M == 4 ? prm.rows[m] : m) * prm.N + row] = f2h_rn(r[m]);
+          prm.y[(size_t)(M >= 2 ? prm.rows[m] : m) * prm.N + row] = f2h_rn(r[m]);
     }
   };
 
@@ -512,13 +512,13 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 #pragma unroll
           for (int m = 0; m < M; ++m) xv[m] = xn[m];
         } else {
-          load_x<M>(prm.x, prm.K, kbn, lane, xv, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr);
+          load_x<M>(prm.x, prm.K, kbn, lane, xv, M == 4 ? prm.M : M, M >= 2 ? prm.rows : nullptr);
         }
       }
       // the next K-block's x is fetched a table ahead (four-row launches
       // load it when needed: its registers would spill in the main loop)
       if (M != 4 && kbn < R.kb_last) {
-        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn);
+        load_x<M>(prm.x, prm.K, kbn + 1, lane, xn, M, M >= 2 ? prm.rows : nullptr);
         xn_kb = kbn + 1;
       }
       // M = 2 has one table: every warp must be done with the old one.
@@ -665,7 +665,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   if (prm.KB > 1) {
     // (rows: compile-time for one- and two-row launches, so the tail keeps
     // only the loads it needs in registers)
-    splitk_tail<M == 1 ? 16 : 8>(prm, R, M == 4 ? prm.M : M, M == 4 ? prm.rows : nullptr, tid,
+    splitk_tail<M == 1 ? 16 : 8>(prm, R, M == 4 ? prm.M : M, M >= 2 ? prm.rows : nullptr, tid,
                                  kConsumers, abort_flag);
   }
 }
@@ -812,7 +812,26 @@ GemvKernel gemv_m1_kernel_for(int P) {
   }
 }
 
-GemvKernel gemv_mma_kernel_for(int NT, int P) {
+GemvKernel gemv_mma_kernel_for(int NT, int P, bool mixed) {
+  if (mixed) {
+    if (NT == 1) {
+      switch (P) {
+        case 2: return gemv_mma_kernel<1, 2, true>;
+        case 3: return gemv_mma_kernel<1, 3, true>;
+        case 4: return gemv_mma_kernel<1, 4, true>;
+        default: return nullptr;
+      }
+    }
+    if (NT == 2) {
+      switch (P) {
+        case 2: return gemv_mma_kernel<2, 2, true>;
+        case 3: return gemv_mma_kernel<2, 3, true>;
+        case 4: return gemv_mma_kernel<2, 4, true>;
+        default: return nullptr;
+      }
+    }
+    return nullptr;
+  }
   if (NT == 1) {
     switch (P) {
       case 1: return gemv_mma_kernel<1, 1>;

@@ -27,8 +27,9 @@ GemvKernel gemv_kernel_for(int M, int P, bool mixed);
 GemvKernel gemv_m1_kernel_for(int P);
 
 // The tensor-core GEMV kernel for NT n-tiles of 8 activation rows (1 or 2)
-// streaming P planes (one precision); nullptr if there is none.
-GemvKernel gemv_mma_kernel_for(int NT, int P);
+// streaming P planes (one precision, or mixed: rows of precisions up to P);
+// nullptr if there is none.
+GemvKernel gemv_mma_kernel_for(int NT, int P, bool mixed);
 
 // The tcgen05 GEMV kernel for up to NN (16 or 64) activation rows streaming
 // P planes (one precision); nullptr if there is none.

@@ -144,17 +144,26 @@ constexpr int kXPitch = 264;                 // halves per row of the activation
 constexpr uint32_t kXTileBytes = kMmaRows * kXPitch * 2;            // 8448
 constexpr uint32_t kMmaGsumOff = 2 * kXTileBytes;                    // 16896
 constexpr uint32_t kMmaScaleOff = kMmaGsumOff + 2 * kMmaRows * 2 * 4; // 17152
-__host__ __device__ constexpr uint32_t mma_scale_buf_bytes(int P) {  // one warp, one group
-  return (uint32_t)32 * (2 * P + 2) * 2;
+// Scales staged per warp and unit: 32 lanes x 2P halves of alpha^(P), then
+// the offsets (2 halves a lane).  Mixed launches (rows of several
+// precisions) stage alpha^(q) of every precision q = 1..4 present, each in
+// its own block of 32 x 2q halves at byte 64 q (q - 1), and the offsets of
+// each precision q present at byte 1280 + 128 (q - 1).
+__host__ __device__ constexpr uint32_t mma_scale_buf_bytes(int P, bool mixed = false) {
+  return mixed ? 1280u + 4u * 128u : (uint32_t)32 * (2 * P + 2) * 2;
 }
-__host__ __device__ constexpr uint32_t mma_ring_off(int P) {
-  return (kMmaScaleOff + 16u * 2u * mma_scale_buf_bytes(P) + 1023u) & ~1023u;
+__host__ __device__ constexpr uint32_t mma_z_off(int P, bool mixed = false, int q = 1) {
+  return mixed ? 1280u + 128u * (uint32_t)(q - 1) : 128u * (uint32_t)P;
 }
-__host__ __device__ constexpr uint32_t mma_off_bar(int D, int P) {
-  return mma_ring_off(P) + (uint32_t)D * gemv_stage_bytes(P);
+__host__ __device__ constexpr uint32_t mma_alpha_block(int q) { return 64u * (uint32_t)q * (uint32_t)(q - 1); }
+__host__ __device__ constexpr uint32_t mma_ring_off(int P, bool mixed = false) {
+  return (kMmaScaleOff + 16u * 2u * mma_scale_buf_bytes(P, mixed) + 1023u) & ~1023u;
 }
-__host__ __device__ constexpr uint32_t mma_dyn_bytes(int D, int P) {
-  return mma_off_bar(D, P) + 16u * (uint32_t)D + 16u;
+__host__ __device__ constexpr uint32_t mma_off_bar(int D, int P, bool mixed = false) {
+  return mma_ring_off(P, mixed) + (uint32_t)D * gemv_stage_bytes(P);
+}
+__host__ __device__ constexpr uint32_t mma_dyn_bytes(int D, int P, bool mixed = false) {
+  return mma_off_bar(D, P, mixed) + 16u * (uint32_t)D + 16u;
 }
 
 // The tcgen05 GEMV (bcq_umma.cuh), for NN = 16 or 64 activation rows per
@@ -224,6 +233,13 @@ struct GemvParams {
   int early_weights;         // with PDL: stream weights before the grid wait
   unsigned long long timeout_ns;
   int rows[kMaxLaunchRows];  // tensor-core launches: x / y row of launch row m
+  // mixed tensor-core launches: precision of launch row m, packed scales and
+  // offsets of each precision q (alpha_q[q - 1], z_q[q - 1]) and the
+  // precisions present (bit q)
+  int qrow[kMaxLaunchRows];
+  const uint16_t* alpha_q[4];
+  const uint16_t* z_q[4];    // their offsets (or nullptr: none)
+  int qmask;
   CtaWork work[kMaxCtas];    // per CTA (C entries)
 };
 

@@ -79,10 +79,38 @@ __device__ __forceinline__ void cp_async_wait() {
 // Lane l of a warp copies row l's scales (2P halves: pass 0 then pass 1) and
 // offsets (2 halves) of unit (kb, rb) into buf: alpha at l * 4P bytes, z at
 // 128P + 4l.  Packed layouts: bcq_layout.h.
-template <int P>
+// (MIXED: the scales of every precision q present, each into its own block
+// of the buffer, see mma_scale_buf_bytes.)
+template <int Q>
+__device__ __forceinline__ void stage_alpha_q(const uint16_t* a, uint32_t da) {
+  if (Q == 1) {
+    cp_async4(da, a);
+  } else if (Q == 2) {
+    cp_async8(da, a);
+  } else if (Q == 3) {
+    cp_async4(da, a);
+    cp_async4(da + 4u, a + 2);
+    cp_async4(da + 8u, a + 4);
+  } else {
+    cp_async16(da, a);
+  }
+}
+
+template <int P, bool MIXED = false>
 __device__ __forceinline__ void stage_scales(const GemvParams& prm, int kb, int rb, int lane,
                                              uint32_t buf) {
   const size_t e = ((size_t)kb * prm.RB + rb) * kRowBlock + lane;
+  if constexpr (MIXED) {
+    if (prm.qmask & 2) stage_alpha_q<1>(prm.alpha_q[0] + e * 2, buf + mma_alpha_block(1) + 4u * lane);
+    if (prm.qmask & 4) stage_alpha_q<2>(prm.alpha_q[1] + e * 4, buf + mma_alpha_block(2) + 8u * lane);
+    if (prm.qmask & 8) stage_alpha_q<3>(prm.alpha_q[2] + e * 6, buf + mma_alpha_block(3) + 12u * lane);
+    if (prm.qmask & 16) stage_alpha_q<4>(prm.alpha_q[3] + e * 8, buf + mma_alpha_block(4) + 16u * lane);
+#pragma unroll
+    for (int q = 1; q <= 4; ++q)
+      if (((prm.qmask >> q) & 1) && prm.z_q[q - 1])
+        cp_async4(buf + mma_z_off(P, true, q) + 4u * lane, prm.z_q[q - 1] + e * 2);
+    return;
+  }
   const uint16_t* a = prm.alpha[0] + e * (2 * P);
   const uint32_t da = buf + (uint32_t)lane * (4u * P);
   if (P == 1) {
@@ -144,10 +172,17 @@ __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, i
 // moving the two bits to bit 7 of their byte (shifts by (8 - 2q) mod 8 and
 // 7 - 2q), replicating each into a sign byte (prmt) and xoring the fp16 sign
 // bits of alpha2 (lop3).
-template <int NT, int P>
+// MIXED: the rows of the launch have precisions of their own (qm[nt][c]:
+// activation row nt * 8 + 2q + c, 0 past the launch's rows).  The fragments
+// then hold +-1 (exact), each (plane, group) product is accumulated apart
+// and folded into acc[0] with alpha^(qm)[row][group][i] of each activation
+// row (zero for a plane i >= qm): the same sum, with each row's own scales;
+// acc[1] stays zero.
+template <int NT, int P, bool MIXED = false>
 __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sbuf, int i,
                                           int g, int q, uint32_t ra0, uint32_t ra1, uint32_t dsh,
-                                          float (&acc)[2][2][NT][4]) {
+                                          float (&acc)[2][2][NT][4],
+                                          const int (&qm)[NT][2]) {
   const uint32_t sh1 = (8u - 2u * (uint32_t)q) & 7u, sh2 = 7u - 2u * (uint32_t)q;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -176,10 +211,21 @@ __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sb
       for (int v = 0; v < 4; ++v) w[v] = lds_u32(base + (((uint32_t)v - ra) & 3u) * 4u);
 #pragma unroll
       for (int v = 0; v < 4; ++v) nw[j][v] = funnel_r(w[v], w[(v + 1) & 3], dsh);
-      // alpha of (row, group h, plane i) in both halves
-      const uint32_t ah = lds_u16(sbuf + ((uint32_t)r * 2u * P + (uint32_t)pass * P + i) * 2u);
-      al[j] = ah | (ah << 16);
+      // alpha of (row, group h, plane i) in both halves (MIXED: +1)
+      if constexpr (MIXED) {
+        al[j] = 0x3C003C00u;
+      } else {
+        const uint32_t ah = lds_u16(sbuf + ((uint32_t)r * 2u * P + (uint32_t)pass * P + i) * 2u);
+        al[j] = ah | (ah << 16);
+      }
     }
+    float tmp[2][NT][4];  // MIXED: this (plane, group) alone
+#pragma unroll
+    for (int f = 0; f < 2; ++f)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tmp[f][nt][e] = 0.f;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       uint32_t x1[4], x2[4];
@@ -202,12 +248,35 @@ __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sb
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           // tile f: rows 16 f + g (j = 2f) and 16 f + g + 8 (j = 2f + 1)
-          mma_16816(acc[h][0][nt], a[0][0], a[1][0], a[0][1], a[1][1], bf[s8][nt][0],
-                    bf[s8][nt][1]);
-          mma_16816(acc[h][1][nt], a[2][0], a[3][0], a[2][1], a[3][1], bf[s8][nt][0],
-                    bf[s8][nt][1]);
+          mma_16816(MIXED ? tmp[0][nt] : acc[h][0][nt], a[0][0], a[1][0], a[0][1], a[1][1],
+                    bf[s8][nt][0], bf[s8][nt][1]);
+          mma_16816(MIXED ? tmp[1][nt] : acc[h][1][nt], a[2][0], a[3][0], a[2][1], a[3][1],
+                    bf[s8][nt][0], bf[s8][nt][1]);
         }
       }
+    }
+    if constexpr (MIXED) {
+      // fold: element e of tile f is weight row 16 f + g + 8 (e / 2) and
+      // activation row nt * 8 + 2q + (e % 2)
+#pragma unroll
+      for (int f = 0; f < 2; ++f)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int r = 16 * f + g + 8 * hr;
+          const int pass = (r >> 4) ^ h;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int qv = qm[nt][c];
+              float al2 = 0.f;
+              if (i < qv)
+                al2 = h2f((uint16_t)lds_u16(sbuf + mma_alpha_block(qv) +
+                                            ((uint32_t)r * 2u * qv + (uint32_t)pass * qv + i) * 2u));
+              // (both groups into acc[0]: the epilogue adds acc[0] + acc[1])
+              acc[0][f][nt][2 * hr + c] = fmaf(al2, tmp[f][nt][2 * hr + c], acc[0][f][nt][2 * hr + c]);
+            }
+        }
     }
   }
 }
@@ -218,7 +287,8 @@ __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sb
 // the planes.  Each K-block's activation tile is loaded by all 16 warps
 // (slot kb & 1) between the same kind of barriers as the table build.
 //   NT  n-tiles of 8 activation rows (M <= 8 NT), P  planes (one precision)
-template <int NT, int P>
+//   MIXED  the rows have precisions of their own (P: the largest)
+template <int NT, int P, bool MIXED = false>
 __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     gemv_mma_kernel(const __grid_constant__ GemvParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -228,10 +298,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   const int warp = tid >> 5;
   const int D = prm.D, NP = prm.NP, RB = prm.RB;
   constexpr uint32_t kStage = gemv_stage_bytes(P);
-  const uint32_t ring = sbase + mma_ring_off(P);
-  const uint32_t full0 = sbase + mma_off_bar(D, P);
+  const uint32_t ring = sbase + mma_ring_off(P, MIXED);
+  const uint32_t full0 = sbase + mma_off_bar(D, P, MIXED);
   const uint32_t empty0 = full0 + 8u * (uint32_t)D;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + mma_off_bar(D, P) + 16u * D);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(smem + mma_off_bar(D, P, MIXED) + 16u * D);
   constexpr int kConsumers = kConsumerWarps * 32;
 
   const bool cfg_ok = D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 && (D & 1) == 0 &&
@@ -271,8 +342,17 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   // rotation constants of this thread's rows (g and g + 8, mod 16)
   const uint32_t ra0 = (uint32_t)(((g + 3) >> 2) & 3), ra1 = (uint32_t)(((g + 11) >> 2) & 3);
   const uint32_t dsh = (uint32_t)((-g) & 3) * 8u;
-  const uint32_t sbuf0 = sbase + kMmaScaleOff + (uint32_t)warp * 2u * mma_scale_buf_bytes(P);
+  constexpr uint32_t kSbuf = mma_scale_buf_bytes(P, MIXED);
+  const uint32_t sbuf0 = sbase + kMmaScaleOff + (uint32_t)warp * 2u * kSbuf;
   const size_t part_stride = (size_t)RB * kRowBlock;
+  int qm[NT][2];  // MIXED: precision of this thread's activation rows
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int m = nt * 8 + 2 * q + c;
+      qm[nt][c] = MIXED && m < prm.M ? prm.qrow[m] : 0;
+    }
   int cur_kb = -1;
   uint4 xn = make_uint4(0u, 0u, 0u, 0u);
   int xn_kb = -1;
@@ -307,7 +387,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   // buffers per warp)
   GroupCursor pc = gc;
   int buf = 0;
-  if (gg < R.NG && tw < pc.n) stage_scales<P>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0);
+  if (gg < R.NG && tw < pc.n) stage_scales<P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0);
   cp_async_commit();
   cursor_next(pc, R.u1, RB);
   cursor_next(pc, R.u1, RB);
@@ -315,11 +395,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   while (gg < R.NG) {
     advance_tiles(gc.kb);
     const bool active = tw < gc.n;
-    const uint32_t sbuf = sbuf0 + (uint32_t)buf * mma_scale_buf_bytes(P);
+    const uint32_t sbuf = sbuf0 + (uint32_t)buf * kSbuf;
     // stage the next group's scales into the other buffer, then make sure
     // this group's have landed
     if (gg + 2 < R.NG && tw < pc.n)
-      stage_scales<P>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0 + (uint32_t)(buf ^ 1) * mma_scale_buf_bytes(P));
+      stage_scales<P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0 + (uint32_t)(buf ^ 1) * kSbuf);
     cp_async_commit();
     cp_async_wait<1>();
     __syncwarp();
@@ -342,8 +422,8 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
       const uint32_t st = ring + (uint32_t)s * kStage + (uint32_t)tw * kUnitPlaneBytes;
 #pragma unroll 1
       for (int i = 0; i < P; ++i)
-        mma_plane<NT, P>(st + (uint32_t)i * kPlaneGroupBytes, xt, sbuf, i, g, q, ra0, ra1, dsh,
-                         acc);
+        mma_plane<NT, P, MIXED>(st + (uint32_t)i * kPlaneGroupBytes, xt, sbuf, i, g, q, ra0, ra1,
+                                dsh, acc, qm);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive_cta(empty0 + 8u * s);
@@ -365,10 +445,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
         for (int hr = 0; hr < 2; ++hr) {
           const int r = 16 * f + g + 8 * hr;
           float zz[2] = {0.f, 0.f};
-          if (prm.z) {
+          if (!MIXED && prm.z) {
 #pragma unroll
             for (int h = 0; h < 2; ++h)
-              zz[h] = h2f((uint16_t)lds_u16(sbuf + 128u * P + (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
+              zz[h] = h2f((uint16_t)lds_u16(sbuf + mma_z_off(P) +
+                                            (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
           }
           const int row = (gc.rb0 + tw) * kRowBlock + r;
 #pragma unroll
@@ -376,6 +457,16 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const int m = nt * 8 + 2 * q + c;
+              if constexpr (MIXED) {  // the offsets of this activation row's precision
+                const int qv = qm[nt][c];
+                zz[0] = zz[1] = 0.f;
+                if (qv > 0 && prm.z_q[qv - 1]) {
+#pragma unroll
+                  for (int h = 0; h < 2; ++h)
+                    zz[h] = h2f((uint16_t)lds_u16(sbuf + mma_z_off(P, true, qv) +
+                                                  (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
+                }
+              }
               float v = acc[0][f][nt][2 * hr + c] + acc[1][f][nt][2 * hr + c];
               v = fmaf(zz[0], sg[nt][c][0], fmaf(zz[1], sg[nt][c][1], v));
               if (m < prm.M) {

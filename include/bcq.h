@@ -200,11 +200,13 @@ bcq_status bcq_gemm_zp(const uint16_t* x, const uint32_t* planes,
 
 /*
  * The launch plan bcq_gemm would use for one launch of M (1..64) activation
- * rows streaming p_load planes (mixed = 1: two rows of different
- * precisions).  M <= 2 plans the lookup-table kernel, 3 <= M <= 4 its
- * four-row launch (two pair tables), 5 <= M <= 16 the tensor-core kernel
- * that bcq_gemm would use for a batch (BCQ_MMA_KIND), and M >= 17 the
- * 64-row tcgen05 launch.  use_device = 1
+ * rows streaming p_load planes (mixed = 1: rows of different precisions, at
+ * most 16).  M = 1 plans the one-row lookup kernel (K > 256; else the
+ * pair-table kernel), M = 2 the pair-table kernel, mixed M >= 3 the mixed
+ * tensor-core kernel, 3 <= M <= 4 of one precision the four-row lookup
+ * launch (two pair tables), 5 <= M <= 16 the tensor-core kernel that
+ * bcq_gemm would use for a batch (BCQ_MMA_KIND), and M >= 17 the 64-row
+ * tcgen05 launch; the same switches as bcq_gemm apply.  use_device = 1
  * plans for the current device; 0 (or no usable device) plans for a nominal
  * 148-SM B200 without touching CUDA.  out[8] receives: CTAs, consumer warps,
  * producer warps, ring stages, dynamic shared memory bytes, bytes per ring
@@ -212,6 +214,31 @@ bcq_status bcq_gemm_zp(const uint16_t* x, const uint32_t* planes,
  * K-blocks (partial sums per output).  For inspection and tests.
  */
 int bcq_plan_query(int M, int N, int K, int p_load, int mixed, int use_device, int* out);
+
+/* Kernels of a launch, as bcq_route_query reports them. */
+enum {
+  BCQ_KERNEL_LUT_PAIR = 1,   /* lookup table, 1-2 rows (pair tables; mixed pairs) */
+  BCQ_KERNEL_LUT_ONE = 2,    /* lookup table, one row, dense table (K > 256) */
+  BCQ_KERNEL_LUT_FOUR = 3,   /* lookup table, 3-4 rows of one precision */
+  BCQ_KERNEL_MMA = 4,        /* tensor cores (mma.sync), up to 16 rows of one precision */
+  BCQ_KERNEL_MMA_MIXED = 5,  /* tensor cores (mma.sync), up to 16 rows of several precisions */
+  BCQ_KERNEL_TCGEN05 = 6     /* tensor cores (tcgen05), up to 64 rows of one precision */
+};
+
+/*
+ * The launches bcq_gemm (or bcq_gemm_zp) makes for M rows at precision p (or
+ * p_row, HOST [M], when p = 0) on an N x K weight, without launching
+ * anything (the same routing code): out[0] = number of launches L; for
+ * launch i < max_launches,
+ * out[1 + 3i], out[2 + 3i], out[3 + 3i] = kernel (BCQ_KERNEL_*), rows, planes
+ * streamed.  out needs 1 + 3 * max_launches ints.  A mixed batch of up to 16
+ * rows is one launch that streams the planes once, up to its largest
+ * precision (AnyBCQ page, "吞吐量": each request at its own precision).
+ * Errors: out NULL -> BCQ_ERR_NULL; M, N, K -> BCQ_ERR_SHAPE; p / p_row
+ * outside 1..4 -> BCQ_ERR_PRECISION.
+ */
+int bcq_route_query(int M, int p, const int32_t* p_row, int N, int K, int* out,
+                    int max_launches);
 
 /*
  * Launch option for the GEMV kernels of this process (all devices):

@@ -125,7 +125,9 @@ def test_plan_query_rejects_bad_arguments(L):
     with pytest.raises(api.BcqError):
         api.plan_query(65, 64, 256, 2)            # at most 64 rows per launch
     with pytest.raises(api.BcqError):
-        api.plan_query(4, 64, 256, 3, mixed=True)  # tensor-core launches: one precision
+        api.plan_query(17, 64, 256, 3, mixed=True)  # mixed launches: 16 rows at most
+    pl = api.plan_query(4, 64, 256, 3, mixed=True)  # the mixed tensor-core kernel
+    assert pl["stage_bytes"] == 8192 * 3
     with pytest.raises(api.BcqError):
         api.plan_query(1, 64, 200, 2)             # K % 128
     with pytest.raises(api.BcqError):
@@ -221,3 +223,56 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(api.BcqLibraryError):
         api.lib()
+
+
+# ---------------------------------------------------------------- routing
+
+def test_mixed_batches_of_up_to_16_rows_are_one_launch(L):
+    """Per-request precision (AnyBCQ page, 吞吐量): a batch whose rows use
+    different precisions streams the planes once, up to its largest
+    precision, in one launch (the mixed tensor-core kernel for 3-16 rows, the
+    mixed pair lookup launch for 2)."""
+    r = api.route_query(8, 28672, 8192, p_row=[4, 3, 3, 2, 2, 2, 2, 2])
+    assert r == [("mma_mixed", 8, 4)]
+    assert api.route_query(16, 4096, 4096, p_row=[2, 3, 4, 2] * 4) == [("mma_mixed", 16, 4)]
+    assert api.route_query(3, 4096, 4096, p_row=[2, 2, 3]) == [("mma_mixed", 3, 3)]
+    assert api.route_query(2, 4096, 4096, p_row=[2, 4]) == [("lut_pair", 2, 4)]
+
+
+def test_uniform_batches_keep_their_kernels(L):
+    assert api.route_query(1, 14336, 4096, p=2) == [("lut_one", 1, 2)]
+    assert api.route_query(2, 14336, 4096, p=3) == [("lut_pair", 2, 3)]
+    assert api.route_query(4, 14336, 4096, p=4) == [("lut_four", 4, 4)]
+    assert api.route_query(8, 14336, 4096, p=2) == [("mma", 8, 2)]
+    assert api.route_query(16, 14336, 4096, p=2) == [("mma", 16, 2)]
+    assert api.route_query(64, 14336, 4096, p=2) == [("tcgen05", 64, 2)]
+    assert api.route_query(17, 14336, 4096, p=2) == [("mma", 16, 2), ("lut_one", 1, 2)]
+
+
+def test_large_mixed_batches_group_by_precision_and_share_the_rest(L):
+    """More than 16 rows: groups of one precision, then the rows left over in
+    every group share mixed launches instead of one launch each."""
+    p_row = [2] * 18 + [3] * 2 + [4] * 2
+    r = api.route_query(22, 4096, 4096, p_row=p_row)
+    assert ("mma", 16, 2) in r
+    assert ("mma_mixed", 6, 4) in r                   # 2 + 2 + 2 rows left over
+    assert sum(n for _, n, _ in r) == 22 and len(r) == 2
+
+
+def test_routing_follows_the_switches(monkeypatch, L):
+    monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "5")
+    assert api.route_query(4, 14336, 4096, p=4) == [("lut_pair", 2, 4), ("lut_pair", 2, 4)]
+    pl = api.plan_query(4, 14336, 4096, 4)    # a four-row launch is no longer lut_four
+    assert pl["stage_bytes"] == 8192 * 4
+    monkeypatch.setenv("BCQ_MMA_MIN_ROWS", "3")
+    monkeypatch.setenv("BCQ_LUT4_MAX_ROWS", "0")
+    assert api.route_query(4, 14336, 4096, p=4) == [("mma", 4, 4)]
+
+
+def test_route_query_rejects_bad_arguments(L):
+    with pytest.raises(api.BcqError):
+        api.route_query(0, 64, 256, p=2)
+    with pytest.raises(api.BcqError):
+        api.route_query(2, 64, 200, p=2)
+    with pytest.raises(api.BcqError):
+        api.route_query(2, 64, 256, p_row=[2, 5])

@@ -135,17 +135,54 @@ def test_parity_wide_batches(N, K, path):
 
 
 @pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
-def test_parity_mixed_precision_70b_sampled(N, K, path):
-    """M = 8 rows with p drawn from {2,3,4}; outputs checked on 1024 sampled
-    rows plus the first and last row-blocks."""
+def test_parity_mixed_precision_70b_every_output(N, K):
+    """M = 8 rows with p drawn from {2,3,4}: one launch that streams the
+    planes once up to the largest precision; every output checked."""
     prob = synth.make_problem(N, K, 8, seed=4, mixed=True)
-    assert set(prob.p_row.tolist()) <= {2, 3, 4}
+    assert set(prob.p_row.tolist()) <= {2, 3, 4} and len(set(prob.p_row.tolist())) > 1
+    assert api.route_query(8, N, K, p_row=prob.p_row) == [("mma_mixed", 8, int(prob.p_row.max()))]
     y = _run(prob, p_row=prob.p_row)
-    rng = np.random.default_rng(40)
-    rows = np.unique(np.concatenate([np.arange(32), np.arange(N - 32, N),
-                                     rng.choice(N, 1024, replace=False)])).astype(np.int32)
-    ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row, rows=rows)
-    _check(y[:, torch.from_numpy(rows).long().cuda()], ref, f"{N}x{K} mixed")
+    ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row)
+    _check(y, ref, f"{N}x{K} mixed")
+
+
+@pytest.mark.parametrize("N,K", [(1000, 2048), (14336, 4096), (300, 128 * 33)])
+@pytest.mark.parametrize("M", [3, 5, 8, 9, 16])
+def test_parity_mixed_batches_in_one_launch(N, K, M):
+    """Per-request precision inside one tensor-core launch (rows of 1 to 4
+    bits), including precision-1 rows and rows past a multiple of 8."""
+    prob = synth.make_problem(N, K, M, seed=30 + M + N, precisions=(1, 2, 3, 4), mixed=True)
+    rng = np.random.default_rng(M * 7 + N)
+    prob.p_row[:] = rng.integers(1, 5, size=M)
+    prob.p_row[0], prob.p_row[-1] = 1, 4   # at least two precisions, 4 the largest
+    assert api.route_query(M, N, K, p_row=prob.p_row) == [("mma_mixed", M, 4)]
+    y = _run(prob, p_row=prob.p_row)
+    _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row),
+           f"N={N} K={K} M={M}")
+
+
+def test_parity_large_mixed_batch_with_leftovers():
+    """22 rows: a group of one precision on the tensor cores, the rows left
+    over in every group sharing one mixed launch."""
+    prob = synth.make_problem(4096, 4096, 22, seed=33, mixed=True)
+    prob.p_row[:] = [2] * 18 + [3] * 2 + [4] * 2
+    rng = np.random.default_rng(34)
+    rng.shuffle(prob.p_row)
+    r = api.route_query(22, 4096, 4096, p_row=prob.p_row)
+    assert ("mma_mixed", 6, 4) in r
+    y = _run(prob, p_row=prob.p_row)
+    _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row))
+
+
+def test_four_row_launch_with_a_row_map_in_one_k_block():
+    """K = 256 (one K-block: results stored directly, no split-K) and a
+    four-row lookup launch that takes rows 1, 3, 5 of the batch."""
+    prob = synth.make_problem(300, 256, 20, seed=35, mixed=True)
+    prob.p_row[:] = [2, 4, 2, 4, 2, 4] + [2] * 14
+    r = api.route_query(20, 300, 256, p_row=prob.p_row)
+    assert ("lut_four", 3, 4) in r
+    y = _run(prob, p_row=prob.p_row)
+    _check(y, oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row))
 
 
 # ------------------------------------------------------------------ invariants

@@ -11,13 +11,22 @@ of every call, with microseconds per call reported per (p, M).
 Timing: CUDA graphs (one per step, 15 calls) replayed back to back; R
 rotating copies of the weights (> 2x L2 in total) so every call streams from
 HBM; CUDA events on the launching stream; W warm-up steps; clocks sampled
-with nvidia-smi during the timed region.  ``e2e`` measures the same calls
-through the C entry point with host buffers (bcq_gemm_host), copies included.
+with nvidia-smi during the timed work.  Per call (`per_call`, `headline_m1`,
+`shapes`): graphs of 200 calls cycling through a weight ring, median of 5
+replays, programmatic dependent launch as --pdl says (back to back);
+`isolated_m1`: one call with PDL off and L2 flushed before it.  `shapes`
+covers the other workload shapes: 4096 x 4096 (M = 1), the MLP decode pair
+with 0.1 % outlier channels (M = 1), and the 70B-like pair with 8 rows of
+per-request precision.  ``e2e`` measures the step's calls through the C
+entry point with host buffers (bcq_gemm_host), copies included.  The
+`roofline` object is that of the step's dominant kernel (most time per
+step), the step aggregate beside it.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
 same workload on the host cores.  With torchrun (N > 1 GPUs) every rank runs
-an independent replica (no collective on the data path), the timed region is
-bracketed by barriers and the time is the max over ranks.
+an independent replica (no collective on the data path; --mode shard: one
+layer split by output rows, an NCCL all-gather of y per call), the timed
+region is bracketed by barriers and the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -48,7 +57,11 @@ def algo_bytes(N, K, M, p):
 
 
 KERNEL_SOURCES = ("bcq_kernels.cu", "bcq_device.cuh", "bcq_pipeline.cuh", "bcq_mma.cuh",
-                  "bcq_layout.h")
+                  "bcq_m1.cuh", "bcq_umma.cuh", "bcq_layout.h")
+# CUDA kernel of each launch kind bcq_route_query reports
+KERNEL_OF_ROUTE = {"lut_one": "gemv_m1_kernel", "lut_pair": "gemv_lut_kernel<2>",
+                   "lut_four": "gemv_lut_kernel<4>", "mma": "gemv_mma_kernel",
+                   "mma_mixed": "gemv_mma_kernel<mixed>", "tcgen05": "gemv_umma_kernel"}
 
 
 def csrc_sha256():
@@ -193,6 +206,31 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
+CALLS_PER_GRAPH = 200   # calls captured per timing graph
+REPLAYS = 5             # timed replays; the median is reported
+
+
+def weight_bytes(w):
+    return w.packed.numel() * 4 + sum(a.numel() * 2 for a in w.alphas.values()) + \
+        (w.z.numel() * 2 if w.z is not None else 0) + \
+        (sum(v.numel() * 2 for v in w.zq.values()) if w.zq else 0)
+
+
+def weight_ring(api, base):
+    """base and copies of it, more than 2x L2 in all, so that every call
+    streams its weights from HBM."""
+    per = weight_bytes(base)
+    R = max(2, math.ceil(2 * L2_BYTES / per) + 1)
+    ring = [base]
+    for _ in range(R - 1):
+        ring.append(api.BcqWeights(
+            packed=base.packed.clone(), alphas={q: a.clone() for q, a in base.alphas.items()},
+            z=None if base.z is None else base.z.clone(), N=base.N, K=base.K, p_H=base.p_H,
+            row_splits=base.row_splits,
+            zq=None if base.zq is None else {q: v.clone() for q, v in base.zq.items()}))
+    return ring, per
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from bit_gemv_bcq_b200 import api, synth
@@ -201,13 +239,8 @@ def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
     base = api.BcqWeights.from_canonical(prob.planes, prob.alphas, prob.z, device=dev)
-    per_copy = base.packed.numel() * 4 + sum(a.numel() * 2 for a in base.alphas.values()) \
-        + base.z.numel() * 2
-    R = max(2, math.ceil(2 * L2_BYTES / per_copy) + 1)
-    copies = [base] + [api.BcqWeights(packed=base.packed.clone(),
-                                      alphas={q: a.clone() for q, a in base.alphas.items()},
-                                      z=base.z.clone(), N=base.N, K=base.K, p_H=base.p_H)
-                       for _ in range(R - 1)]
+    copies, per_copy = weight_ring(api, base)
+    R = len(copies)
     x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).to(dev)
     ys = {M: torch.empty((M, N_OUT), dtype=torch.float16, device=dev) for M in BATCHES}
     cases = [(p, M) for p in PRECISIONS for M in BATCHES]
@@ -216,14 +249,14 @@ def run_gpu(args, rank, world, local_rank):
         cases = [(p, M) for p, M in cases if (M, p) in want]
     bytes_step = sum(algo_bytes(N_OUT, K_IN, M, p) for p, M in cases)
     api.set_pdl(args.pdl)
-    launches_per_step = sum(launches_per_call(M) for p, M in cases)
+    routes = {(p, M): api.route_query(M, N_OUT, K_IN, p=p) for p, M in cases}
+    launches_per_step = sum(len(r) for r in routes.values())
 
     stream = torch.cuda.Stream(device=dev)
     # eager pass: plans and caches every launch shape before capture
     with torch.cuda.stream(stream):
-        for w in copies[:1]:
-            for p, M in cases:
-                w.gemm(x[:M], p=p, out=ys[M], stream=stream)
+        for p, M in cases:
+            base.gemm(x[:M], p=p, out=ys[M], stream=stream)
     stream.synchronize()
     assert api.device_error(stream) == api.BCQ_OK
 
@@ -233,20 +266,29 @@ def run_gpu(args, rank, world, local_rank):
             fn()
         return g
 
+    def us_per_call(fn_calls, ncalls):
+        """Median over REPLAYS of one replay of a graph of ncalls calls."""
+        g = capture(fn_calls)
+        times = []
+        with torch.cuda.stream(stream):
+            g.replay()
+            for _ in range(REPLAYS):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                times.append((a, b))
+        stream.synchronize()
+        del g
+        return statistics.median(a.elapsed_time(b) for a, b in times) * 1000.0 / ncalls
+
     step_graphs = []
     for r in range(R):
         def step(r=r):
             for i, (p, M) in enumerate(cases):
                 copies[(r + i) % R].gemm(x[:M], p=p, out=ys[M], stream=stream)
         step_graphs.append(capture(step))
-
-    # per-call timing of each case: R calls (one per copy) per replay
-    case_graphs = {}
-    for p, M in cases:
-        def one(p=p, M=M):
-            for w in copies:
-                w.gemm(x[:M], p=p, out=ys[M], stream=stream)
-        case_graphs[(p, M)] = capture(one)
 
     def barrier():
         rank_barrier(world)
@@ -256,6 +298,8 @@ def run_gpu(args, rank, world, local_rank):
             step_graphs[k % R].replay()
     stream.synchronize()
 
+    # clocks are sampled over all the timed work below (the step, then the
+    # per-call timings)
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.2)
@@ -272,31 +316,102 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     barrier()
     ms_total = t0.elapsed_time(t1)
-    clocks = sampler.stop()
+    del step_graphs
     err = api.device_error(stream)
     if err != api.BCQ_OK:
         raise RuntimeError(f"device error {api.status_string(err)}")
-
     ms_total = max_over_ranks(ms_total, world, dev)
 
-    # per-case microseconds (same stream, events around each replay)
+    # per-call microseconds of each case, back to back: a graph of 200 calls
+    # cycling through the weight ring, median of 5 replays
     per_case = []
-    reps = max(3, min(50, args.steps // 20))
     for p, M in cases:
-        g = case_graphs[(p, M)]
-        with torch.cuda.stream(stream):
-            g.replay()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                g.replay()
-            b.record(stream)
-        b.synchronize()
-        us = a.elapsed_time(b) * 1000.0 / (reps * R)
+        def calls(p=p, M=M):
+            for i in range(CALLS_PER_GRAPH):
+                copies[i % R].gemm(x[:M], p=p, out=ys[M], stream=stream)
+        us = us_per_call(calls, CALLS_PER_GRAPH)
         by = algo_bytes(N_OUT, K_IN, M, p)
         per_case.append({"p": p, "M": M, "us": round(us, 3), "bytes": by,
-                         "GBps": round(by / us / 1e3, 1)})
+                         "GBps": round(by / us / 1e3, 1),
+                         "kernels": [k for k, _, _ in routes[(p, M)]]})
+
+    # one call alone: programmatic dependent launch off, L2 flushed (a write
+    # of 2x L2) before it, CUDA events around that call only
+    isolated = None
+    if not args.cases:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+        api.set_pdl(0)
+        isolated = {"method": "PDL off, L2 flushed before each call, median of 20 calls"}
+        for p in PRECISIONS:
+            g = capture(lambda p=p: copies[0].gemm(x[:1], p=p, out=ys[1], stream=stream))
+            times = []
+            with torch.cuda.stream(stream):
+                for _ in range(21):
+                    flush.fill_(1)
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    g.replay()
+                    b.record(stream)
+                    times.append((a, b))
+            stream.synchronize()
+            us = statistics.median(a.elapsed_time(b) for a, b in times[1:]) * 1000.0
+            by = algo_bytes(N_OUT, K_IN, 1, p)
+            isolated[f"M1p{p}"] = {"us": round(us, 3), "GBps": round(by / us / 1e3, 1)}
+            del g
+        del flush
+        api.set_pdl(args.pdl)
+    clocks = sampler.stop()
+
+    # the other workload shapes, same back-to-back method (each on its own
+    # weight ring): the attention projection, the MLP down projection (and
+    # gate/up) with 0.1 % outlier channels, and the 70B-like shapes with 8 rows
+    # of per-request precision
+    shapes = None
+    if not args.cases:
+        shapes = {}
+        specs = [("attn_4096x4096_M1", 4096, 4096, 1, False, False),
+                 ("mlp_gate_up_14336x4096_M1_outliers", 14336, 4096, 1, True, False),
+                 ("mlp_down_4096x14336_M1_outliers", 4096, 14336, 1, True, False),
+                 ("70b_28672x8192_M8_mixed", 28672, 8192, 8, False, True),
+                 ("70b_8192x28672_M8_mixed", 8192, 28672, 8, False, True)]
+        for label, N, K, M, outl, mixed in specs:
+            pr = synth.make_problem(N, K, M, seed=args.seed + 4, outliers=outl, mixed=mixed)
+            wb = api.BcqWeights.from_canonical(pr.planes, pr.alphas, pr.z, device=dev)
+            ring, per = weight_ring(api, wb)
+            xs = torch.from_numpy(pr.x.view(np.int16)).view(torch.float16).to(dev)
+            yy = torch.empty((M, N), dtype=torch.float16, device=dev)
+            entry = {"N": N, "K": K, "M": M, "ring": f"{len(ring)} copies of {per / 2**20:.1f} MiB"}
+            for p in ([None] if mixed else PRECISIONS):
+                kw = {"p_row": pr.p_row} if mixed else {"p": p}
+                with torch.cuda.stream(stream):
+                    wb.gemm(xs, out=yy, stream=stream, **kw)
+                stream.synchronize()
+
+                def calls(kw=kw):
+                    for i in range(CALLS_PER_GRAPH):
+                        ring[i % len(ring)].gemm(xs, out=yy, stream=stream, **kw)
+                us = us_per_call(calls, CALLS_PER_GRAPH)
+                G = K // GROUP
+                if mixed:
+                    qs = sorted(set(pr.p_row.tolist()))
+                    by = N * K * max(qs) // 8 + sum(N * G * q * 2 for q in qs) + N * G * 2 \
+                        + M * K * 2 + M * N * 2
+                    key = "mixed"
+                    entry["p_row"] = [int(v) for v in pr.p_row]
+                else:
+                    by = algo_bytes(N, K, M, p)
+                    key = f"p{p}"
+                route = api.route_query(M, N, K, **kw)
+                entry[key] = {"us": round(us, 3), "bytes": by, "GBps": round(by / us / 1e3, 1),
+                              "launches": [f"{k}:{n}rows:{pl}planes" for k, n, pl in route]}
+            shapes[label] = entry
+            del ring, wb, xs, yy
+            torch.cuda.synchronize(dev)
+        shapes["attn_4096x4096_M1"]["context"] = (
+            "ABQ-LLM page (GEMV ablation): 6.68 us for a (1,4096)x(4096,4096) W2A8 GEMV "
+            "on RTX 3070/4080 -- other hardware, activations quantised to 8 bits; context only")
+        assert api.device_error(stream) == api.BCQ_OK
 
     # an MLP's gate and up projections (same x) stacked into one weight: one
     # call for both (M = 1, 2), against two calls on the separate weights
@@ -305,14 +420,7 @@ def run_gpu(args, rank, world, local_rank):
         prob_b = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed + 1)
         sbase = api.BcqWeights.stack([(prob.planes, prob.alphas, prob.z),
                                       (prob_b.planes, prob_b.alphas, prob_b.z)], device=dev)
-        s_copy = sbase.packed.numel() * 4 + sum(a.numel() * 2 for a in sbase.alphas.values()) \
-            + sbase.z.numel() * 2
-        RS = max(2, math.ceil(2 * L2_BYTES / s_copy) + 1)
-        scopies = [sbase] + [api.BcqWeights(packed=sbase.packed.clone(),
-                                            alphas={q: a.clone() for q, a in sbase.alphas.items()},
-                                            z=sbase.z.clone(), N=sbase.N, K=sbase.K, p_H=sbase.p_H,
-                                            row_splits=sbase.row_splits)
-                             for _ in range(RS - 1)]
+        scopies, s_copy = weight_ring(api, sbase)
         ys2 = {M: torch.empty((M, sbase.N), dtype=torch.float16, device=dev) for M in (1, 2)}
         with torch.cuda.stream(stream):
             for M in (1, 2):
@@ -320,35 +428,24 @@ def run_gpu(args, rank, world, local_rank):
                     sbase.gemm(x[:M], p=p, out=ys2[M], stream=stream)
         stream.synchronize()
         stacked = {"weights": f"2 x {N_OUT} rows (gate and up) x {K_IN}, stacked along N",
-                   "l2": f"{RS} rotating copies of {s_copy / 2**20:.1f} MiB"}
+                   "l2": f"{len(scopies)} rotating copies of {s_copy / 2**20:.1f} MiB"}
         single = {(c["p"], c["M"]): c["us"] for c in per_case}
         for M in (1, 2):
             for p in PRECISIONS:
                 def sone(p=p, M=M):
-                    for w in scopies:
-                        w.gemm(x[:M], p=p, out=ys2[M], stream=stream)
-                g = capture(sone)
-                with torch.cuda.stream(stream):
-                    g.replay()
-                    a = torch.cuda.Event(enable_timing=True)
-                    b = torch.cuda.Event(enable_timing=True)
-                    a.record(stream)
-                    for _ in range(reps):
-                        g.replay()
-                    b.record(stream)
-                b.synchronize()
-                us = a.elapsed_time(b) * 1000.0 / (reps * RS)
+                    for i in range(CALLS_PER_GRAPH):
+                        scopies[i % len(scopies)].gemm(x[:M], p=p, out=ys2[M], stream=stream)
+                us = us_per_call(sone, CALLS_PER_GRAPH)
                 by = algo_bytes(2 * N_OUT, K_IN, M, p)
                 two = 2 * single[(p, M)] if (p, M) in single else None
                 stacked[f"M{M}p{p}"] = {"us": round(us, 3), "GBps": round(by / us / 1e3, 1),
                                         "us_two_calls": None if two is None else round(two, 3)}
-                del g
         del scopies, sbase
         assert api.device_error(stream) == api.BCQ_OK
 
     # offsets per precision (bcq_gemm_zp): M = 1 at each precision and one
-    # two-row launch with two precisions (row 1's offsets read apart), against
-    # the same calls with shared offsets
+    # two-row launch with two precisions, against the same calls with shared
+    # offsets
     zp = None
     if not args.cases:
         rng = np.random.default_rng(args.seed + 3)
@@ -361,33 +458,23 @@ def run_gpu(args, rank, world, local_rank):
         single = {(c["p"], c["M"]): c["us"] for c in per_case}
         for label, M, pr in [("M1p2", 1, [2]), ("M1p3", 1, [3]), ("M1p4", 1, [4]),
                              ("M2p2p4", 2, [2, 4])]:
-            def zone(M=M, pr=pr):
-                for w in zcopies:
-                    w.gemm(x[:M], p_row=pr, out=ys[M], stream=stream)
             with torch.cuda.stream(stream):
-                zone()
+                zbase.gemm(x[:M], p_row=pr, out=ys[M], stream=stream)
             stream.synchronize()
-            g = capture(zone)
-            with torch.cuda.stream(stream):
-                g.replay()
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                for _ in range(reps):
-                    g.replay()
-                b.record(stream)
-            b.synchronize()
-            us = a.elapsed_time(b) * 1000.0 / (reps * R)
+
+            def zone(M=M, pr=pr):
+                for i in range(CALLS_PER_GRAPH):
+                    zcopies[i % len(zcopies)].gemm(x[:M], p_row=pr, out=ys[M], stream=stream)
+            us = us_per_call(zone, CALLS_PER_GRAPH)
             shared = single.get((pr[0], M)) if len(set(pr)) == 1 else None
             zp[label] = {"us": round(us, 3), "us_shared_offsets": shared}
-            del g
         del zcopies, zbase
         assert api.device_error(stream) == api.BCQ_OK
 
     result = {"ms_total": ms_total, "bytes_step": bytes_step, "R": R,
               "per_copy_bytes": per_copy, "launches_per_step": launches_per_step,
               "per_case": per_case, "clocks": clocks, "stacked": stacked,
-              "per_precision_offsets": zp}
+              "per_precision_offsets": zp, "shapes": shapes, "isolated": isolated}
 
     # end to end through bcq_gemm_host: pinned host x and y, copies inside
     # the timed region.  Calls alternate between two streams, each with its
@@ -428,8 +515,99 @@ def run_gpu(args, rank, world, local_rank):
         b.synchronize()
         e2e_ms = a.elapsed_time(b)
         e2e_ms = max_over_ranks(e2e_ms, world, dev)
+        assert api.device_error(streams[0]) == api.BCQ_OK and api.device_error(streams[1]) == api.BCQ_OK
+        # (outside the timed region) the host path gives the device path's bits
+        for p, M in cases:
+            api.gemm_host(x_host[:M], copies[0], y_host[0][M], x_dev[0][:M], y_dev[0][M], p=p,
+                          stream=streams[0])
+            copies[0].gemm(x[:M], p=p, out=ys[M], stream=streams[0])
+            streams[0].synchronize()
+            if not torch.equal(y_host[0][M], ys[M].cpu()):
+                raise RuntimeError(f"e2e output differs from the device path (p={p}, M={M})")
         result["e2e"] = {"ms": e2e_ms, "steps": e2e_steps, "h2d": h2d, "d2h": d2h}
     return result
+
+
+def run_sharded(args, rank, world, local_rank):
+    """One 14336 x 4096 layer split by output rows over the ranks: each rank
+    packs its rows, runs the step's 15 calls on them and all-gathers y after
+    every call (NCCL; the only collective).  Steps are CUDA graphs over a ring
+    of copies of the rank's rows; the time is the max over ranks; `value` is
+    the whole layer's algorithmic bytes per step over that time (strong
+    scaling: the total work is fixed)."""
+    import torch
+    from bit_gemv_bcq_b200 import api, shard, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
+    sw = shard.ShardedBcqWeights.from_canonical(prob.planes, prob.alphas, prob.z, world, rank,
+                                                device=dev)
+    ring, per = weight_ring(api, sw.local)
+    copies = [shard.ShardedBcqWeights(w, N_OUT, sw.r0, sw.r1, world, rank) for w in ring]
+    x = torch.from_numpy(prob.x.view(np.int16)).view(torch.float16).to(dev)
+    cases = [(p, M) for p in PRECISIONS for M in BATCHES]
+    bytes_step = sum(algo_bytes(N_OUT, K_IN, M, p) for p, M in cases)
+    api.set_pdl(args.pdl)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for p, M in cases:
+            copies[0].gemm(x[:M], p=p, stream=stream)
+    stream.synchronize()
+    graphs = []
+    for r in range(len(copies)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i, (p, M) in enumerate(cases):
+                copies[(r + i) % len(copies)].gemm(x[:M], p=p, stream=stream)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            graphs[k % len(graphs)].replay()
+    stream.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    rank_barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for k in range(args.steps):
+            graphs[k % len(graphs)].replay()
+        t1.record(stream)
+    t1.synchronize()
+    torch.cuda.synchronize(dev)
+    rank_barrier(world)
+    clocks = sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    del graphs
+    assert api.device_error(stream) == api.BCQ_OK
+    peak, peak_kind = measured_peaks()
+    ms_step = ms / args.steps
+    value = bytes_step / (ms_step * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "bcq_gemv N=14336 K=4096 g=128 p_H=4, split by output rows "
+                                   f"over {world} ranks; one step = one call per p in {{2,3,4}} x "
+                                   "M in {1,2,4,8,16} + an all-gather of y after each",
+                       "l2": f"{len(ring)} rotating copies of this rank's {per / 2**20:.1f} MiB",
+                       "parallelism": f"column-parallel x{world} (NCCL all-gather)"},
+            "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(value / world / peak, 4),
+                         "peak_kind": peak_kind, "traffic": None,
+                         "kernel": "per GPU: the rank's rows of every call of the step"},
+            "gpu_launches": sum(len(api.route_query(M, sw.r1 - sw.r0, K_IN, p=p))
+                                for p, M in cases) * args.steps,
+            "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
 
 
 def run_quantizer(args, dev, rows=N_OUT):
@@ -530,25 +708,6 @@ def run_quantizer_oracle(seed, n_groups=1024):
             "sample": f"{n_groups} random groups of the same weight ({dt:.1f} s)"}
 
 
-MMA_MIN_ROWS = 3   # bcq_gemm's default switch to the tensor-core kernel
-
-
-def launches_per_call(M):
-    """GEMV kernel launches of one single-precision bcq_gemm call: the lookup
-    kernel takes two activation rows per launch, the tensor-core kernel up to
-    sixteen."""
-    return -(-M // 16) if M >= MMA_MIN_ROWS else -(-M // 2)
-
-
-LUT4_MIN_BITS = 1  # bcq_gemm's four-row lookup launches: 3-4 rows of any precision
-
-
-def kernel_of(M, p):
-    if M < MMA_MIN_ROWS or (M <= 4 and p >= LUT4_MIN_BITS):
-        return "gemv_lut_kernel"
-    return "gemv_mma_kernel"
-
-
 # ------------------------------------------------------------- CPU oracle arm
 
 def run_oracle_sample(seed, rows_per_call, prob=None):
@@ -589,6 +748,10 @@ def main():
     ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
                     help="bcq_set_pdl mode for the GEMV launches (2: weights may stream "
                          "while the previous kernel drains; no kernel of the step writes them)")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "shard"],
+                    help="N > 1 GPUs: independent replicas of the workload (weak scaling), "
+                         "or one layer split by output rows over the ranks with an NCCL "
+                         "all-gather of y per call (strong scaling)")
     ap.add_argument("--profile", action="store_true",
                     help="GPU timing only (no e2e or CPU legs), for profiler runs")
     ap.add_argument("--quantizer-only", type=int, default=0, metavar="ROWS",
@@ -643,6 +806,8 @@ def main():
         if rank == 0:
             print(json.dumps({"quantizer": q}), flush=True)
         return 0
+    if args.mode == "shard":
+        return run_sharded(args, rank, world, local_rank)
     res = run_gpu(args, rank, world, local_rank)
     quant = run_quantizer(args, torch.device("cuda", local_rank)) if not args.cases else None
 
@@ -660,33 +825,53 @@ def main():
                    "l2": f"inputs larger than L2: {res['R']} rotating weight copies of "
                          f"{res['per_copy_bytes'] / 2**20:.1f} MiB",
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "timing": "CUDA graph per step, CUDA events on the launching stream",
+                   "timing": "CUDA graph per step, CUDA events on the launching stream; "
+                             "per call: graphs of 200 calls over the weight ring, median of 5 "
+                             "replays",
                    "pdl": args.pdl},
-        "roofline": {"bound": "hbm", "achieved": round(achieved_per_gpu, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved_per_gpu / peak, 4),
-                     "peak_kind": peak_kind, "traffic": None,
-                     "kernel": "every launch of the step (gemv_lut_kernel for M <= 4, "
-                               "gemv_mma_kernel for M = 8 and 16)"},
         "per_call": res["per_case"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
     }
-    tr = recorded_traffic()
-    if tr is not None:
-        line["roofline"]["traffic"] = round(tr["dram_bytes_per_launch"])
-        line["roofline"]["traffic_per"] = "launch (mean over one step's launches, ncu launch list)"
-        line["roofline"]["algorithmic_bytes_per_launch"] = round(tr["algorithmic_bytes_per_launch"])
-        line["roofline"]["traffic_source"] = tr["source"]
+    # the roofline of the dominant kernel of the step (the most time per
+    # step): algorithmic bytes of its calls / their measured time; the step
+    # aggregate beside it
     by_kernel = {}
     for c in res["per_case"]:
-        k = by_kernel.setdefault(kernel_of(c["M"], c["p"]), {"us": 0.0, "bytes": 0})
+        name = "+".join(KERNEL_OF_ROUTE[k] for k in c["kernels"])
+        k = by_kernel.setdefault(name, {"us": 0.0, "bytes": 0, "launches": 0})
         k["us"] += c["us"]
         k["bytes"] += c["bytes"]
+        k["launches"] += len(c["kernels"])
     for name, k in by_kernel.items():
         gbps = k["bytes"] / k["us"] / 1e3
         by_kernel[name] = {"us_per_step": round(k["us"], 2), "GBps": round(gbps, 1),
-                           "frac": round(gbps / peak, 4)}
-    line["roofline"]["by_kernel"] = by_kernel
+                           "frac": round(gbps / peak, 4),
+                           "algorithmic_bytes_per_launch": round(k["bytes"] / k["launches"])}
+    dom = max(by_kernel, key=lambda n: by_kernel[n]["us_per_step"])
+    line["roofline"] = {"bound": "hbm", "achieved": by_kernel[dom]["GBps"], "peak": peak,
+                        "unit": "GB/s", "frac": by_kernel[dom]["frac"], "peak_kind": peak_kind,
+                        "traffic": None, "kernel": dom,
+                        "step_aggregate": {"achieved": round(achieved_per_gpu, 1),
+                                           "frac": round(achieved_per_gpu / peak, 4)},
+                        "by_kernel": by_kernel}
+    tr = recorded_traffic()
+    if tr is not None and dom in tr.get("kernels", {}):
+        t = tr["kernels"][dom]
+        line["roofline"]["traffic"] = round(t["dram_bytes_per_launch"])
+        line["roofline"]["traffic_per"] = "launch (mean over the step's launches of it, ncu)"
+        line["roofline"]["traffic_source"] = tr["source"]
+    if res.get("shapes"):
+        for label, e in res["shapes"].items():
+            for key, v in e.items():
+                if isinstance(v, dict) and "GBps" in v:
+                    v["frac"] = round(v["GBps"] / peak, 4)
+        line["shapes"] = res["shapes"]
+    if res.get("isolated"):
+        for key, v in res["isolated"].items():
+            if isinstance(v, dict):
+                v["frac"] = round(v["GBps"] / peak, 4)
+        line["isolated_m1"] = res["isolated"]
     if res.get("stacked"):
         line["stacked_gate_up"] = res["stacked"]
     if res.get("per_precision_offsets"):

@@ -327,9 +327,9 @@ def run_gpu(args, rank, world, local_rank):
     per_case = []
     for p, M in cases:
         def calls(p=p, M=M):
-            for i in range(CALLS_PER_GRAPH):
+            for i in range(args.calls):
                 copies[i % R].gemm(x[:M], p=p, out=ys[M], stream=stream)
-        us = us_per_call(calls, CALLS_PER_GRAPH)
+        us = us_per_call(calls, args.calls)
         by = algo_bytes(N_OUT, K_IN, M, p)
         per_case.append({"p": p, "M": M, "us": round(us, 3), "bytes": by,
                          "GBps": round(by / us / 1e3, 1),
@@ -389,9 +389,9 @@ def run_gpu(args, rank, world, local_rank):
                 stream.synchronize()
 
                 def calls(kw=kw):
-                    for i in range(CALLS_PER_GRAPH):
+                    for i in range(args.calls):
                         ring[i % len(ring)].gemm(xs, out=yy, stream=stream, **kw)
-                us = us_per_call(calls, CALLS_PER_GRAPH)
+                us = us_per_call(calls, args.calls)
                 G = K // GROUP
                 if mixed:
                     qs = sorted(set(pr.p_row.tolist()))
@@ -433,9 +433,9 @@ def run_gpu(args, rank, world, local_rank):
         for M in (1, 2):
             for p in PRECISIONS:
                 def sone(p=p, M=M):
-                    for i in range(CALLS_PER_GRAPH):
+                    for i in range(args.calls):
                         scopies[i % len(scopies)].gemm(x[:M], p=p, out=ys2[M], stream=stream)
-                us = us_per_call(sone, CALLS_PER_GRAPH)
+                us = us_per_call(sone, args.calls)
                 by = algo_bytes(2 * N_OUT, K_IN, M, p)
                 two = 2 * single[(p, M)] if (p, M) in single else None
                 stacked[f"M{M}p{p}"] = {"us": round(us, 3), "GBps": round(by / us / 1e3, 1),
@@ -463,9 +463,9 @@ def run_gpu(args, rank, world, local_rank):
             stream.synchronize()
 
             def zone(M=M, pr=pr):
-                for i in range(CALLS_PER_GRAPH):
+                for i in range(args.calls):
                     zcopies[i % len(zcopies)].gemm(x[:M], p_row=pr, out=ys[M], stream=stream)
-            us = us_per_call(zone, CALLS_PER_GRAPH)
+            us = us_per_call(zone, args.calls)
             shared = single.get((pr[0], M)) if len(set(pr)) == 1 else None
             zp[label] = {"us": round(us, 3), "us_shared_offsets": shared}
         del zcopies, zbase
@@ -748,6 +748,8 @@ def main():
     ap.add_argument("--pdl", type=int, default=2, choices=[0, 1, 2],
                     help="bcq_set_pdl mode for the GEMV launches (2: weights may stream "
                          "while the previous kernel drains; no kernel of the step writes them)")
+    ap.add_argument("--calls", type=int, default=CALLS_PER_GRAPH,
+                    help="calls per per-call timing graph (fewer for profiler runs)")
     ap.add_argument("--mode", default="replicas", choices=["replicas", "shard"],
                     help="N > 1 GPUs: independent replicas of the workload (weak scaling), "
                          "or one layer split by output rows over the ranks with an NCCL "

@@ -142,13 +142,34 @@ __device__ __forceinline__ void load_x_tile(const GemvParams& prm, int kb, int w
   }
 }
 
+// Position of column c (0..255) of a K-block in the tile's K order: inside
+// each 32-column word U of group h, the natural word of a weight row holds
+// column c at stored bit b (bytes rotated: b = 8 (c / 8) + (c + 7) mod 8),
+// and fragment register s = 8 t + i (k-step 2 U + t, k-pair i) holds bits
+// 15 - s (its low half, k = 2i) and 31 - s (high half, k = 2i + 1).
+__host__ __device__ __forceinline__ int mma_k_position(int c) {
+  const int h = c >> 7, U = (c >> 5) & 3, cw = c & 31;
+  const int b = (cw & ~7) | ((cw + 7) & 7);
+  const int e = b >> 4;
+  const int s = (e ? 31 : 15) - b;
+  return h * 128 + (2 * U + (s >> 3)) * 16 + 2 * (s & 7) + e;
+}
+
+// Launch row `warp` of K-block kb's activation tile into slot kb & 1: lane l
+// holds columns 8l .. 8l + 7 (v), stored at their positions in the tile's K
+// order (mma_k_position); also the row's group sums.
 __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, int lane,
                                              const uint4& v) {
   const uint32_t slot = (uint32_t)(kb & 1);
-  const uint32_t t = sbase + slot * kXTileBytes + (uint32_t)(warp * kXPitch + lane * 8) * 2u;
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(t), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
+  const uint32_t t = sbase + slot * kXTileBytes + (uint32_t)(warp * kXPitch) * 2u;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e8 = 0; e8 < 8; ++e8) {
+    const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(t + (uint32_t)mma_k_position(lane * 8 + e8) * 2u),
+                 "h"((unsigned short)half)
+                 : "memory");
+  }
   float f[8];
   unpack8(v, f);
   float s = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
@@ -156,6 +177,14 @@ __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, i
   for (int o = 1; o < 16; o <<= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
   if ((lane & 15) == 0)  // lane 0: group A, lane 16: group B
     sts_f32(sbase + kMmaGsumOff + ((slot * kMmaRows + warp) * 2 + (lane >> 4)) * 4u, s);
+}
+
+// x * y, asked for as an integer multiply (the FMA pipe) rather than a
+// shift (the ALU pipe, which the fragment lop3s keep busy).
+__device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t y) {
+  uint32_t d;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(y));
+  return d;
 }
 
 // One plane of one row-block for this warp: both 16-row tiles, both groups,
@@ -167,11 +196,11 @@ __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, i
 // byte (4v - rho) mod 16, rho = r mod 16: it is the funnel shift of rotated
 // words (v - R) mod 4 and (v - R + 1) mod 4 by 8 delta bits, with
 // R = ceil(rho / 4) mod 4 and delta = (-rho) mod 4 -- per-thread constants.
-// A fragment element pair (columns 2q, 2q + 1 of an 8-column chunk; stored
-// bits (2q + 7) mod 8 and 2q, the bytes being rotated) becomes +-alpha by
-// moving the two bits to bit 7 of their byte (shifts by (8 - 2q) mod 8 and
-// 7 - 2q), replicating each into a sign byte (prmt) and xoring the fp16 sign
-// bits of alpha2 (lop3).
+// In the tile's K order (mma_k_position) fragment register s = 8 t + i of
+// a row and 32-column word holds the word's bits 15 - s and 31 - s: it is
+// (word << s) with every bit but 15 and 31 masked, turned into +-alpha by
+// xoring the fp16 sign bits of alpha2 (one lop3).  Thread q needs s = q,
+// q + 4 (k-step 2U: k-pairs q, q + 4) and 8 + q, 12 + q (k-step 2U + 1).
 // MIXED: the rows of the launch have precisions of their own (qm[nt][c]:
 // activation row nt * 8 + 2q + c, 0 past the launch's rows).  The fragments
 // then hold +-1 (exact), each (plane, group) product is accumulated apart
@@ -183,7 +212,8 @@ __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sb
                                           int g, int q, uint32_t ra0, uint32_t ra1, uint32_t dsh,
                                           float (&acc)[2][2][NT][4],
                                           const int (&qm)[NT][2]) {
-  const uint32_t sh1 = (8u - 2u * (uint32_t)q) & 7u, sh2 = 7u - 2u * (uint32_t)q;
+  // multipliers for the shifts by q, q + 4, 8 + q, 12 + q
+  const uint32_t mq0 = 1u << q, mq4 = 1u << (q + 4), mq8 = 1u << (q + 8), mq12 = 1u << (q + 12);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     // activation fragments of the group's 8 k-steps, off the critical path
@@ -227,23 +257,15 @@ __device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sb
 #pragma unroll
         for (int e = 0; e < 4; ++e) tmp[f][nt][e] = 0.f;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint32_t x1[4], x2[4];
+    for (int v = 0; v < 4; ++v) {  // word U = v of group h: k-steps 2v, 2v + 1
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        x1[j] = nw[j][v] << sh1;
-        x2[j] = nw[j][v] << sh2;
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {  // k-step s8 = 2v + e: bytes 2e (cols 0-7), 2e + 1 (8-15)
-        const int s8 = 2 * v + e;
-        const uint32_t sel0 = (uint32_t)(((8 + 2 * e) << 4) | ((12 + 2 * e) << 12));
-        const uint32_t sel1 = (uint32_t)(((9 + 2 * e) << 4) | ((13 + 2 * e) << 12));
-        uint32_t a[4][2];
+      for (int t = 0; t < 2; ++t) {
+        const int s8 = 2 * v + t;
+        uint32_t a[4][2];  // row j: k-pairs q (register 8t + q) and q + 4
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          a[j][0] = xor_andnot(al[j], prmt(x1[j], x2[j], sel0), 0x80008000u);  // cols 2q, 2q+1
-          a[j][1] = xor_andnot(al[j], prmt(x1[j], x2[j], sel1), 0x80008000u);  // cols 2q+8, 2q+9
+          a[j][0] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq8 : mq0), 0x80008000u);
+          a[j][1] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq12 : mq4), 0x80008000u);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {

@@ -136,14 +136,13 @@ struct CtaWork {
 constexpr int kMaxCtas = 256;
 
 // The tensor-core GEMV (bcq_mma.cuh): activations of the current K-block
-// (two slots, 16 rows of 256 columns padded to 264 halves so fragment loads
-// hit distinct banks) and their group sums, then per-warp double buffers of
-// scales and offsets, then the ring.
+// (two slots of 16 rows x 256 columns, stored in the order of the MMA's B
+// fragments: xtile_offset) and their group sums, then per-warp double
+// buffers of scales and offsets, then the ring.
 constexpr int kMmaRows = 16;                 // activation rows per tensor-core launch (max)
-constexpr int kXPitch = 264;                 // halves per row of the activation tile
-constexpr uint32_t kXTileBytes = kMmaRows * kXPitch * 2;            // 8448
-constexpr uint32_t kMmaGsumOff = 2 * kXTileBytes;                    // 16896
-constexpr uint32_t kMmaScaleOff = kMmaGsumOff + 2 * kMmaRows * 2 * 4; // 17152
+constexpr uint32_t kXTileBytes = kMmaRows * kKBlock * 2;             // 8192
+constexpr uint32_t kMmaGsumOff = 2 * kXTileBytes;                    // 16384
+constexpr uint32_t kMmaScaleOff = kMmaGsumOff + 2 * kMmaRows * 2 * 4; // 16640
 // Scales staged per warp and unit: 32 lanes x 2P halves of alpha^(P), then
 // the offsets (2 halves a lane).  Mixed launches (rows of several
 // precisions) stage alpha^(q) of every precision q = 1..4 present, each in

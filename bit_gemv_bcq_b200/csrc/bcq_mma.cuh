@@ -142,6 +142,13 @@ __device__ __forceinline__ void load_x_tile(const GemvParams& prm, int kb, int w
   }
 }
 
+// The same row's columns of K-block kb, prefetched into L2 only.
+__device__ __forceinline__ void prefetch_x_tile(const GemvParams& prm, int kb, int warp, int lane) {
+  const int k = kb * kKBlock + lane * 8;
+  if (warp < prm.M && k < prm.K)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(prm.x + (size_t)prm.rows[warp] * prm.K + k));
+}
+
 // Position of column c (0..255) of a K-block in the tile's K order: inside
 // each 32-column word U of group h, the natural word of a weight row holds
 // column c at stored bit b (bytes rotated: b = 8 (c / 8) + (c + 7) mod 8),
@@ -155,18 +162,33 @@ __host__ __device__ __forceinline__ int mma_k_position(int c) {
   return h * 128 + (2 * U + (s >> 3)) * 16 + 2 * (s & 7) + e;
 }
 
+
+// Byte offset of tile K position kpos (mma_k_position) of launch row n in the
+// fragment-ordered activation tile.  For group h, natural word v of the group
+// (its k-steps 2v and 2v + 1), n-tile n / 8 and lane 4 (n % 8) + q, 16 bytes
+// hold that thread's B fragments of k-step 2v and then of k-step 2v + 1 (b0:
+// k-pair q of the k-step, b1: k-pair q + 4), so one 16-byte load, free of
+// bank conflicts across the warp, gives a thread the fragments of two k-steps.
+__host__ __device__ __forceinline__ uint32_t xtile_offset(int n, int kpos) {
+  const int h = kpos >> 7, s8 = (kpos >> 4) & 7, kk = kpos & 15;
+  const int v = s8 >> 1, odd = s8 & 1;
+  const int q = (kk >> 1) & 3, reg = kk >> 3, half = kk & 1;
+  return (uint32_t)((((h * 4 + v) * 2 + (n >> 3)) * 32 + (n & 7) * 4 + q) * 16 +
+                    (odd * 2 + reg) * 4 + half * 2);
+}
+
 // Launch row `warp` of K-block kb's activation tile into slot kb & 1: lane l
-// holds columns 8l .. 8l + 7 (v), stored at their positions in the tile's K
-// order (mma_k_position); also the row's group sums.
+// holds columns 8l .. 8l + 7 (v), each stored at its place in the fragment
+// order (xtile_offset of its tile K position); also the row's group sums.
 __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, int lane,
                                              const uint4& v) {
   const uint32_t slot = (uint32_t)(kb & 1);
-  const uint32_t t = sbase + slot * kXTileBytes + (uint32_t)(warp * kXPitch) * 2u;
+  const uint32_t t = sbase + slot * kXTileBytes;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int e8 = 0; e8 < 8; ++e8) {
     const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(t + (uint32_t)mma_k_position(lane * 8 + e8) * 2u),
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(t + xtile_offset(warp, mma_k_position(lane * 8 + e8))),
                  "h"((unsigned short)half)
                  : "memory");
   }
@@ -187,119 +209,123 @@ __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t y) {
   return d;
 }
 
-// One plane of one row-block for this warp: both 16-row tiles, both groups,
-// all 16 k-steps.  rot: the stage bytes of this row-block and plane;
-// thread (g = lane / 4, q = lane % 4) holds rows g, g + 8, g + 16, g + 24.
+// Tagged partial store (see st_partial) when pred is set, as one predicated
+// instruction rather than a branch.
+__device__ __forceinline__ void st_partial_if(float* p, float v, int pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t"
+      "@q st.relaxed.gpu.global.u32 [%0], %1;\n\t}" ::"l"(p),
+      "r"(~__float_as_uint(v)), "r"(pred)
+      : "memory");
+}
+
+// A shared-memory load at byte offset `off` of the dynamic shared memory, as
+// a plain load (the compiler folds constant parts of the offset into the
+// instruction).  The callers read ring stages only after waiting on their
+// barriers, which are compiler memory barriers too.
+template <typename T>
+__device__ __forceinline__ T sld(const unsigned char* sm, uint32_t off) {
+  return *reinterpret_cast<const T*>(sm + off);
+}
+
+// One plane i of one group h of this warp's row-block: both 16-row tiles, the
+// group's 8 k-steps, every n-tile.  Thread (g = lane / 4, q = lane % 4) holds
+// weight rows g, g + 8, g + 16, g + 24.
 //
-// The packed bytes of row r are rotated by r mod 16 (see bcq_layout.h); the
-// natural 4-byte word v of a pass (chunks 4v .. 4v + 3) starts at rotated
-// byte (4v - rho) mod 16, rho = r mod 16: it is the funnel shift of rotated
-// words (v - R) mod 4 and (v - R + 1) mod 4 by 8 delta bits, with
-// R = ceil(rho / 4) mod 4 and delta = (-rho) mod 4 -- per-thread constants.
-// In the tile's K order (mma_k_position) fragment register s = 8 t + i of
-// a row and 32-column word holds the word's bits 15 - s and 31 - s: it is
-// (word << s) with every bit but 15 and 31 masked, turned into +-alpha by
-// xoring the fp16 sign bits of alpha2 (one lop3).  Thread q needs s = q,
-// q + 4 (k-step 2U: k-pairs q, q + 4) and 8 + q, 12 + q (k-step 2U + 1).
+// Offsets (bytes, from the dynamic shared memory base sm): wa[e][v] of the
+// stored word that begins natural word v of row g (e = 0) or g + 8 (e = 1) in
+// plane i, pass 0; bx of this lane's B fragments in the K-block's tile; sa of
+// the alpha of row g in the warp's scale buffer sbuf.  The packed bytes of row
+// r are rotated by r mod 16 (bcq_layout.h): natural 4-byte word v of a pass
+// (chunks 4v .. 4v + 3) is the funnel shift, by dsh bits, of the stored words
+// (v - R) mod 4 and (v - R + 1) mod 4, R and dsh constants of the thread's
+// rows (rows g + 16 and g + 24 rotate as g and g + 8; passes are 512 bytes
+// apart, rows 16 apart).  In the tile's K order (mma_k_position) fragment
+// register s = 8 t + k-pair of a row and word v (k-step 2v + t) holds the
+// word's bits 15 - s and 31 - s: (word << s) with every other bit masked,
+// turned into +-alpha by xoring the fp16 sign bits of alpha2 (one lop3).
+// Thread q needs k-pairs q and q + 4 of each k-step.
 // MIXED: the rows of the launch have precisions of their own (qm[nt][c]:
 // activation row nt * 8 + 2q + c, 0 past the launch's rows).  The fragments
-// then hold +-1 (exact), each (plane, group) product is accumulated apart
-// and folded into acc[0] with alpha^(qm)[row][group][i] of each activation
-// row (zero for a plane i >= qm): the same sum, with each row's own scales;
-// acc[1] stays zero.
-template <int NT, int P, bool MIXED = false>
-__device__ __forceinline__ void mma_plane(uint32_t rot, uint32_t xt, uint32_t sbuf, int i,
-                                          int g, int q, uint32_t ra0, uint32_t ra1, uint32_t dsh,
-                                          float (&acc)[2][2][NT][4],
-                                          const int (&qm)[NT][2]) {
-  // multipliers for the shifts by q, q + 4, 8 + q, 12 + q
+// then hold +-1 (exact), the (plane, group) product is accumulated apart and
+// folded into acc with alpha^(qm)[row][group][i] of each activation row
+// (zero for a plane i >= qm): the same sum, with each row's own scales.
+template <int NT, int P, bool MIXED>
+__device__ __forceinline__ void mma_group_plane(const unsigned char* sm, const uint32_t (&wa)[2][4],
+                                                uint32_t bx, uint32_t sbuf, uint32_t sa, int i, int h,
+                                                int g, int q, uint32_t dsh, float (&acc)[2][NT][4],
+                                                const int (&qm)[NT][2]) {
   const uint32_t mq0 = 1u << q, mq4 = 1u << (q + 4), mq8 = 1u << (q + 8), mq12 = 1u << (q + 12);
+  uint32_t nw[4][4];
+  uint32_t al[4];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    // activation fragments of the group's 8 k-steps, off the critical path
-    uint32_t bf[8][NT][2];
+  for (int j = 0; j < 4; ++j) {
+    const int pass = (j >> 1) ^ h;  // rows >= 16 hold group A in pass 1
+    const uint32_t o = (uint32_t)(pass * 512 + (j >> 1) * 256);
+    uint32_t w[4];
 #pragma unroll
-    for (int s8 = 0; s8 < 8; ++s8)
+    for (int v = 0; v < 4; ++v) w[v] = sld<uint32_t>(sm, wa[j & 1][v] + o);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t bx =
-            xt + (uint32_t)((nt * 8 + g) * kXPitch + h * 128 + s8 * 16 + 2 * q) * 2u;
-        bf[s8][nt][0] = lds_u32(bx);
-        bf[s8][nt][1] = lds_u32(bx + 16u);
-      }
-    // natural words of group h for rows g, g + 8, g + 16, g + 24
-    uint32_t nw[4][4];
-    uint32_t al[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = g + 8 * j;          // row in the row-block
-      const int pass = (j >> 1) ^ h;    // rows >= 16 hold group A in pass 1
-      const uint32_t ra = (j & 1) ? ra1 : ra0;  // R of this row's rotation
-      const uint32_t base = rot + (uint32_t)pass * 512u + (uint32_t)r * 16u;
-      uint32_t w[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) w[v] = lds_u32(base + (((uint32_t)v - ra) & 3u) * 4u);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) nw[j][v] = funnel_r(w[v], w[(v + 1) & 3], dsh);
-      // alpha of (row, group h, plane i) in both halves (MIXED: +1)
-      if constexpr (MIXED) {
-        al[j] = 0x3C003C00u;
-      } else {
-        const uint32_t ah = lds_u16(sbuf + ((uint32_t)r * 2u * P + (uint32_t)pass * P + i) * 2u);
-        al[j] = ah | (ah << 16);
-      }
+    for (int v = 0; v < 4; ++v) nw[j][v] = funnel_r(w[v], w[(v + 1) & 3], dsh);
+    if constexpr (MIXED) {
+      al[j] = 0x3C003C00u;
+    } else {  // alpha of (row g + 8 j, group h, plane i) in both halves
+      const uint32_t ah = sld<uint16_t>(sm, sa + (uint32_t)(8 * j * 4 * P + pass * 2 * P) + 2u * (uint32_t)i);
+      al[j] = prmt(ah, 0u, 0x1010u);
     }
-    float tmp[2][NT][4];  // MIXED: this (plane, group) alone
+  }
+  float tmp[2][NT][4];  // MIXED: this (plane, group) alone
+  if constexpr (MIXED) {
 #pragma unroll
     for (int f = 0; f < 2; ++f)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) tmp[f][nt][e] = 0.f;
+  }
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {  // word U = v of group h: k-steps 2v, 2v + 1
+  for (int v = 0; v < 4; ++v) {  // word v of group h: k-steps 2v, 2v + 1
+    uint4 bq[NT];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int s8 = 2 * v + t;
-        uint32_t a[4][2];  // row j: k-pairs q (register 8t + q) and q + 4
+    for (int nt = 0; nt < NT; ++nt) bq[nt] = sld<uint4>(sm, bx + (uint32_t)(((h * 4 + v) * 2 + nt) * 512));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          a[j][0] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq8 : mq0), 0x80008000u);
-          a[j][1] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq12 : mq4), 0x80008000u);
-        }
+    for (int t = 0; t < 2; ++t) {
+      uint32_t a[4][2];  // row j: k-pairs q (register 8t + q) and q + 4
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          // tile f: rows 16 f + g (j = 2f) and 16 f + g + 8 (j = 2f + 1)
-          mma_16816(MIXED ? tmp[0][nt] : acc[h][0][nt], a[0][0], a[1][0], a[0][1], a[1][1],
-                    bf[s8][nt][0], bf[s8][nt][1]);
-          mma_16816(MIXED ? tmp[1][nt] : acc[h][1][nt], a[2][0], a[3][0], a[2][1], a[3][1],
-                    bf[s8][nt][0], bf[s8][nt][1]);
-        }
+      for (int j = 0; j < 4; ++j) {
+        a[j][0] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq8 : mq0), 0x80008000u);
+        a[j][1] = xor_andnot(al[j], mul_lo(nw[j][v], t ? mq12 : mq4), 0x80008000u);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t b0 = t ? bq[nt].z : bq[nt].x, b1 = t ? bq[nt].w : bq[nt].y;
+        // tile f: rows 16 f + g (j = 2f) and 16 f + g + 8 (j = 2f + 1)
+        mma_16816(MIXED ? tmp[0][nt] : acc[0][nt], a[0][0], a[1][0], a[0][1], a[1][1], b0, b1);
+        mma_16816(MIXED ? tmp[1][nt] : acc[1][nt], a[2][0], a[3][0], a[2][1], a[3][1], b0, b1);
       }
     }
-    if constexpr (MIXED) {
-      // fold: element e of tile f is weight row 16 f + g + 8 (e / 2) and
-      // activation row nt * 8 + 2q + (e % 2)
+  }
+  if constexpr (MIXED) {
+    // fold: element e of tile f is weight row 16 f + g + 8 (e / 2) and
+    // activation row nt * 8 + 2q + (e % 2)
 #pragma unroll
-      for (int f = 0; f < 2; ++f)
+    for (int f = 0; f < 2; ++f)
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int r = 16 * f + g + 8 * hr;
-          const int pass = (r >> 4) ^ h;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = 16 * f + g + 8 * hr;
+        const int pass = (r >> 4) ^ h;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const int qv = qm[nt][c];
-              float al2 = 0.f;
-              if (i < qv)
-                al2 = h2f((uint16_t)lds_u16(sbuf + mma_alpha_block(qv) +
-                                            ((uint32_t)r * 2u * qv + (uint32_t)pass * qv + i) * 2u));
-              // (both groups into acc[0]: the epilogue adds acc[0] + acc[1])
-              acc[0][f][nt][2 * hr + c] = fmaf(al2, tmp[f][nt][2 * hr + c], acc[0][f][nt][2 * hr + c]);
-            }
-        }
-    }
+          for (int c = 0; c < 2; ++c) {
+            const int qv = qm[nt][c];
+            float al2 = 0.f;
+            if (i < qv)
+              al2 = h2f(sld<uint16_t>(sm, sbuf + mma_alpha_block(qv) +
+                                      ((uint32_t)r * 2u * qv + (uint32_t)pass * qv + i) * 2u));
+            acc[f][nt][2 * hr + c] = fmaf(al2, tmp[f][nt][2 * hr + c], acc[f][nt][2 * hr + c]);
+          }
+      }
   }
 }
 
@@ -361,36 +387,38 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   const int team = warp / kTeamWarps;
   const int tw = warp % kTeamWarps;
   const int g = lane >> 2, q = lane & 3;
-  // rotation constants of this thread's rows (g and g + 8, mod 16)
+  // rotation of this thread's rows g and g + 8 (mod 16; see mma_group_plane)
   const uint32_t ra0 = (uint32_t)(((g + 3) >> 2) & 3), ra1 = (uint32_t)(((g + 11) >> 2) & 3);
   const uint32_t dsh = (uint32_t)((-g) & 3) * 8u;
+  uint32_t woff[2][4];  // stored word that begins natural word v of row g / g + 8, pass 0
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      woff[e][v] = (uint32_t)(g + 8 * e) * 16u + (((uint32_t)v - (e ? ra1 : ra0)) & 3u) * 4u;
   constexpr uint32_t kSbuf = mma_scale_buf_bytes(P, MIXED);
   const uint32_t sbuf0 = sbase + kMmaScaleOff + (uint32_t)warp * 2u * kSbuf;
   const size_t part_stride = (size_t)RB * kRowBlock;
   int qm[NT][2];  // MIXED: precision of this thread's activation rows
+  uint32_t mok = 0;  // bit 2 nt + c: activation row nt * 8 + 2q + c is a row of the launch
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int m = nt * 8 + 2 * q + c;
+      if (m < prm.M) mok |= 1u << (2 * nt + c);
       qm[nt][c] = MIXED && m < prm.M ? prm.qrow[m] : 0;
     }
   int cur_kb = -1;
-  uint4 xn = make_uint4(0u, 0u, 0u, 0u);
-  int xn_kb = -1;
 
-  // tiles of every K-block up to kbt, in order, by all 16 warps
+  // tiles of every K-block up to kbt, in order, by all 16 warps; the next
+  // K-block's activations are prefetched into L2 (no registers held over
+  // the main loop)
   auto advance_tiles = [&](int kbt) {
     while (cur_kb < kbt) {
       const int kbn = cur_kb < 0 ? R.kb0 : cur_kb + 1;
-      if (cur_kb >= 0) {
-        if (xn_kb == kbn) xv = xn;
-        else load_x_tile(prm, kbn, warp, lane, xv);
-      }
-      if (kbn < R.kb_last) {
-        load_x_tile(prm, kbn + 1, warp, lane, xn);
-        xn_kb = kbn + 1;
-      }
+      if (cur_kb >= 0) load_x_tile(prm, kbn, warp, lane, xv);
+      if (kbn < R.kb_last) prefetch_x_tile(prm, kbn + 1, warp, lane);
       // the slot rebuilt was last read two K-blocks ago, before the previous
       // build's barrier
       store_x_tile(sbase, kbn, warp, lane, xv);
@@ -407,12 +435,9 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
   uint32_t ph = 0;
   // scales of the team's groups, staged one group ahead (cp.async, two
   // buffers per warp)
-  GroupCursor pc = gc;
   int buf = 0;
-  if (gg < R.NG && tw < pc.n) stage_scales<P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0);
+  if (gg < R.NG && tw < gc.n) stage_scales<P, MIXED>(prm, gc.kb, gc.rb0 + tw, lane, sbuf0);
   cp_async_commit();
-  cursor_next(pc, R.u1, RB);
-  cursor_next(pc, R.u1, RB);
 
   while (gg < R.NG) {
     advance_tiles(gc.kb);
@@ -420,8 +445,13 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
     const uint32_t sbuf = sbuf0 + (uint32_t)buf * kSbuf;
     // stage the next group's scales into the other buffer, then make sure
     // this group's have landed
-    if (gg + 2 < R.NG && tw < pc.n)
-      stage_scales<P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0 + (uint32_t)(buf ^ 1) * kSbuf);
+    if (gg + 2 < R.NG) {
+      GroupCursor pc = gc;
+      cursor_next(pc, R.u1, RB);
+      cursor_next(pc, R.u1, RB);
+      if (tw < pc.n)
+        stage_scales<P, MIXED>(prm, pc.kb, pc.rb0 + tw, lane, sbuf0 + (uint32_t)(buf ^ 1) * kSbuf);
+    }
     cp_async_commit();
     cp_async_wait<1>();
     __syncwarp();
@@ -430,72 +460,87 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
       record_error(&g_device_error, BCQ_ERR_TIMEOUT);
       *abort_flag = 1;
     }
-    float acc[2][2][NT][4];  // [group][tile]: independent accumulator chains
+    float acc[2][NT][4];  // [16-row tile][n-tile]: both groups, every plane
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int f = 0; f < 2; ++f)
 #pragma unroll
-      for (int f = 0; f < 2; ++f)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[h][f][nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[f][nt][e] = 0.f;
     if (ok && active) {
-      const uint32_t xt = sbase + (uint32_t)(gc.kb & 1) * kXTileBytes;
-      const uint32_t st = ring + (uint32_t)s * kStage + (uint32_t)tw * kUnitPlaneBytes;
+      // (offsets from the shared memory base)
+      const uint32_t st = ring - sbase + (uint32_t)s * kStage + (uint32_t)tw * kUnitPlaneBytes;
+      const uint32_t bx = (uint32_t)(gc.kb & 1) * kXTileBytes + (uint32_t)lane * 16u;
+      const uint32_t so = sbuf - sbase;
+      const uint32_t sa = so + (uint32_t)g * (4u * P);  // alpha of row g
 #pragma unroll 1
-      for (int i = 0; i < P; ++i)
-        mma_plane<NT, P, MIXED>(st + (uint32_t)i * kPlaneGroupBytes, xt, sbuf, i, g, q, ra0, ra1,
-                                dsh, acc, qm);
+      for (int i = 0; i < P; ++i) {
+        const uint32_t sp = st + (uint32_t)i * kPlaneGroupBytes;
+        uint32_t wa[2][4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) wa[e][v] = sp + woff[e][v];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          mma_group_plane<NT, P, MIXED>(smem, wa, bx, so, sa, i, h, g, q, dsh, acc, qm);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive_cta(empty0 + 8u * s);
     if (ok && active && *abort_flag == 0) {
       // offsets: z[row][group] * S[m][group]; then the unit's partial sums
-      const uint32_t gsl = sbase + kMmaGsumOff + (uint32_t)(gc.kb & 1) * kMmaRows * 8u;
-      float sg[NT][2][2];  // S[m][group] of this thread's activation rows m
+      const uint32_t gsl = kMmaGsumOff + (uint32_t)(gc.kb & 1) * kMmaRows * 8u;
+      const uint32_t so = sbuf - sbase;
+      float2 sg[NT][2];  // S[m][group 0 / 1] of this thread's activation rows m
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int m = nt * 8 + 2 * q + c;
-          sg[nt][c][0] = lds_f32_dyn(gsl + (uint32_t)(m * 2) * 4u);
-          sg[nt][c][1] = lds_f32_dyn(gsl + (uint32_t)(m * 2 + 1) * 4u);
-        }
+        for (int c = 0; c < 2; ++c)
+          sg[nt][c] = sld<float2>(smem, gsl + (uint32_t)(nt * 8 + 2 * q + c) * 8u);
+      const int row0 = (gc.rb0 + tw) * kRowBlock + g;  // weight row of f = hr = 0
+      float* pm[NT][2];
+      if (prm.KB > 1) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            pm[nt][c] = prm.part + ((size_t)gc.kb * prm.M + (nt * 8 + 2 * q + c)) * part_stride +
+                        (size_t)row0;
+      }
 #pragma unroll
       for (int f = 0; f < 2; ++f) {
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
           const int r = 16 * f + g + 8 * hr;
-          float zz[2] = {0.f, 0.f};
+          // offsets of groups 0 and 1: group h sits in pass (r / 16) ^ h
+          float z0 = 0.f, z1 = 0.f;
           if (!MIXED && prm.z) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              zz[h] = h2f((uint16_t)lds_u16(sbuf + mma_z_off(P) +
-                                            (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
+            const uint32_t zw = sld<uint32_t>(smem, so + mma_z_off(P) + (uint32_t)r * 4u);
+            z0 = h2f((uint16_t)(f ? zw >> 16 : zw & 0xFFFFu));
+            z1 = h2f((uint16_t)(f ? zw & 0xFFFFu : zw >> 16));
           }
-          const int row = (gc.rb0 + tw) * kRowBlock + r;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const int m = nt * 8 + 2 * q + c;
               if constexpr (MIXED) {  // the offsets of this activation row's precision
                 const int qv = qm[nt][c];
-                zz[0] = zz[1] = 0.f;
+                z0 = z1 = 0.f;
                 if (qv > 0 && prm.z_q[qv - 1]) {
-#pragma unroll
-                  for (int h = 0; h < 2; ++h)
-                    zz[h] = h2f((uint16_t)lds_u16(sbuf + mma_z_off(P, true, qv) +
-                                                  (uint32_t)(r * 2 + ((r >> 4) ^ h)) * 2u));
+                  const uint32_t zw = sld<uint32_t>(smem, so + mma_z_off(P, true, qv) + (uint32_t)r * 4u);
+                  z0 = h2f((uint16_t)(f ? zw >> 16 : zw & 0xFFFFu));
+                  z1 = h2f((uint16_t)(f ? zw & 0xFFFFu : zw >> 16));
                 }
               }
-              float v = acc[0][f][nt][2 * hr + c] + acc[1][f][nt][2 * hr + c];
-              v = fmaf(zz[0], sg[nt][c][0], fmaf(zz[1], sg[nt][c][1], v));
-              if (m < prm.M) {
-                if (prm.KB > 1)
-                  st_partial(prm.part + ((size_t)gc.kb * prm.M + m) * part_stride + (size_t)row, v);
-                else if (row < prm.N)
-                  prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(v);
+              const float v =
+                  fmaf(z0, sg[nt][c].x, fmaf(z1, sg[nt][c].y, acc[f][nt][2 * hr + c]));
+              if (prm.KB > 1) {
+                st_partial_if(pm[nt][c] + (16 * f + 8 * hr), v, (int)((mok >> (2 * nt + c)) & 1u));
+              } else {
+                const int m = nt * 8 + 2 * q + c;
+                const int row = row0 + 16 * f + 8 * hr;
+                if (((mok >> (2 * nt + c)) & 1u) && row < prm.N) prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(v);
               }
             }
           }
@@ -503,8 +548,6 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
       }
     }
     buf ^= 1;
-    cursor_next(pc, R.u1, RB);
-    cursor_next(pc, R.u1, RB);
     cursor_next(gc, R.u1, RB);
     cursor_next(gc, R.u1, RB);
     s += 2;

@@ -136,6 +136,69 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
   __syncwarp();
 }
 
+// One reduction task of splitk_tail: the lane's row of launch rows m0 ..
+// m0 + NM - 1 (pp: its first partial), all KB K-blocks, kC at a time; sums
+// them in K-block order into sum[] and zeroes them.  FULL: KB is a multiple
+// of kC (no guard on the loads).  False when a wait ran out (warp-uniform).
+template <int kC, int NM, bool FULL>
+__device__ __forceinline__ bool reduce_task(const GemvParams& prm, float* pp, size_t part_stride,
+                                            size_t kstride, int KB, float (&sum)[2],
+                                            volatile int* abort_flag) {
+  for (int k0 = 0; k0 < KB; k0 += kC) {
+    float* pk = pp + (size_t)k0 * kstride;
+    uint32_t v[NM][kC];  // every load of the chunk in flight at once
+#pragma unroll
+    for (int mm = 0; mm < NM; ++mm) {
+      const float* pl = pk + (size_t)mm * part_stride;
+#pragma unroll
+      for (int j = 0; j < kC; ++j) {
+        v[mm][j] = (FULL || k0 + j < KB) ? ld_partial_tag(pl) : 1u;
+        pl += kstride;
+      }
+    }
+    bool have = true;
+#pragma unroll
+    for (int mm = 0; mm < NM; ++mm)
+#pragma unroll
+      for (int j = 0; j < kC; ++j) have = have && v[mm][j] != 0u;
+    if (!__all_sync(0xFFFFFFFFu, have)) {
+      // some partials are still on their way: re-load the missing ones
+      const unsigned long long t0 = globaltimer_ns();
+#pragma unroll 1
+      while (true) {
+        __nanosleep(32);
+        have = true;
+#pragma unroll
+        for (int mm = 0; mm < NM; ++mm)
+#pragma unroll
+          for (int j = 0; j < kC; ++j) {
+            if (v[mm][j] == 0u)
+              v[mm][j] = ld_partial_tag(pk + (size_t)mm * part_stride + (size_t)j * kstride);
+            have = have && v[mm][j] != 0u;
+          }
+        if (__all_sync(0xFFFFFFFFu, have)) break;
+        // (warp-uniform: every lane leaves the loop together)
+        if (__any_sync(0xFFFFFFFFu, *abort_flag != 0 || globaltimer_ns() - t0 > prm.timeout_ns))
+          return false;
+      }
+    }
+#pragma unroll
+    for (int mm = 0; mm < NM; ++mm) {
+      float* pz = pk + (size_t)mm * part_stride;
+#pragma unroll
+      for (int j = 0; j < kC; ++j) {
+        if (FULL || k0 + j < KB) {
+          sum[mm] += partial_value(v[mm][j]);
+          // the workspace is left zero-filled for any later shape
+          stg_cg_zero(pz);
+        }
+        pz += kstride;
+      }
+    }
+  }
+  return true;
+}
+
 // Split-K reduction, run by each of the CTA's nthreads consumer threads once
 // its warp has stored its own partial sums (no barrier).  Every unit's fp32
 // partials [kb][m][row] go to the workspace as tagged words (st_partial: zero
@@ -147,12 +210,11 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
 // computed its unit in K-block rb mod KB, so the work is spread evenly
 // whatever the order in which CTAs finish.  The (row-block, two launch rows)
 // tasks of the CTA are dealt to its warps in turn; a warp loads all KB
-// partials of its task at once, re-loads (bounded) those still zero, adds
-// them in K-block order (the result does not depend on scheduling), writes y
-// (row m of the launch goes to y row ymap[m], or m without a map) and zeroes
-// those partials, so the workspace is zero again for the next call.  kC
-// K-blocks of partials are loaded at once (one round trip each): 16 where
-// registers allow (the lookup kernel), 8 in the tensor-core kernels.
+// partials of its task kC K-blocks at a time (one round trip each), re-loads
+// (bounded) those still zero, adds them in K-block order (the result does not
+// depend on scheduling), writes y (row m of the launch goes to y row ymap[m],
+// or m without a map) and zeroes those partials, so the workspace is zero
+// again for the next call.
 template <int kC>
 __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRange& R, int Mrows,
                                             const int* ymap, int tid, int nthreads,
@@ -162,6 +224,7 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
   const size_t part_stride = (size_t)RB * kRowBlock;
   const size_t kstride = (size_t)Mrows * part_stride;  // one K-block of partials
   const bool live = *abort_flag == 0;
+  const bool full = KB % kC == 0;
   // Tasks are dealt round-robin (no division), starting at the first warp of
   // the second team: the first team takes the odd group out of an odd
   // number, so the second team is done first and polls earlier (measured:
@@ -180,52 +243,11 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
         const int nm = Mrows - m0 < 2 ? Mrows - m0 : 2;
         float* pp = prm.part + (size_t)m0 * part_stride + (size_t)row;
         float sum[2] = {0.f, 0.f};
-        bool ok = true;
-        for (int k0 = 0; k0 < KB && ok; k0 += kC) {
-          uint32_t v[2][kC];  // every load of the chunk in flight at once
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int j = 0; j < kC; ++j)
-              v[mm][j] = mm < nm && k0 + j < KB
-                             ? ld_partial_tag(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride)
-                             : 1u;
-          bool have = true;
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int j = 0; j < kC; ++j) have = have && v[mm][j] != 0u;
-          if (!__all_sync(0xFFFFFFFFu, have)) {
-            // some partials are still on their way: re-load the missing ones
-            const unsigned long long t0 = globaltimer_ns();
-#pragma unroll 1
-            while (true) {
-              __nanosleep(32);
-              have = true;
-#pragma unroll
-              for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-                for (int j = 0; j < kC; ++j) {
-                  if (v[mm][j] == 0u)
-                    v[mm][j] = ld_partial_tag(pp + (size_t)mm * part_stride + (size_t)(k0 + j) * kstride);
-                  have = have && v[mm][j] != 0u;
-                }
-              if (__all_sync(0xFFFFFFFFu, have)) break;
-              // (warp-uniform: every lane leaves the loop together)
-              if (__any_sync(0xFFFFFFFFu,
-                             *abort_flag != 0 || globaltimer_ns() - t0 > prm.timeout_ns)) {
-                ok = false;
-                break;
-              }
-            }
-          }
-          if (!ok) break;
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm)
-#pragma unroll
-            for (int j = 0; j < kC; ++j)
-              if (k0 + j < KB) sum[mm] += partial_value(v[mm][j]);
-        }
+        const bool ok =
+            nm == 2 ? (full ? reduce_task<kC, 2, true>(prm, pp, part_stride, kstride, KB, sum, abort_flag)
+                            : reduce_task<kC, 2, false>(prm, pp, part_stride, kstride, KB, sum, abort_flag))
+                    : (full ? reduce_task<kC, 1, true>(prm, pp, part_stride, kstride, KB, sum, abort_flag)
+                            : reduce_task<kC, 1, false>(prm, pp, part_stride, kstride, KB, sum, abort_flag));
         if (!ok) {
           if (lane == 0 && *abort_flag == 0) {
             record_error(&g_device_error, BCQ_ERR_TIMEOUT);
@@ -233,12 +255,9 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
           }
           continue;
         }
-        for (int mm = 0; mm < nm; ++mm) {
-          const int ym = ymap ? ymap[m0 + mm] : m0 + mm;
-          if (row < prm.N) prm.y[(size_t)ym * prm.N + row] = f2h_rn(sum[mm]);
-          // the workspace is left zero-filled for any later shape
-          for (int k = 0; k < KB; ++k)
-            stg_cg_zero(pp + (size_t)mm * part_stride + (size_t)k * kstride);
+        if (row < prm.N) {
+          prm.y[(size_t)(ymap ? ymap[m0] : m0) * prm.N + row] = f2h_rn(sum[0]);
+          if (nm == 2) prm.y[(size_t)(ymap ? ymap[m0 + 1] : m0 + 1) * prm.N + row] = f2h_rn(sum[1]);
         }
       }
     }

@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
   // (no barrier: a warp starts its reduction tasks as soon as it is done;
   // the partials it waits for are polled, not counted)
   if (prm.KB > 1) {
-    splitk_tail<4>(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
+    splitk_tail<8>(prm, R, prm.M, prm.rows, tid, kConsumers, abort_flag);
   }
 }
 

@@ -533,18 +533,38 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + 2), 1)
                   z1 = h2f((uint16_t)(f ? zw & 0xFFFFu : zw >> 16));
                 }
               }
-              const float v =
+              acc[f][nt][2 * hr + c] =
                   fmaf(z0, sg[nt][c].x, fmaf(z1, sg[nt][c].y, acc[f][nt][2 * hr + c]));
-              if (prm.KB > 1) {
-                st_partial_if(pm[nt][c] + (16 * f + 8 * hr), v, (int)((mok >> (2 * nt + c)) & 1u));
-              } else {
-                const int m = nt * 8 + 2 * q + c;
-                const int row = row0 + 16 * f + 8 * hr;
-                if (((mok >> (2 * nt + c)) & 1u) && row < prm.N) prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(v);
-              }
             }
           }
         }
+      }
+      // (one uniform branch around all the stores)
+      if (prm.KB > 1) {
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                st_partial_if(pm[nt][c] + (16 * f + 8 * hr), acc[f][nt][2 * hr + c],
+                              (int)((mok >> (2 * nt + c)) & 1u));
+      } else {
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                const int m = nt * 8 + 2 * q + c;
+                const int row = row0 + 16 * f + 8 * hr;
+                if (((mok >> (2 * nt + c)) & 1u) && row < prm.N)
+                  prm.y[(size_t)prm.rows[m] * prm.N + row] = f2h_rn(acc[f][nt][2 * hr + c]);
+              }
       }
     }
     buf ^= 1;

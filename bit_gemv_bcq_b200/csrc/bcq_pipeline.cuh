@@ -235,8 +235,13 @@ __device__ __forceinline__ void splitk_tail(const GemvParams& prm, const CtaRang
     const int b = kb == R.kb_last ? R.u1 - kb * RB : RB;
     int first = kb;  // designated row-blocks: kb, kb + KB, ...
     if (first < a) first += (a - first + KB - 1) / KB * KB;
+    const int mp = (Mrows + 1) >> 1;  // tasks per row-block: two launch rows each
     for (int rbx = first; rbx < b; rbx += KB) {
-      for (int m0 = 0; m0 < Mrows; m0 += 2, ++task) {  // two launch rows per task
+      if (mine >= task + mp) {  // none of this row-block's tasks is this warp's
+        task += mp;
+        continue;
+      }
+      for (int m0 = 0; m0 < Mrows; m0 += 2, ++task) {
         if (task != mine) continue;
         mine += nwarps;
         const int row = rbx * kRowBlock + lane;

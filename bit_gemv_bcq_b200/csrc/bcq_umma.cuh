@@ -301,6 +301,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
     for (int gg = team; gg < R.NG; gg += 2) {
       if (hf * 4 < gc.n) {  // the same test as the group's expanding warps
         const uint32_t xt = sbase + (uint32_t)(gc.kb & 1) * S::kXTileBytes;
+        // descriptor of the tile's first K-slice; slice j is NN * 32 bytes on,
+        // i.e. NN * 2 in the descriptor's start-address field (address / 16,
+        // 14 bits: shared addresses stay below 2^18, so the add never carries
+        // out of the field)
+        const uint64_t bd0 = umma_bdesc<NN>(xt);
         const uint32_t tacc = tg + (uint32_t)accb * (uint32_t)NN;
         // the accumulator's previous unit has been read
         if (acc_round > 0 &&
@@ -316,12 +321,11 @@ __global__ void __launch_bounds__(32 * (kConsumerWarps + kUmmaGroups + 2), 1)
             if (lane == 0) {
               if (*abort_flag == 0) {
                 const uint32_t acol = tg + S::kACol + (uint32_t)ab * kUmmaABufCols;
+                const uint64_t bdc = bd0 + (uint64_t)(4 * c) * (NN * 2u);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                  umma_f16_ts(tacc, acol + 8u * (uint32_t)j,
-                              umma_bdesc<NN>(xt + (uint32_t)(4 * c + j) * (NN * 32u)),
-                              umma_idesc<NN>(),
-                              (i | c | j) != 0 ? 1u : 0u);
+                  umma_f16_ts(tacc, acol + 8u * (uint32_t)j, bdc + (uint64_t)j * (NN * 2u),
+                              umma_idesc<NN>(), j != 0 || (i | c) != 0 ? 1u : 0u);
               }
               umma_commit(bars.aempty + 8u * ab);
             }

@@ -126,30 +126,35 @@ __device__ __forceinline__ float plane_sum1c(const uint4& w, const uint32_t (&cr
 
 // ------------------------------------------------------------- producers
 
-// Producer warp pw of NP streams stages k = pw, pw + NP, ... of the CTA:
-// stage k = group k (at most 8 row-blocks of one K-block in one row group):
-// its P planes (one bulk copy for a whole row group, one per plane
-// otherwise), its packed scales alpha^(P) and its packed offsets.  Planes,
-// scales and offsets are read once per call: evict-first in L2, so x and
-// the workspace stay there.  Lane 0 issues; the warp returns when every
-// copy it issued has landed (or the CTA gave up).
+// The three producer warps stream every stage k of the CTA (stage k = group
+// k: at most 8 row-blocks of one K-block in one row group), each its own
+// part: warp 0 the P planes (one bulk copy for a whole row group, one per
+// plane otherwise), warp 1 the packed scales alpha^(P), warp 2 the packed
+// offsets (or, without offsets, only its arrival).  Each arrives on the
+// stage's full barrier with the bytes it copies (three arrivals a phase), so
+// the first stage's copies go out at once instead of one after another.  A
+// producer cannot run a ring ahead of the others: slot s is refilled only
+// after the stage before it was consumed, which needed all three parts.
+// Planes, scales and offsets are read once per call: evict-first in L2, so x
+// and the workspace stay there.  Lane 0 issues; the warp returns when every
+// stage of the last ring has landed (or the CTA gave up).
+constexpr int kM1Producers = 3;
 template <int P>
 __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const CtaRange& R,
                                                   int pw, int lane, uint32_t ring,
                                                   uint32_t full0, uint32_t empty0,
                                                   volatile int* abort_flag) {
   constexpr uint32_t kStage = m1_stage_bytes(P);
-  const int D = prm.D, NP = prm.NP, RB = prm.RB;
+  const int D = prm.D, RB = prm.RB;
   if (!prm.early_weights) grid_dependency_wait();
   if (lane == 0) {
     const uint64_t pol = evict_first_policy();
     int issued = 0;
     GroupCursor gc;
     cursor_init(gc, R.u0, R.u1, R.kb0, RB);
-    for (int t = 0; t < pw; ++t) cursor_next(gc, R.u1, RB);
-    int s = pw;
+    int s = 0;
     uint32_t eph = 1;
-    for (int k = pw; k < R.NG; k += NP) {
+    for (int k = 0; k < R.NG; ++k) {
       if (k >= D && !mbar_wait_bounded(empty0 + 8u * s, eph, prm.timeout_ns)) {
         record_error(&g_device_error, BCQ_ERR_TIMEOUT);
         *abort_flag = 1;
@@ -157,34 +162,42 @@ __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const C
       if (*abort_flag) break;
       const uint32_t bar = full0 + 8u * s;
       const uint32_t dst = ring + (uint32_t)s * kStage;
-      const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
       const uint32_t n = (uint32_t)gc.n;
-      const uint32_t* src =
-          prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H * (kRowGroup * kWordsPerUnitPlane);
       const size_t unit = (size_t)gc.kb * RB + gc.rb0;  // packed scale unit of row-block rb0
-      mbar_arrive_expect_tx(bar, n * (P * kUnitPlaneBytes + 128u * P + (prm.z ? 128u : 0u)));
-      if (gc.n == kRowGroup) {
-        bulk_g2s_hint(dst, src, (uint32_t)P * kPlaneGroupBytes, bar, pol);
-      } else {
+      if (pw == 0) {
+        const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
+        const uint32_t* src =
+            prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H * (kRowGroup * kWordsPerUnitPlane);
+        mbar_arrive_expect_tx(bar, n * (uint32_t)P * kUnitPlaneBytes);
+        if (gc.n == kRowGroup) {
+          bulk_g2s_hint(dst, src, (uint32_t)P * kPlaneGroupBytes, bar, pol);
+        } else {
 #pragma unroll
-        for (int i = 0; i < P; ++i)
-          bulk_g2s_hint(dst + (uint32_t)i * kPlaneGroupBytes,
-                        src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
-                        n * kUnitPlaneBytes, bar, pol);
+          for (int i = 0; i < P; ++i)
+            bulk_g2s_hint(dst + (uint32_t)i * kPlaneGroupBytes,
+                          src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
+                          n * kUnitPlaneBytes, bar, pol);
+        }
+      } else if (pw == 1) {
+        mbar_arrive_expect_tx(bar, n * 128u * P);
+        bulk_g2s_hint(dst + m1_alpha_off(P), prm.alpha[0] + unit * (64u * P), n * 128u * P, bar,
+                      pol);
+      } else if (prm.z) {
+        mbar_arrive_expect_tx(bar, n * 128u);
+        bulk_g2s_hint(dst + m1_z_off(P), prm.z + unit * 64u, n * 128u, bar, pol);
+      } else {
+        mbar_arrive_cta(bar);
       }
-      bulk_g2s_hint(dst + m1_alpha_off(P), prm.alpha[0] + unit * (64u * P), n * 128u * P, bar,
-                    pol);
-      if (prm.z) bulk_g2s_hint(dst + m1_z_off(P), prm.z + unit * 64u, n * 128u, bar, pol);
       issued = k + 1;
-      for (int t = 0; t < NP; ++t) cursor_next(gc, R.u1, RB);
-      s += NP;
-      if (s >= D) {
-        s -= D;
+      cursor_next(gc, R.u1, RB);
+      if (++s == D) {
+        s = 0;
         eph ^= 1u;
       }
     }
-    // every copy this warp issued lands before the CTA may exit
-    for (int s2 = pw; s2 < D && s2 < issued; s2 += NP) {
+    // every copy this warp issued lands before the CTA may exit (the full
+    // barriers of the last ring's stages complete only when all parts have)
+    for (int s2 = 0; s2 < D && s2 < issued; ++s2) {
       const int klast = issued - 1 - ((issued - 1 - s2) % D);
       (void)mbar_wait_bounded(full0 + 8u * s2, (uint32_t)((klast / D) & 1), prm.timeout_ns);
     }
@@ -196,11 +209,11 @@ __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const C
 
 // One CTA per SM over units [u0, u1) (kb-major, host-planned): warps 0..15
 // consume in two teams of 8 that take alternate stages (team warp w:
-// row-block rb0 + w of the stage), warps 16..15+NP produce (producer pw:
-// stages pw, pw + NP, ...).  P: the precision (planes streamed, scales
+// row-block rb0 + w of the stage), warps 16..18 produce (planes, scales,
+// offsets of every stage).  P: the precision (planes streamed, scales
 // alpha^(P)).
 template <int P>
-__global__ void __launch_bounds__(32 * (kM1Warps + 2), 1)
+__global__ void __launch_bounds__(32 * (kM1Warps + kM1Producers), 1)
     gemv_m1_kernel(const __grid_constant__ GemvParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -217,15 +230,15 @@ __global__ void __launch_bounds__(32 * (kM1Warps + 2), 1)
 
   // The table is addressed through load immediates: the dynamic shared
   // memory must start where they assume.  A stage's team consumed the stage
-  // D earlier (D even: teams alternate), and each producer refills only its
-  // own slots (D a multiple of NP).
-  const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP >= 1 && NP <= 2 &&
-                      (D & 1) == 0 && D % NP == 0 && (int)blockDim.x == 32 * (kM1Warps + NP);
+  // D earlier (D even: teams alternate); three producers (one part of every
+  // stage each).
+  const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP == kM1Producers &&
+                      (D & 1) == 0 && (int)blockDim.x == 32 * (kM1Warps + NP);
   CtaRange R;
   make_range(prm, R);
   if (warp == kM1Warps) {
     if (cfg_ok && lane < D) {  // one lane per ring slot
-      mbar_init(full0 + 8u * lane, 1);
+      mbar_init(full0 + 8u * lane, kM1Producers);
       mbar_init(empty0 + 8u * lane, kM1TeamWarps);
     }
     if (lane == 0) {

@@ -92,6 +92,7 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
   const int D = prm.D, NP = prm.NP, RB = prm.RB;
   if (!prm.early_weights) grid_dependency_wait();
   if (lane == 0) {
+    const uint64_t pol = evict_first_policy();  // planes are read once per call
     int issued = 0;
     GroupCursor gc;
     cursor_init(gc, R.u0, R.u1, R.kb0, RB);
@@ -111,13 +112,13 @@ __device__ __forceinline__ void produce_stages(const GemvParams& prm, const CtaR
           prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H * (kRowGroup * kWordsPerUnitPlane);
       mbar_arrive_expect_tx(bar, (uint32_t)(P * gc.n) * kUnitPlaneBytes);
       if (gc.n == kRowGroup) {
-        bulk_g2s(dst, src, kStage, bar);
+        bulk_g2s_hint(dst, src, kStage, bar, pol);
       } else {
 #pragma unroll
         for (int i = 0; i < P; ++i)
-          bulk_g2s(dst + (uint32_t)i * kPlaneGroupBytes,
-                   src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
-                   (uint32_t)gc.n * kUnitPlaneBytes, bar);
+          bulk_g2s_hint(dst + (uint32_t)i * kPlaneGroupBytes,
+                        src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
+                        (uint32_t)gc.n * kUnitPlaneBytes, bar, pol);
       }
       issued = k + 1;
       for (int t = 0; t < NP; ++t) cursor_next(gc, R.u1, RB);

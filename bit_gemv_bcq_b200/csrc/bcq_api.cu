@@ -137,8 +137,8 @@ bcq_status plan_gemv(int M, int N, int K, int P, bool mixed, int path, Plan* out
   const long long KB = (long long)k_blocks(K);
   const long long U = RB * KB;
   pl.KB = (int)KB;
-  // (the one-row kernel: three producers, one part of every stage each)
-  pl.NP = path == kPathM1 ? 3 : std::max(1, std::min(2, env_int("BCQ_FORCE_NP", kDefaultProducers)));
+  // (the one-row kernel: m1_producers(P) producers, one part of every stage each)
+  pl.NP = path == kPathM1 ? m1_producers(P) : std::max(1, std::min(2, env_int("BCQ_FORCE_NP", kDefaultProducers)));
   // ring stages: even (the two teams alternate) and a multiple of NP
   const int step = 2;
   const size_t dyn_cap = kMaxDynSmem;

@@ -108,6 +108,10 @@ __host__ __device__ constexpr uint32_t gemv_dyn_bytes(int D, int P, int M = 1) {
 // scales + offsets; then the full / empty barriers and the abort flag.
 constexpr int kM1Warps = 16;
 constexpr int kM1TeamWarps = 8;
+// Producer warps of the one-row kernel for P planes, one part of every stage
+// each (measured: splitting the planes between two warps pays at four planes
+// only).
+__host__ __device__ constexpr int m1_producers(int P) { return P >= 4 ? 4 : 3; }
 constexpr uint32_t kLut1Bytes = 32768;
 __host__ __device__ constexpr uint32_t m1_alpha_off(int P) {
   return (uint32_t)P * kPlaneGroupBytes;

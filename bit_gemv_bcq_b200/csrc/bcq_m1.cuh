@@ -126,19 +126,19 @@ __device__ __forceinline__ float plane_sum1c(const uint4& w, const uint32_t (&cr
 
 // ------------------------------------------------------------- producers
 
-// The three producer warps stream every stage k of the CTA (stage k = group
+// The four producer warps stream every stage k of the CTA (stage k = group
 // k: at most 8 row-blocks of one K-block in one row group), each its own
-// part: warp 0 the P planes (one bulk copy for a whole row group, one per
-// plane otherwise), warp 1 the packed scales alpha^(P), warp 2 the packed
-// offsets (or, without offsets, only its arrival).  Each arrives on the
-// stage's full barrier with the bytes it copies (three arrivals a phase), so
-// the first stage's copies go out at once instead of one after another.  A
-// producer cannot run a ring ahead of the others: slot s is refilled only
-// after the stage before it was consumed, which needed all three parts.
+// part: warps 0 and 1 the first half of the planes and the rest at P = 4,
+// warp 0 all of them below (one bulk copy for a whole row group, one per
+// plane otherwise), warp 2 the packed scales alpha^(P), warp 3 the packed
+// offsets (a warp with nothing to copy only arrives).  Each arrives on the stage's full barrier with the bytes it
+// copies (four arrivals a phase), so a stage's copies go out at once instead
+// of one after another.  A producer cannot run a ring ahead of the others:
+// slot s is refilled only after the stage before it was consumed, which
+// needed every part.
 // Planes, scales and offsets are read once per call: evict-first in L2, so x
 // and the workspace stay there.  Lane 0 issues; the warp returns when every
 // stage of the last ring has landed (or the CTA gave up).
-constexpr int kM1Producers = 3;
 template <int P>
 __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const CtaRange& R,
                                                   int pw, int lane, uint32_t ring,
@@ -147,6 +147,9 @@ __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const C
   constexpr uint32_t kStage = m1_stage_bytes(P);
   const int D = prm.D, RB = prm.RB;
   if (!prm.early_weights) grid_dependency_wait();
+  // role: 0 / 1 the two halves of the planes (1 unused below four planes),
+  // 2 the scales, 3 the offsets
+  const int role = m1_producers(P) == 3 && pw >= 1 ? pw + 1 : pw;
   if (lane == 0) {
     const uint64_t pol = evict_first_policy();
     int issued = 0;
@@ -164,21 +167,24 @@ __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const C
       const uint32_t dst = ring + (uint32_t)s * kStage;
       const uint32_t n = (uint32_t)gc.n;
       const size_t unit = (size_t)gc.kb * RB + gc.rb0;  // packed scale unit of row-block rb0
-      if (pw == 0) {
+      if (role < 2) {  // planes [i0, i1): the first half of them, or the rest
+        constexpr int kHalf = m1_producers(P) == 4 ? P / 2 : P;
+        const int i0 = role ? kHalf : 0, i1 = role ? P : kHalf;
         const int rg = gc.rb0 / kRowGroup, r0 = gc.rb0 - rg * kRowGroup;
         const uint32_t* src =
             prm.planes + ((size_t)gc.kb * prm.RG + rg) * prm.p_H * (kRowGroup * kWordsPerUnitPlane);
-        mbar_arrive_expect_tx(bar, n * (uint32_t)P * kUnitPlaneBytes);
-        if (gc.n == kRowGroup) {
-          bulk_g2s_hint(dst, src, (uint32_t)P * kPlaneGroupBytes, bar, pol);
+        mbar_arrive_expect_tx(bar, n * (uint32_t)(i1 - i0) * kUnitPlaneBytes);
+        if (i1 > i0 && gc.n == kRowGroup) {
+          bulk_g2s_hint(dst + (uint32_t)i0 * kPlaneGroupBytes,
+                        src + (size_t)i0 * kRowGroup * kWordsPerUnitPlane,
+                        (uint32_t)(i1 - i0) * kPlaneGroupBytes, bar, pol);
         } else {
-#pragma unroll
-          for (int i = 0; i < P; ++i)
+          for (int i = i0; i < i1; ++i)
             bulk_g2s_hint(dst + (uint32_t)i * kPlaneGroupBytes,
                           src + (size_t)(i * kRowGroup + r0) * kWordsPerUnitPlane,
                           n * kUnitPlaneBytes, bar, pol);
         }
-      } else if (pw == 1) {
+      } else if (role == 2) {
         mbar_arrive_expect_tx(bar, n * 128u * P);
         bulk_g2s_hint(dst + m1_alpha_off(P), prm.alpha[0] + unit * (64u * P), n * 128u * P, bar,
                       pol);
@@ -209,11 +215,11 @@ __device__ __forceinline__ void produce_m1_stages(const GemvParams& prm, const C
 
 // One CTA per SM over units [u0, u1) (kb-major, host-planned): warps 0..15
 // consume in two teams of 8 that take alternate stages (team warp w:
-// row-block rb0 + w of the stage), warps 16..18 produce (planes, scales,
+// row-block rb0 + w of the stage), warps 16.. produce (planes, scales,
 // offsets of every stage).  P: the precision (planes streamed, scales
 // alpha^(P)).
 template <int P>
-__global__ void __launch_bounds__(32 * (kM1Warps + kM1Producers), 1)
+__global__ void __launch_bounds__(32 * (kM1Warps + m1_producers(P)), 1)
     gemv_m1_kernel(const __grid_constant__ GemvParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -232,13 +238,13 @@ __global__ void __launch_bounds__(32 * (kM1Warps + kM1Producers), 1)
   // memory must start where they assume.  A stage's team consumed the stage
   // D earlier (D even: teams alternate); three producers (one part of every
   // stage each).
-  const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP == kM1Producers &&
+  const bool cfg_ok = sbase == kDynBase && D >= 2 && D <= kMaxStages && NP == m1_producers(P) &&
                       (D & 1) == 0 && (int)blockDim.x == 32 * (kM1Warps + NP);
   CtaRange R;
   make_range(prm, R);
   if (warp == kM1Warps) {
     if (cfg_ok && lane < D) {  // one lane per ring slot
-      mbar_init(full0 + 8u * lane, kM1Producers);
+      mbar_init(full0 + 8u * lane, m1_producers(P));
       mbar_init(empty0 + 8u * lane, kM1TeamWarps);
     }
     if (lane == 0) {

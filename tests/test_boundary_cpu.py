@@ -99,8 +99,9 @@ def test_launch_plans_respect_the_pipeline_rules(L, M, N, K, p, mixed):
         assert pl["consumer_warps"] == 16
         assert pl["dyn_bytes"] <= 232448
         assert pl["dyn_bytes"] >= 32768 + pl["D"] * pl["stage_bytes"]
-        # three producers, one part of every stage each (planes, scales, offsets)
-        assert pl["NP"] == 3
+        # a producer per part of every stage: planes (two halves at four
+        # planes), scales, offsets
+        assert pl["NP"] == (4 if p >= 4 else 3)
         assert pl["D"] % 2 == 0 and 2 <= pl["D"] <= 20
         assert pl["D"] == 20 or pl["dyn_bytes"] + 2 * pl["stage_bytes"] > 232448
         assert pl["units_max"] == -(-U // pl["C"])

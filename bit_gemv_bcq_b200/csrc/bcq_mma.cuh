@@ -177,21 +177,49 @@ __host__ __device__ __forceinline__ uint32_t xtile_offset(int n, int kpos) {
                     (odd * 2 + reg) * 4 + half * 2);
 }
 
+// Where column 8l + e8 of a K-block goes in the fragment-ordered tile
+// (xtile_offset of its mma_k_position), written out for a lane: with j = l % 4
+// the column's stored bit is b = 8j + (e8 + 7) mod 8, its register index
+// s = (j odd ? 7 : 15) - (e8 + 7) mod 8, and its byte offset is
+//   base(n, l) + (s mod 4) * 16 + (s / 8) * 8 + ((s / 4) mod 2) * 4
+// with base(n, l) = ((((l / 16) * 4 + (l / 4) % 4) * 2 + n / 8) * 32 + (n % 8) * 4) * 16
+// + 2 ((l / 2) % 2).  For odd j every such offset is 8 bytes below the even
+// one, so the lane's base takes - 8 (l % 2) and the eight offsets are
+// compile-time constants (checked against xtile_offset for every n, l, e8).
+__host__ __device__ constexpr uint32_t xtile_col_off(int e8) {
+  return (uint32_t)(((15 - ((e8 + 7) & 7)) & 3) * 16 + ((15 - ((e8 + 7) & 7)) >> 3) * 8 +
+                    (((15 - ((e8 + 7) & 7)) >> 2) & 1) * 4);
+}
+template <uint32_t OFF>
+__device__ __forceinline__ void sts_u16_at(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0+%1], %2;" ::"r"(addr), "n"(OFF), "h"((unsigned short)v)
+               : "memory");
+}
+template <int E8>
+struct XTileCols {
+  static __device__ __forceinline__ void run(uint32_t base, const uint32_t (&w)[4]) {
+    sts_u16_at<xtile_col_off(E8)>(base, (w[E8 >> 1] >> (16 * (E8 & 1))) & 0xFFFFu);
+    XTileCols<E8 + 1>::run(base, w);
+  }
+};
+template <>
+struct XTileCols<8> {
+  static __device__ __forceinline__ void run(uint32_t, const uint32_t (&)[4]) {}
+};
+
 // Launch row `warp` of K-block kb's activation tile into slot kb & 1: lane l
 // holds columns 8l .. 8l + 7 (v), each stored at its place in the fragment
-// order (xtile_offset of its tile K position); also the row's group sums.
+// order (xtile_offset of its tile K position, in the closed form above);
+// also the row's group sums.
 __device__ __forceinline__ void store_x_tile(uint32_t sbase, int kb, int warp, int lane,
                                              const uint4& v) {
   const uint32_t slot = (uint32_t)(kb & 1);
   const uint32_t t = sbase + slot * kXTileBytes;
+  const int h = lane >> 4, U = (lane >> 2) & 3, e = (lane >> 1) & 1;
+  const uint32_t base = t + (uint32_t)(((((h * 4 + U) * 2 + (warp >> 3)) * 32 + (warp & 7) * 4) * 16) + e * 2) -
+                        8u * (uint32_t)(lane & 1);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int e8 = 0; e8 < 8; ++e8) {
-    const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(t + xtile_offset(warp, mma_k_position(lane * 8 + e8))),
-                 "h"((unsigned short)half)
-                 : "memory");
-  }
+  XTileCols<0>::run(base, w);
   float f[8];
   unpack8(v, f);
   float s = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));

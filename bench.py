@@ -56,8 +56,10 @@ def algo_bytes(N, K, M, p):
     return N * K * p // 8 + N * G * p * 2 + N * G * 2 + M * K * 2 + M * N * 2
 
 
+# Sources of the kernels the bench step launches (one-row, pair, four-row and
+# mma.sync kernels; the step launches no tcgen05 kernel)
 KERNEL_SOURCES = ("bcq_kernels.cu", "bcq_device.cuh", "bcq_pipeline.cuh", "bcq_mma.cuh",
-                  "bcq_m1.cuh", "bcq_umma.cuh", "bcq_layout.h")
+                  "bcq_m1.cuh", "bcq_layout.h")
 # CUDA kernel of each launch kind bcq_route_query reports
 KERNEL_OF_ROUTE = {"lut_one": "gemv_m1_kernel", "lut_pair": "gemv_lut_kernel<2>",
                    "lut_four": "gemv_lut_kernel<4>", "mma": "gemv_mma_kernel",

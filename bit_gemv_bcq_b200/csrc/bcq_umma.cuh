@@ -138,11 +138,35 @@ __device__ __forceinline__ uint64_t umma_bdesc(uint32_t addr) {
 
 // ------------------------------------------------------- activation tile
 
+// Tile positions of one lane's columns.  Column 8l + e8 of a K-block sits at
+// its permuted K position (see above) j of the canonical layout: row n,
+// position j at (j / 8) * NN * 16 + (n / 8) * 128 + (n % 8) * 16 + (j % 8) * 2.
+// In closed form: with r = (e8 + 7) mod 8 the column's
+// shift is s = (l odd ? 7 : 15) - r, its position j = 2 (64 h + 16 U + s) + e
+// (e = (l / 2) mod 2) and its byte offset in the row's slice
+//   (16 h + 4 U) NN * 16 + 2e - 32 NN (l mod 2) + ((15 - r) / 4) NN * 16 + ((15 - r) mod 4) * 4,
+// a per-lane base plus a compile-time constant per column (checked against
+// the definition above for every row, lane and column).
+template <int NN>
+__host__ __device__ constexpr uint32_t umma_xtile_col_off(int e8) {
+  return (uint32_t)(((15 - ((e8 + 7) & 7)) >> 2) * NN * 16 + ((15 - ((e8 + 7) & 7)) & 3) * 4);
+}
+template <int NN, int E8>
+struct UmmaXTileCols {
+  static __device__ __forceinline__ void run(uint32_t base, const uint32_t (&w)[4]) {
+    sts_u16_at<umma_xtile_col_off<NN>(E8)>(base, (w[E8 >> 1] >> (16 * (E8 & 1))) & 0xFFFFu);
+    UmmaXTileCols<NN, E8 + 1>::run(base, w);
+  }
+};
+template <int NN>
+struct UmmaXTileCols<NN, 8> {
+  static __device__ __forceinline__ void run(uint32_t, const uint32_t (&)[4]) {}
+};
+
 // Launch row n of K-block kb's activation tile into slot kb & 1: lane l
-// holds columns 8l .. 8l + 7 (v, from load_x_tile), stored at their permuted
-// K positions (see above) of the canonical layout: row n, position j at
-// (j / 8) * NN * 16 + (n / 8) * 128 + (n % 8) * 16 + (j % 8) * 2.  Also the
-// row's group sums, and the fence that shows the tile to the MMAs.
+// holds columns 8l .. 8l + 7 (v, from load_x_tile), stored at their
+// positions (above).  Also the row's group sums, and the fence that shows
+// the tile to the MMAs.
 template <int NN>
 __device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int n, int lane,
                                                   const uint4& v) {
@@ -150,20 +174,11 @@ __device__ __forceinline__ void umma_store_x_tile(uint32_t sbase, int kb, int n,
   const uint32_t slot = (uint32_t)(kb & 1);
   const uint32_t tile = sbase + slot * S::kXTileBytes +
                         (uint32_t)((n >> 3) * 128 + (n & 7) * 16);
-  const int h = lane >> 4, U = (lane >> 2) & 3, t0 = 8 * (lane & 3);
+  const int h = lane >> 4, U = (lane >> 2) & 3, e = (lane >> 1) & 1;
+  const uint32_t base = tile + (uint32_t)((16 * h + 4 * U) * NN * 16 + e * 2) -
+                        (uint32_t)(lane & 1) * (32u * NN);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int e8 = 0; e8 < 8; ++e8) {
-    const int t = t0 + e8;                   // column 128 h + 32 U + t
-    const int bt = (t & ~7) | ((t + 7) & 7); // its bit in the natural (rotated-byte) word
-    const int e = bt >> 4;                   // low (bit < 16) or high half
-    const int s = (e ? 31 : 15) - bt;        // the shift that brings that bit to a sign
-    const int j = 2 * (64 * h + 16 * U + s) + e;
-    const uint32_t half = (w[e8 >> 1] >> (16 * (e8 & 1))) & 0xFFFFu;
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(tile + (uint32_t)((j >> 3) * (NN * 16) + (j & 7) * 2)),
-                 "h"((unsigned short)half)
-                 : "memory");
-  }
+  UmmaXTileCols<NN, 0>::run(base, w);
   float f[8];
   unpack8(v, f);
   float sum = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));

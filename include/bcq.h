@@ -246,10 +246,11 @@ int bcq_route_query(int M, int p, const int32_t* p_row, int N, int K, int* out,
  *   1  programmatic dependent launch: a GEMV kernel may be scheduled while the
  *      preceding kernel in its stream finishes; it touches no global memory
  *      before that kernel has completed;
- *   2  as 1, but the kernel may start streaming its planes before the
- *      preceding kernel has completed (x, y, scales and the workspace still
- *      wait).  Only valid when no kernel immediately before it in the stream
- *      writes the planes it reads.
+ *   2  as 1, but the kernel may start streaming its weights (planes, and in
+ *      the one-row kernel also the packed scales and offsets) before the
+ *      preceding kernel has completed (x, y and the workspace still wait).
+ *      Only valid when no kernel immediately before it in the stream writes
+ *      the planes, scales or offsets it reads.
  * Returns BCQ_OK, or BCQ_ERR_UNSUPPORTED for another mode.
  */
 int bcq_set_pdl(int mode);

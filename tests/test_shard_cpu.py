@@ -72,8 +72,10 @@ def _rank(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 3])
 def test_sharded_layer_gathers_the_full_output(world):
     port = _free_port()
-    out = mp.Manager().dict()
-    mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
+        out = dict(out)
     prob = synth.make_problem(300, 512, 2, seed=41, mixed=True)
     ref = oracle.gemm(prob.x, prob.planes, prob.alphas, prob.z, p_row=prob.p_row)
     for r in range(world):

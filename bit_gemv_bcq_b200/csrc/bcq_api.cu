@@ -299,10 +299,13 @@ struct Launch {
 
 // The launches of one call (no device work; bcq_gemm and the queries share
 // it).  Rows of one precision, M >= BCQ_MMA_MIN_ROWS (3): tcgen05 launches
-// of up to 64 rows while at least 32 are left (measured: 64 rows in one
-// launch cost 0.6 of four 16-row launches), a four-row lookup launch for a
-// group of 3-4 rows (measured on 14336 x 4096: p = 2 / 3 / 4 in 17.2 / 23.6 /
-// 26.2 us against 22.9 / 29.6 / 36.6 us on the tensor-core kernel;
+// of up to 64 rows while at least 32 are left, 33 at one or two bits
+// (measured on 14336 x 4096: 64 rows in one launch cost 0.6 of four 16-row
+// launches; exactly 32 rows at p = 2 take 54.5 us as one launch and 46.7 us
+// as two 16-row launches, at p = 4 70.0 against 75.2 us), a four-row
+// lookup launch for a group of 3-4 rows (measured on 14336 x 4096: p = 2 /
+// 3 / 4 in 17.2 / 23.6 / 26.2 us against 22.9 / 29.6 / 36.6 us on the
+// tensor-core kernel;
 // BCQ_LUT4_MAX_ROWS=0 turns it off, BCQ_LUT4_MIN_BITS sets a precision
 // threshold), tensor-core launches of up to 16 rows, lookup launches for a
 // remainder of 1-2 rows.  Rows of several precisions (per-request
@@ -362,7 +365,7 @@ int route_call(int M, int p, const int32_t* p_row, int K, Launch* out) {
       if (qof(m) == q) rows[cnt++] = m;
     for (int r0 = 0; r0 < cnt;) {
       const int left = cnt - r0;
-      if (left >= 2 * kMmaRows) {
+      if (left > 2 * kMmaRows || (left == 2 * kMmaRows && q > 2)) {
         const int c = std::min(kMaxLaunchRows, left);
         add(kPathUmma, rows + r0, c);
         r0 += c;

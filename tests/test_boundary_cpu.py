@@ -249,6 +249,11 @@ def test_uniform_batches_keep_their_kernels(L):
     assert api.route_query(8, 14336, 4096, p=2) == [("mma", 8, 2)]
     assert api.route_query(16, 14336, 4096, p=2) == [("mma", 16, 2)]
     assert api.route_query(64, 14336, 4096, p=2) == [("tcgen05", 64, 2)]
+    # exactly 32 rows: two 16-row launches at one or two bits, one at three or four
+    assert api.route_query(32, 14336, 4096, p=2) == [("mma", 16, 2), ("mma", 16, 2)]
+    assert api.route_query(32, 14336, 4096, p=1) == [("mma", 16, 1), ("mma", 16, 1)]
+    assert api.route_query(32, 14336, 4096, p=4) == [("tcgen05", 32, 4)]
+    assert api.route_query(33, 14336, 4096, p=2) == [("tcgen05", 33, 2)]
     assert api.route_query(17, 14336, 4096, p=2) == [("mma", 16, 2), ("lut_one", 1, 2)]
 
 

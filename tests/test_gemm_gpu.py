@@ -120,11 +120,11 @@ def test_parity_batch_sweep(N, K, path):
 @pytest.mark.parametrize("N,K", [(4096, 4096), (1000, 2048), (14336, 4096)])
 def test_parity_wide_batches(N, K, path):
     """17 to 64 rows of one precision: one tcgen05 launch of up to 64 rows (the
-    lookup kernel in pairs), and mixed precisions that split into groups of
-    more and of fewer than 16 rows."""
+    lookup kernel in pairs; 32 rows at two bits are two 16-row launches), and
+    mixed precisions that split into groups of more and of fewer than 16 rows."""
     prob = synth.make_problem(N, K, 64, seed=4)
     w = _weights(prob)
-    for M in (17, 33, 64):
+    for M in (17, 32, 33, 64):
         sub = synth.Problem(x=prob.x[:M], planes=prob.planes, alphas=prob.alphas, z=prob.z)
         for p in (2, 4):
             y = _run(sub, w, p=p)

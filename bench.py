@@ -48,6 +48,9 @@ N_OUT, K_IN, GROUP, P_H = 14336, 4096, 128, 4
 PRECISIONS = (2, 3, 4)
 BATCHES = (1, 2, 4, 8, 16)
 METRIC = "BCQ GEMV µs & HBM GB/s (% of B200 peak) at p=2/3/4, M=1..16, 14336×4096"
+WORKLOAD = ("bcq_gemv N=14336 K=4096 g=128 p_H=4; one step = one call per p in {2,3,4} x "
+            "M in {1,2,4,8,16} (15 calls), fp16 x/y/scales")
+REF_BUDGET_S = 90.0   # host work of one reference-arm run (warm-up and timed steps)
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -731,6 +734,44 @@ def run_oracle_sample(seed, rows_per_call, prob=None):
     return dt, by, oracle.num_threads()
 
 
+def reference_arm(args):
+    """The oracle as the reference arm: W untimed and exactly K timed steps, each
+    step the 15 calls of the workload on a sample of output rows.  The sample is
+    sized so that the whole run costs about REF_BUDGET_S seconds of host work:
+    a step costs a fixed part (15 oracle calls) plus a part per sampled row,
+    both taken from two calibration samples."""
+    from bit_gemv_bcq_b200 import synth
+    prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
+    t_lo = run_oracle_sample(args.seed, 16, prob)[0]
+    t_hi = run_oracle_sample(args.seed, 256, prob)[0]
+    per_row = max((t_hi - t_lo) / 240, 1e-9)
+    fixed = max(t_lo - 16 * per_row, 0.0)
+    per_step = REF_BUDGET_S / (args.steps + args.warmup)
+    rows = int((per_step - fixed) / per_row) // 16 * 16
+    rows = max(16, min(args.cpu_rows, 2048, rows))
+    for k in range(args.warmup):
+        run_oracle_sample(args.seed + 1 + k, rows, prob)
+    secs, by, thr = 0.0, 0.0, 1
+    for k in range(args.steps):
+        s, b, thr = run_oracle_sample(args.seed + 1 + args.warmup + k, rows, prob)
+        secs += s
+        by += b
+    gbps = by / secs / 1e9
+    return {"metric": METRIC, "value": round(gbps, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "parallelism": "single process, host cores"},
+            "cpu_baseline": {"value": round(gbps, 4), "unit": "GB/s", "cores": thr,
+                             "kind": "oracle",
+                             "sample": f"{rows} of {N_OUT} output rows of each of the 15 calls "
+                                       f"per step, {args.steps} timed steps after "
+                                       f"{args.warmup} untimed"},
+            "e2e": {"value": round(gbps, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -771,30 +812,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        steps = max(1, args.steps)
-        # each step: the oracle on a bounded sample of one step of the workload
-        rows = max(16, min(args.cpu_rows, 2048))
-        from bit_gemv_bcq_b200 import synth
-        prob = synth.make_problem(N_OUT, K_IN, max(BATCHES), seed=args.seed)
-        n_steps = min(steps, 5)
-        secs, by, thr = 0.0, 0.0, 1
-        for k in range(n_steps):
-            s, b, thr = run_oracle_sample(args.seed + k, rows, prob)
-            secs += s
-            by += b
-        gbps = by / secs / 1e9
-        line = {"metric": METRIC, "value": round(gbps, 4), "unit": "GB/s", "n_gpus": args.gpus,
-                "steps": n_steps, "warmup": 0, "ms_per_step": round(secs / n_steps * 1e3, 3),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": "bcq_gemv N=14336 K=4096 g=128 p_H=4; p in {2,3,4} x "
-                                       "M in {1,2,4,8,16}", "parallelism": "single process, host cores"},
-                "cpu_baseline": {"value": round(gbps, 4), "unit": "GB/s", "cores": thr,
-                                 "kind": "oracle",
-                                 "sample": f"{rows} of {N_OUT} output rows of each of the 15 calls per step"},
-                "e2e": {"value": round(gbps, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        print(json.dumps(reference_arm(args)), flush=True)
         return 0
 
     import torch
@@ -824,8 +842,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "bcq_gemv N=14336 K=4096 g=128 p_H=4; one step = one call per "
-                               "p in {2,3,4} x M in {1,2,4,8,16} (15 calls), fp16 x/y/scales",
+        "config": {"workload": WORKLOAD,
                    "l2": f"inputs larger than L2: {res['R']} rotating weight copies of "
                          f"{res['per_copy_bytes'] / 2**20:.1f} MiB",
                    "parallelism": "replicas" if world > 1 else "single GPU",

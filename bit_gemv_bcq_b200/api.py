@@ -13,6 +13,7 @@ zero-filled buffer per (device, stream), grown on demand.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -117,9 +118,22 @@ def _check(status: int, where: str) -> None:
         raise BcqError(status, where)
 
 
-def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+def _stream(stream=None, device=None):
+    """The CUDA stream handle: `stream` (which must belong to `device`), else
+    the current stream of `device` (of the current device when None)."""
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the data on {device}")
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(device):
+    """The C ABI works on the current CUDA device: make `device` current for
+    the call when it is not already."""
+    if device.index is None or device.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(device)
 
 
 def _ptr(t):
@@ -133,6 +147,41 @@ def _need_cuda(t: torch.Tensor, name: str, dtype=None):
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_on(t: torch.Tensor, name: str, device) -> None:
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, x on {device}")
+
+
+def _weights_on(w: "BcqWeights", device) -> None:
+    """Every device array of w on `device` (the kernels take raw pointers)."""
+    _need_on(w.packed, "planes", device)
+    for q, a in w.alphas.items():
+        _need_on(a, f"alpha[{q}]", device)
+    if w.z is not None:
+        _need_on(w.z, "z", device)
+    for q, a in (w.zq or {}).items():
+        _need_on(a, f"z[{q}]", device)
+
+
+def _need_out(out: torch.Tensor | None, M: int, N: int, device) -> torch.Tensor:
+    """The output [M][N] fp16 on `device`: allocated when None, else checked
+    (the kernels write M*N values through its pointer)."""
+    if out is None:
+        return torch.empty((M, N), dtype=torch.float16, device=device)
+    _need_cuda(out, "out", torch.float16)
+    _need_on(out, "out", device)
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be [{M}][{N}], got {list(out.shape)}")
+    return out
+
+
+def _need_x(x: torch.Tensor, K: int) -> int:
+    _need_cuda(x, "x", torch.float16)
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError(f"x must be [M][{K}]")
+    return x.shape[0]
 
 
 def _alpha_array(alphas: dict, what: str = "alpha"):
@@ -162,9 +211,11 @@ def pack_planes(planes_canon: torch.Tensor, stream=None) -> torch.Tensor:
     nbytes = packed_planes_bytes(p_H, N, K)
     if nbytes == 0:
         raise BcqError(BCQ_ERR_SHAPE, "bcq_packed_planes_bytes")
-    out = torch.empty(nbytes // 4, dtype=torch.int32, device=planes_canon.device)
-    _check(lib().bcq_pack_planes(_ptr(planes_canon), _ptr(out), p_H, N, K,
-                                 _stream(stream)), "bcq_pack_planes")
+    dev = planes_canon.device
+    out = torch.empty(nbytes // 4, dtype=torch.int32, device=dev)
+    with _on(dev):
+        _check(lib().bcq_pack_planes(_ptr(planes_canon), _ptr(out), p_H, N, K,
+                                     _stream(stream, dev)), "bcq_pack_planes")
     return out
 
 
@@ -183,9 +234,11 @@ def pack_scales(src: torch.Tensor, q: int, stream=None) -> torch.Tensor:
     nbytes = packed_scales_bytes(q, N, K)
     if nbytes == 0:
         raise BcqError(BCQ_ERR_SHAPE, "bcq_packed_scales_bytes")
-    out = torch.empty(nbytes // 2, dtype=torch.float16, device=src.device)
-    _check(lib().bcq_pack_scales(_ptr(src), int(q), N, K, _ptr(out), _stream(stream)),
-           "bcq_pack_scales")
+    dev = src.device
+    out = torch.empty(nbytes // 2, dtype=torch.float16, device=dev)
+    with _on(dev):
+        _check(lib().bcq_pack_scales(_ptr(src), int(q), N, K, _ptr(out), _stream(stream, dev)),
+               "bcq_pack_scales")
     return out
 
 
@@ -212,14 +265,17 @@ def quantize(w: torch.Tensor, p_L: int = 2, p_H: int = 4, rounds: int = 20,
            if with_sse else None)
     if offsets == "per_precision":
         z = {p: torch.empty((N, G), dtype=torch.float16, device=dev) for p in alphas}
-        _check(lib().bcq_quantize_zp(_ptr(w), N, K, int(p_L), int(p_H), int(rounds),
-                                     _ptr(planes), _alpha_array(alphas), _alpha_array(z, "z"),
-                                     _ptr(sse), _stream(stream)), "bcq_quantize_zp")
+        with _on(dev):
+            _check(lib().bcq_quantize_zp(_ptr(w), N, K, int(p_L), int(p_H), int(rounds),
+                                         _ptr(planes), _alpha_array(alphas),
+                                         _alpha_array(z, "z"), _ptr(sse), _stream(stream, dev)),
+                   "bcq_quantize_zp")
         return planes, alphas, z, sse
     z = torch.empty((N, G), dtype=torch.float16, device=dev)
-    _check(lib().bcq_quantize(_ptr(w), N, K, int(p_L), int(p_H), int(rounds), _ptr(planes),
-                              _alpha_array(alphas), _ptr(z), _ptr(sse), _stream(stream)),
-           "bcq_quantize")
+    with _on(dev):
+        _check(lib().bcq_quantize(_ptr(w), N, K, int(p_L), int(p_H), int(rounds), _ptr(planes),
+                                  _alpha_array(alphas), _ptr(z), _ptr(sse),
+                                  _stream(stream, dev)), "bcq_quantize")
     return planes, alphas, z, sse
 
 
@@ -401,30 +457,27 @@ def _prec_args(p, p_row, M):
 def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
          out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x . W_hat^T (fp16 [M][N]) with uniform precision p or per-row p_row."""
-    _need_cuda(x, "x", torch.float16)
-    if x.dim() != 2 or x.shape[1] != w.K:
-        raise ValueError(f"x must be [M][{w.K}]")
-    M = x.shape[0]
+    M = _need_x(x, w.K)
+    _weights_on(w, x.device)
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
-    if out is None:
-        out = torch.empty((M, w.N), dtype=torch.float16, device=x.device)
-    else:
-        _need_cuda(out, "out", torch.float16)
+    out = _need_out(out, M, w.N, x.device)
     alpha = _alpha_array(w.alphas)
-    ws = workspace(M, w.N, w.K, x.device, stream)
-    if w.zq is not None:
-        zarr = _alpha_array(w.zq, "z")   # 4 device pointers or NULL
-        st = lib().bcq_gemm_zp(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                               ctypes.cast(zarr, ctypes.c_void_p), pv, pr_ptr, M, w.N, w.K,
-                               w.p_H, GROUP, _ptr(out), _ptr(ws),
-                               0 if ws is None else ws.numel(), _stream(stream))
-        _check(st, "bcq_gemm_zp")
-    else:
-        st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                            _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                            _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
-                            _stream(stream))
-        _check(st, "bcq_gemm")
+    dev = x.device
+    sh = _stream(stream, dev)
+    ws = workspace(M, w.N, w.K, dev, stream)
+    with _on(dev):
+        if w.zq is not None:
+            zarr = _alpha_array(w.zq, "z")   # 4 device pointers or NULL
+            st = lib().bcq_gemm_zp(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                                   ctypes.cast(zarr, ctypes.c_void_p), pv, pr_ptr, M, w.N, w.K,
+                                   w.p_H, GROUP, _ptr(out), _ptr(ws),
+                                   0 if ws is None else ws.numel(), sh)
+            _check(st, "bcq_gemm_zp")
+        else:
+            st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                                _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                                _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(), sh)
+            _check(st, "bcq_gemm")
     del pr_keep
     return out
 
@@ -439,19 +492,16 @@ def gemm_noalloc(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=Non
     binding allocates it otherwise)."""
     if w.zq is not None:
         raise ValueError("per-precision offsets: use gemm (bcq_gemm_zp)")
-    _need_cuda(x, "x", torch.float16)
-    if x.dim() != 2 or x.shape[1] != w.K:
-        raise ValueError(f"x must be [M][{w.K}]")
-    M = x.shape[0]
+    M = _need_x(x, w.K)
+    _weights_on(w, x.device)
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
-    if out is None:
-        out = torch.empty((M, w.N), dtype=torch.float16, device=x.device)
-    else:
-        _need_cuda(out, "out", torch.float16)
+    out = _need_out(out, M, w.N, x.device)
     alpha = _alpha_array(w.alphas)
-    st = lib().bcq_gemm_noalloc(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                                _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                                _ptr(out), _stream(stream))
+    sh = _stream(stream, x.device)
+    with _on(x.device):
+        st = lib().bcq_gemm_noalloc(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                                    _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                                    _ptr(out), sh)
     _check(st, "bcq_gemm_noalloc")
     del pr_keep
     return out
@@ -466,14 +516,28 @@ def gemm_host(x_host: torch.Tensor, w: BcqWeights, y_host: torch.Tensor,
         raise ValueError("per-precision offsets: use gemm (bcq_gemm_zp)")
     if x_host.is_cuda or y_host.is_cuda:
         raise ValueError("x_host and y_host must be host tensors")
+    for t, name in ((x_host, "x_host"), (y_host, "y_host")):
+        if t.dtype != torch.float16 or not t.is_contiguous() or t.dim() != 2:
+            raise ValueError(f"{name} must be a contiguous fp16 matrix")
     M = x_host.shape[0]
+    if x_host.shape[1] != w.K or tuple(y_host.shape) != (M, w.N):
+        raise ValueError(f"x_host must be [M][{w.K}] and y_host [M][{w.N}]")
+    for t, name, n in ((x_dev, "x_dev", M * w.K), (y_dev, "y_dev", M * w.N)):
+        _need_cuda(t, name, torch.float16)
+        if t.numel() < n:
+            raise ValueError(f"{name} must hold at least {n} values")
+    dev = x_dev.device
+    _need_on(y_dev, "y_dev", dev)
+    _weights_on(w, dev)
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
     alpha = _alpha_array(w.alphas)
-    ws = workspace(M, w.N, w.K, x_dev.device, stream)
-    st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                             _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                             _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(ws),
-                             0 if ws is None else ws.numel(), _stream(stream))
+    sh = _stream(stream, dev)
+    ws = workspace(M, w.N, w.K, dev, stream)
+    with _on(dev):
+        st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
+                                 _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
+                                 _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(ws),
+                                 0 if ws is None else ws.numel(), sh)
     _check(st, "bcq_gemm_host")
     del pr_keep
 
@@ -485,8 +549,9 @@ def build_lut(x: torch.Tensor, stream=None):
     M, K = x.shape
     lut = torch.empty((M, K // 8, 256), dtype=torch.float32, device=x.device)
     gs = torch.empty((M, K // GROUP), dtype=torch.float32, device=x.device)
-    _check(lib().bcq_build_lut(_ptr(x), M, K, _ptr(lut), _ptr(gs), _stream(stream)),
-           "bcq_build_lut")
+    with _on(x.device):
+        _check(lib().bcq_build_lut(_ptr(x), M, K, _ptr(lut), _ptr(gs), _stream(stream, x.device)),
+               "bcq_build_lut")
     return lut, gs
 
 

@@ -26,7 +26,8 @@
  *   - fp16 data is passed as its IEEE binary16 bit pattern (uint16_t).
  *   - Canonical bit-planes: uint32 [p_H][N][K/32]; bit j of word w of row n is
  *     column 32w + j (LSB first); bit value 1 means +1, 0 means -1.
- *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - `stream` is a cudaStream_t of the current device passed as void* (NULL =
+ *     legacy default stream).
  *     Work is enqueued asynchronously on it; the call returns after the launch.
  *   - Every argument is validated before anything is launched.  A call that
  *     returns an error status has launched nothing and touched no buffer.

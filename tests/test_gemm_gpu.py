@@ -289,6 +289,41 @@ def test_host_buffers_path_matches_device_path():
     assert torch.equal(y_host, y_dev_ref.cpu())
 
 
+def test_binding_rejects_buffers_of_the_wrong_size_before_any_launch():
+    """The kernels write through raw pointers: the binding checks every
+    caller-given buffer's shape before it calls the library."""
+    prob = synth.make_problem(256, 512, 2, seed=12)
+    w = _weights(prob)
+    x = _x(prob)
+    dev = x.device
+    bad_out = [torch.empty((2, 255), dtype=torch.float16, device=dev),
+               torch.empty((1, 256), dtype=torch.float16, device=dev),
+               torch.empty((2, 256), dtype=torch.float32, device=dev)]
+    for out in bad_out:
+        with pytest.raises(ValueError):
+            api.gemm(x, w, p=2, out=out)
+        with pytest.raises(ValueError):
+            api.gemm_noalloc(x, w, p=2, out=out)
+    with pytest.raises(ValueError):
+        api.gemm(x[:, :384].contiguous(), w, p=2)
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((2, 256), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty((2, 512), dtype=torch.float16, device=dev)
+    y_dev = torch.empty((2, 256), dtype=torch.float16, device=dev)
+    for args in [(x_host, torch.empty((2, 255), dtype=torch.float16), x_dev, y_dev),
+                 (x_host, y_host, x_dev[:1], y_dev),
+                 (x_host, y_host, x_dev, y_dev[:1]),
+                 (x_host[:, :256].contiguous(), y_host, x_dev, y_dev)]:
+        with pytest.raises(ValueError):
+            api.gemm_host(args[0], w, args[1], args[2], args[3], p=2)
+    torch.cuda.synchronize()
+    assert api.device_error() == api.BCQ_OK
+    # the right buffers still work
+    api.gemm_host(x_host, w, y_host, x_dev, y_dev, p=2)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, api.gemm(x, w, p=2).cpu())
+
+
 # ------------------------------------------------------------- bounded waits
 
 def test_bounded_wait_reports_timeout_and_context_survives():

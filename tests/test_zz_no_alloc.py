@@ -83,8 +83,14 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     w = api.BcqWeights(packed=dummy, alphas={2: scales}, z=None, N=N, K=K, p_H=2)
     x = torch.zeros((M, K), dtype=torch.float16, device="cuda")
     y = torch.zeros((M, 8), dtype=torch.float16, device="cuda")
-    with pytest.raises(api.BcqError) as e:
+    # the binding refuses the undersized output itself ...
+    with pytest.raises(ValueError):
         api.gemm_noalloc(x, w, p=2, out=y)
-    assert e.value.status == api.BCQ_ERR_SCRATCH
+    # ... and the library, given the same pointers, refuses the shape
+    alpha = api._alpha_array(w.alphas)
+    st = api.lib().bcq_gemm_noalloc(api._ptr(x), api._ptr(dummy),
+                                    api.ctypes.cast(alpha, api.ctypes.c_void_p), None, 2, None,
+                                    M, N, K, 2, 128, api._ptr(y), api._stream())
+    assert st == api.BCQ_ERR_SCRATCH
     torch.cuda.synchronize()
     assert torch.count_nonzero(y).item() == 0

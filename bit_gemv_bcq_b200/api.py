@@ -16,7 +16,7 @@ from __future__ import annotations
 import contextlib
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import numpy as np
 import torch
@@ -137,7 +137,8 @@ def _on(device):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain int: every entry point declares its pointer arguments as void*
+    return None if t is None else t.data_ptr()
 
 
 def _need_cuda(t: torch.Tensor, name: str, dtype=None):
@@ -163,6 +164,27 @@ def _weights_on(w: "BcqWeights", device) -> None:
         _need_on(w.z, "z", device)
     for q, a in (w.zq or {}).items():
         _need_on(a, f"z[{q}]", device)
+
+
+_data_ptr = torch.Tensor.data_ptr
+
+
+def _weight_args(w: "BcqWeights", device):
+    """(alpha, z) pointer arrays of w for the gemm entry points (z: the
+    per-precision offsets, else None), its arrays checked to be on `device`.
+    Kept on w while the signature -- device and every array's address --
+    stays the same, so repeated calls skip the checks and the marshalling."""
+    sig = (device, w.packed.data_ptr(), None if w.z is None else w.z.data_ptr(),
+           tuple(w.alphas), tuple(map(_data_ptr, w.alphas.values())),
+           None if w.zq is None else (tuple(w.zq), tuple(map(_data_ptr, w.zq.values()))))
+    c = w._marshal
+    if c is not None and c[0] == sig:
+        return c[1], c[2]
+    _weights_on(w, device)
+    alpha = _alpha_array(w.alphas)
+    zarr = None if w.zq is None else _alpha_array(w.zq, "z")
+    w._marshal = (sig, alpha, zarr)
+    return alpha, zarr
 
 
 def _need_out(out: torch.Tensor | None, M: int, N: int, device) -> torch.Tensor:
@@ -358,6 +380,8 @@ class BcqWeights:
     p_H: int
     row_splits: tuple = ()      # rows of each stacked matrix (see stack), else ()
     zq: dict | None = None      # {q: packed offsets z^(q)} when every precision has its own
+    # (signature, alpha pointer array, z pointer array) of the last call: see _weight_args
+    _marshal: tuple | None = field(default=None, init=False, repr=False, compare=False)
 
     @classmethod
     def from_canonical(cls, planes, alphas: dict, z=None, device="cuda", stream=None):
@@ -458,25 +482,22 @@ def gemm(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=None,
          out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x . W_hat^T (fp16 [M][N]) with uniform precision p or per-row p_row."""
     M = _need_x(x, w.K)
-    _weights_on(w, x.device)
-    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
-    out = _need_out(out, M, w.N, x.device)
-    alpha = _alpha_array(w.alphas)
     dev = x.device
+    alpha, zarr = _weight_args(w, dev)   # arrays of 4 device pointers or NULL
+    pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
+    out = _need_out(out, M, w.N, dev)
     sh = _stream(stream, dev)
     ws = workspace(M, w.N, w.K, dev, stream)
     with _on(dev):
-        if w.zq is not None:
-            zarr = _alpha_array(w.zq, "z")   # 4 device pointers or NULL
-            st = lib().bcq_gemm_zp(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                                   ctypes.cast(zarr, ctypes.c_void_p), pv, pr_ptr, M, w.N, w.K,
-                                   w.p_H, GROUP, _ptr(out), _ptr(ws),
+        if zarr is not None:
+            st = lib().bcq_gemm_zp(_ptr(x), _ptr(w.packed), alpha, zarr, pv, pr_ptr, M, w.N,
+                                   w.K, w.p_H, GROUP, _ptr(out), _ptr(ws),
                                    0 if ws is None else ws.numel(), sh)
             _check(st, "bcq_gemm_zp")
         else:
-            st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                                _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                                _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(), sh)
+            st = lib().bcq_gemm(_ptr(x), _ptr(w.packed), alpha, _ptr(w.z), pv, pr_ptr, M, w.N,
+                                w.K, w.p_H, GROUP, _ptr(out), _ptr(ws),
+                                0 if ws is None else ws.numel(), sh)
             _check(st, "bcq_gemm")
     del pr_keep
     return out
@@ -493,15 +514,13 @@ def gemm_noalloc(x: torch.Tensor, w: BcqWeights, p: int | None = None, p_row=Non
     if w.zq is not None:
         raise ValueError("per-precision offsets: use gemm (bcq_gemm_zp)")
     M = _need_x(x, w.K)
-    _weights_on(w, x.device)
+    alpha, _ = _weight_args(w, x.device)
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
     out = _need_out(out, M, w.N, x.device)
-    alpha = _alpha_array(w.alphas)
     sh = _stream(stream, x.device)
     with _on(x.device):
-        st = lib().bcq_gemm_noalloc(_ptr(x), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                                    _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                                    _ptr(out), sh)
+        st = lib().bcq_gemm_noalloc(_ptr(x), _ptr(w.packed), alpha, _ptr(w.z), pv, pr_ptr, M,
+                                    w.N, w.K, w.p_H, GROUP, _ptr(out), sh)
     _check(st, "bcq_gemm_noalloc")
     del pr_keep
     return out
@@ -528,16 +547,14 @@ def gemm_host(x_host: torch.Tensor, w: BcqWeights, y_host: torch.Tensor,
             raise ValueError(f"{name} must hold at least {n} values")
     dev = x_dev.device
     _need_on(y_dev, "y_dev", dev)
-    _weights_on(w, dev)
+    alpha, _ = _weight_args(w, dev)
     pv, pr_keep, pr_ptr = _prec_args(p, p_row, M)
-    alpha = _alpha_array(w.alphas)
     sh = _stream(stream, dev)
     ws = workspace(M, w.N, w.K, dev, stream)
     with _on(dev):
-        st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), ctypes.cast(alpha, ctypes.c_void_p),
-                                 _ptr(w.z), pv, pr_ptr, M, w.N, w.K, w.p_H, GROUP,
-                                 _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(ws),
-                                 0 if ws is None else ws.numel(), sh)
+        st = lib().bcq_gemm_host(_ptr(x_host), _ptr(w.packed), alpha, _ptr(w.z), pv, pr_ptr, M,
+                                 w.N, w.K, w.p_H, GROUP, _ptr(y_host), _ptr(x_dev), _ptr(y_dev),
+                                 _ptr(ws), 0 if ws is None else ws.numel(), sh)
     _check(st, "bcq_gemm_host")
     del pr_keep
 

@@ -7,6 +7,7 @@ rank's bytes, over the slowest rank's time).  Here two spawned processes
 take those steps with gloo on CPU tensors; a third check runs the
 reference arm as rank 1 of 2, which must exit 0 without doing any work.
 """
+import json
 import os
 import socket
 
@@ -64,3 +65,30 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
                                      "--steps", "1", "--warmup", "3"])
     assert bench.main() == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch, capsys):
+    """Rank 0 of the reference arm: one JSON line with the main arm's metric,
+    unit, workload and direction, exactly the requested timed and warm-up
+    steps, and the oracle described as the CPU baseline."""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("LOCAL_RANK", "0")
+    monkeypatch.setattr(bench, "REF_BUDGET_S", 0.01)   # the smallest sample: 16 rows
+    monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2",
+                                     "--warmup", "3"])
+    assert bench.main() == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s"
+    assert line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.WORKLOAD
+    assert line["steps"] == 2 and line["warmup"] == 3
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert "16 of 14336 output rows" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
